@@ -1,0 +1,110 @@
+"""Seeded synthetic inputs and the workload table.
+
+This module holds no arithmetic of the method: it only draws random numbers,
+rounds them to the storage precision and names the workloads. The CUDA path
+and the CPU oracle both consume what it returns.
+
+Recipe (per workload): ``numpy.random.default_rng(seed)`` (PCG64), float32
+normal draws in this order: X [B, N, C]; the outlier token indices (when the
+workload has outliers: exactly round(0.05 N) distinct tokens per batch item,
+all channels scaled by 8); then the weights cf3_w, cf1_w, q_w, k_w, v_w,
+kdw_w, vdw_w, each N(0, 1/fan_in) with fan_in = 9C, Cr, C, C, C, 9, 9; for
+MM-EDiT workloads then x_txt [B, N_T, C] and the prompt weights tq_w, tk_w,
+tv_w (fan_in C). Biases are 0, GroupNorm gamma = 1 and beta = 0, unless
+``nonzero_affine`` asks for random ones (drawn last, so the stream above is
+unchanged). bf16 workloads round every array once to bf16
+(round-to-nearest-even) and hand out float32 arrays holding exactly those
+values.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# Workloads shaped like the pages' 512..8192 px text-to-image resolutions.
+WORKLOADS = {
+    "tiny_fp32": dict(dtype="f32", B=1, H=16, W=16, C=64, c_red=16, gn_groups=4,
+                      heads=2, seed=0, outliers=False, n_txt=None),
+    "px512_b2": dict(dtype="bf16", B=2, H=32, W=32, C=1152, c_red=288, gn_groups=32,
+                     heads=16, seed=1, outliers=False, n_txt=None),
+    "px1024": dict(dtype="bf16", B=1, H=64, W=64, C=1152, c_red=288, gn_groups=32,
+                   heads=16, seed=2, outliers=False, n_txt=None),
+    "px2048": dict(dtype="bf16", B=1, H=128, W=128, C=1152, c_red=288, gn_groups=32,
+                   heads=16, seed=2, outliers=False, n_txt=None),
+    "px4096": dict(dtype="bf16", B=1, H=256, W=256, C=1152, c_red=288, gn_groups=32,
+                   heads=16, seed=3, outliers=True, n_txt=None),
+    "px8192": dict(dtype="bf16", B=1, H=512, W=512, C=1152, c_red=288, gn_groups=32,
+                   heads=16, seed=3, outliers=True, n_txt=None),
+    "mm1024": dict(dtype="bf16", B=1, H=64, W=64, C=1536, c_red=384, gn_groups=32,
+                   heads=24, seed=4, outliers=False, n_txt=333),
+}
+
+DECLARED = dict(gn_eps=1e-5, leaky_slope=0.01, attn_eps=1e-6)
+
+
+def round_bf16(a):
+    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).reshape(a.shape)
+
+
+def _normal(rng, shape, var):
+    return rng.standard_normal(shape, dtype=np.float32) * np.float32(np.sqrt(var))
+
+
+def make_inputs(B, H, W, C, c_red, gn_groups, heads, seed, dtype="bf16",
+                outliers=False, n_txt=None, nonzero_affine=False, **_ignored):
+    """Draw one workload. Returns a dict with x (and x_txt) plus every weight
+    under the C header's names and the declared constants; arrays are float32
+    (bf16-exact for bf16 workloads). Shapes: x [B, H*W, C]; cf3_w [Cr, 3, 3, C];
+    cf1_w [C, Cr]; q_w/k_w/v_w [C, C]; kdw_w/vdw_w [C, 3, 3]; biases [out]."""
+    rng = np.random.default_rng(seed)
+    N = H * W
+    x = rng.standard_normal((B, N, C), dtype=np.float32)
+    if outliers:
+        k = int(round(0.05 * N))
+        for b in range(B):
+            idx = rng.choice(N, k, replace=False)
+            x[b, idx, :] *= np.float32(8.0)
+    d = {"x": x}
+    d["cf3_w"] = _normal(rng, (c_red, 3, 3, C), 1.0 / (9 * C))
+    d["cf1_w"] = _normal(rng, (C, c_red), 1.0 / c_red)
+    d["q_w"] = _normal(rng, (C, C), 1.0 / C)
+    d["k_w"] = _normal(rng, (C, C), 1.0 / C)
+    d["v_w"] = _normal(rng, (C, C), 1.0 / C)
+    d["kdw_w"] = _normal(rng, (C, 3, 3), 1.0 / 9)
+    d["vdw_w"] = _normal(rng, (C, 3, 3), 1.0 / 9)
+    if n_txt is not None:
+        d["x_txt"] = rng.standard_normal((B, n_txt, C), dtype=np.float32)
+        d["tq_w"] = _normal(rng, (C, C), 1.0 / C)
+        d["tk_w"] = _normal(rng, (C, C), 1.0 / C)
+        d["tv_w"] = _normal(rng, (C, C), 1.0 / C)
+    zeros = lambda n: np.zeros((n,), dtype=np.float32)  # noqa: E731
+    d["cf3_b"] = zeros(c_red)
+    d["gn_gamma"] = np.ones((c_red,), dtype=np.float32)
+    d["gn_beta"] = zeros(c_red)
+    for name in ("cf1_b", "q_b", "k_b", "v_b", "kdw_b", "vdw_b"):
+        d[name] = zeros(C)
+    if n_txt is not None:
+        for name in ("tq_b", "tk_b", "tv_b"):
+            d[name] = zeros(C)
+    if nonzero_affine:
+        d["cf3_b"] = _normal(rng, (c_red,), 0.01)
+        d["gn_gamma"] = (1.0 + _normal(rng, (c_red,), 0.01)).astype(np.float32)
+        d["gn_beta"] = _normal(rng, (c_red,), 0.01)
+        for name in ("cf1_b", "q_b", "k_b", "v_b", "kdw_b", "vdw_b"):
+            d[name] = _normal(rng, (C,), 0.01)
+        if n_txt is not None:
+            for name in ("tq_b", "tk_b", "tv_b"):
+                d[name] = _normal(rng, (C,), 0.01)
+    if dtype == "bf16":
+        d = {k: round_bf16(v) for k, v in d.items()}
+    d.update(dict(c_red=c_red, gn_groups=gn_groups, **DECLARED))
+    return d
+
+
+def make_workload(name, **overrides):
+    cfg = dict(WORKLOADS[name])
+    cfg.update(overrides)
+    return cfg, make_inputs(**cfg)
