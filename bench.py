@@ -1,0 +1,371 @@
+"""Throughput of one EDiT linear compressed attention layer on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload px4096] [--impl ours|reference]
+
+A step is one full layer forward (every kernel of the path) over one image
+of the workload. `value` is tokens/s over all ranks (each rank runs its own
+image: weak scaling, no collective on the data path), timed on the device
+with CUDA events on the launching stream, L2 flushed between steps. `e2e`
+is the same metric with the input copied from pinned host memory and the
+output copied back inside the timed region. `--impl reference` times the
+fp64 CPU oracle on bounded crops of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_compressed_attention_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+# Stage boundaries recorded by the library's timing hook (include/edit_attn.h).
+STAGES = ["kv_linear", "dwconv_s2", "kv_state", "fold_weights", "conv3x3", "groupnorm", "q_linear", "apply"]
+DOMINANT = "conv3x3"   # largest FLOP share of the layer (40%)
+
+# DRAM traffic of the dominant kernel from an ncu capture (profiles/), valid
+# only while the kernel sources are unchanged (hash of tc_gemm.cuh + common.cuh).
+TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
+
+
+def kernel_src_sha():
+    h = hashlib.sha256()
+    for f in ("tc_gemm.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "linear_compressed_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def layer_flops(cfg):
+    """Algorithmic FLOPs of one layer (2 per multiply-add), per step kind."""
+    B, N, C, Cr = cfg["B"], cfg["H"] * cfg["W"], cfg["C"], cfg["c_red"]
+    M = ((cfg["H"] + 1) // 2) * ((cfg["W"] + 1) // 2)
+    d = C // cfg["heads"]
+    f = {
+        "conv3x3": 2.0 * B * N * Cr * 9 * C,
+        "conv1x1": 2.0 * B * N * C * Cr,
+        "q_linear": 2.0 * B * N * C * C,
+        "kv_linear": 4.0 * B * N * C * C,
+        "dwconv": 2.0 * 9 * B * M * 2 * C,
+        "kv_state": 2.0 * B * M * C * (d + 1),
+        "apply": 2.0 * B * N * C * (d + 1),
+    }
+    f["total"] = sum(f.values())
+    return f
+
+
+def min_bytes(cfg, es=2):
+    B, N, C = cfg["B"], cfg["H"] * cfg["W"], cfg["C"]
+    Cr = cfg["c_red"]
+    weights = (9 * C * Cr + Cr * C + 3 * C * C + 18 * C) * es
+    return 2 * B * N * C * es + weights
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_id)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return 1
+
+
+def oracle_rate(cfg, side, reps=1):
+    """tokens/s of the fp64 oracle on a side x side crop of the workload."""
+    import oracle.edit_oracle as O
+    sub = dict(cfg, B=1, H=min(side, cfg["H"]), W=min(side, cfg["W"]))
+    d = make_inputs(**sub)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+    dt = time.perf_counter() - t0
+    return reps * sub["H"] * sub["W"] / dt, dt, sub
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    side = 16
+    rate, dt, sub = oracle_rate(cfg, side)
+    # grow the crop until one call takes a good part of the budget
+    while dt < budget_s / 4 and side < min(cfg["H"], cfg["W"]):
+        side *= 2
+        rate, dt, sub = oracle_rate(cfg, side)
+    reps = max(1, int(budget_s / 2 / max(dt, 1e-3)))
+    rate, dt, sub = oracle_rate(cfg, side, reps)
+    return {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, {reps} call(s) on a {sub['H']}x{sub['W']}-token crop of the "
+                      f"workload (C={cfg['C']}, {cfg['heads']} heads, same distributions), {dt:.1f} s; "
+                      "its cost per token does not depend on the grid size"}
+
+
+# ------------------------------------------------------------------ arms
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, cfg):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import oracle.edit_oracle as O
+    # size each step so that warm-up + steps fit in about two minutes
+    r16, _, _ = oracle_rate(cfg, 16)
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    side = 2
+    while side < min(cfg["H"], cfg["W"]) and (2 * side) ** 2 / r16 <= per_step:
+        side *= 2
+    sub = dict(cfg, B=1, H=min(side, cfg["H"]), W=min(side, cfg["W"]))
+    d = make_inputs(**sub)
+    for _ in range(args.warmup):
+        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+    dt = time.perf_counter() - t0
+    tok = sub["H"] * sub["W"] * args.steps
+    value = tok / dt
+    line = {
+        "impl": "reference", "metric": args.metric, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload_desc, "sample": f"{sub['H']}x{sub['W']}-token crop per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"fp64 numpy oracle, one {sub['H']}x{sub['W']}-token crop of the workload per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    from linear_compressed_attention_b200 import binding as bd
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+    N = H * W
+    d = make_inputs(**cfg)
+    layer = bd.EditAttention(d, B, H, W, C, heads, cfg["dtype"], device=dev)
+    x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
+    out = torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    nst = bd.STAGE_EVENTS_EDIT
+    def new_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
+        for e in evs:
+            e.record(stream)      # materialise the handle
+        return evs
+
+    for _ in range(args.warmup):
+        layer.forward(x, out)
+    torch.cuda.synchronize(dev)
+    assert layer.status() == 0, "device-side status after warm-up"
+
+    per_step_events = [new_events() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    gpu_id = local
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = bd.edit_attn_kernel_launches()
+    for s in range(args.steps):
+        flush.zero_()                                    # L2 flush, outside the step's events
+        evs = per_step_events[s]
+        bd.edit_attn_set_stage_events([e.cuda_event for e in evs])
+        layer.forward(x, out)
+        bd.edit_attn_set_stage_events(None)
+    torch.cuda.synchronize(dev)
+    launches = bd.edit_attn_kernel_launches() - launches0
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    assert layer.status() == 0, "device-side status after timing"
+
+    step_ms = [evs[0].elapsed_time(evs[-1]) for evs in per_step_events]
+    stage_ms = {name: [evs[i].elapsed_time(evs[i + 1]) for evs in per_step_events] for i, name in enumerate(STAGES)}
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    tokens = world * B * N * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    # e2e: pinned host input -> device -> layer -> pinned host output
+    xh = torch.from_numpy(d["x"]).to(layer.tdtype).pin_memory()
+    oh = torch.empty(xh.shape, dtype=layer.tdtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        x.copy_(xh, non_blocking=True)
+        layer.forward(x, out)
+        oh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(xh, non_blocking=True)
+        layer.forward(x, out)
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    e2e_value = world * B * N * e2e_steps / (e2e_ms / 1e3)
+    nbytes = xh.numel() * xh.element_size()
+
+    if rank == 0:
+        peaks = load_peaks()
+        fl = layer_flops(cfg)
+        dom_ms = statistics.mean(stage_ms[DOMINANT])
+        achieved = fl["conv3x3"] / (dom_ms / 1e3) / 1e12
+        traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["src_sha"] == kernel_src_sha() else None
+        ms_per_step = total_ms / args.steps
+        roof_t = max(fl["total"] / (peaks["bf16_tflops"] * 1e12), min_bytes(cfg) / (peaks["hbm_gbs"] * 1e9))
+        line = {
+            "metric": args.metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if cfg["dtype"] == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": args.workload_desc, "global_batch": world * B, "seq_len": N,
+                       "parallelism": f"independent images, {world} rank(s)",
+                       "l2": "flushed between steps (256 MB write, outside the timed events); input 151 MB > L2"},
+            "roofline": {"bound": "tensor", "kernel": "tc_gemm conv3x3 implicit GEMM", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                         "peak_source": f"{peaks['source']} bf16 burst", "launch_ms": dom_ms},
+            "layer_roofline": {"ms": roof_t * 1e3, "frac": roof_t * 1e3 / ms_per_step,
+                               "note": "max(layer FLOPs / bf16 peak, minimum bytes / HBM) over measured step time"},
+            "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                    "d2h_bytes_per_step": nbytes},
+            "gpu_launches": launches,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="px4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = dict(WORKLOADS[args.workload])
+    if cfg.get("n_txt"):
+        raise SystemExit("bench.py times the EDiT layer workloads; MM-EDiT is covered by the tests")
+    args.metric = "EDiT attention-layer tokens/sec (bf16, B=1) at 4K/16K/64K tokens; % roofline"
+    M = ((cfg["H"] + 1) // 2) * ((cfg["W"] + 1) // 2)
+    args.workload_desc = (f"{args.workload}: EDiT layer, B={cfg['B']}, {cfg['H']}x{cfg['W']} grid "
+                          f"(N={cfg['H'] * cfg['W']}, M={M}), C={cfg['C']}, c_red={cfg['c_red']}, "
+                          f"{cfg['heads']} heads x {cfg['C'] // cfg['heads']}, GN {cfg['gn_groups']} groups, "
+                          f"{cfg['dtype']}" + (", 5% outlier tokens x8" if cfg["outliers"] else ""))
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/*
+ * edit_attn.h -- C ABI of the B200 (sm_100a) EDiT linear compressed attention
+ * library (libedit_attn.so).
+ *
+ * What it computes. The paper-notes page "EDiT: Efficient Diffusion
+ * Transformers with Linear Compressed Attention" (ICCV 2025, arXiv
+ * 2503.16726), section "Method in detail", defines one attention layer:
+ *   - ConvFusion query, eq. (Q^EDiT):
+ *       Q = ReLU(Linear_Q(X + Conv1x1(LeakyReLU(GN(Conv3x3(X))))))
+ *     on the token sequence viewed as its H x W grid; the 3x3 conv compresses
+ *     C -> c_red channels, the 1x1 conv restores c_red -> C.
+ *   - Spatial Compressor, eq. (phi_SC): K = ReLU(DW(Linear_K(X))),
+ *     V = DW(Linear_V(X)), DW a 3x3 depthwise conv of stride 2 (padding 1),
+ *     leaving M = ceil(H/2) * ceil(W/2) key/value tokens.
+ *   - Linear attention per head, eq. (y_i):
+ *       y_i = (Q_i S) / (Q_i z + attn_eps),  S = sum_j K_j^T V_j,  z = sum_j K_j
+ *     with heads = contiguous blocks of d = C/heads channels, no 1/sqrt(d)
+ *     and no output projection.
+ * Section "MM-EDiT", eq. (A^Hybrid), mixes it with softmax attention for
+ * every interaction with prompt tokens, with eta = N_I / (N_I + N_T):
+ *   out_img = eta * y + (1 - eta) * A(Q_I, K_P, V_P)
+ *   out_txt = eta * A(Q_P, K_I, V_I) + (1 - eta) * A(Q_P, K_P, V_P)
+ * where A(q,k,v) = softmax(q k^T / sqrt(d)) v per head, Q_I/K_I/V_I are the
+ * EDiT query and compressed keys/values above, and Q_P/K_P/V_P are plain
+ * Linear projections of the prompt tokens.
+ *
+ * Conventions for every entry point below.
+ *   Layout:  x, out: [B, H*W, C], token n = h*W + w, channels innermost.
+ *            x_txt, out_txt: [B, N_T, C].
+ *   dtype:   x, out and every weight/bias share one dtype (EDIT_F32 or
+ *            EDIT_BF16); all accumulation is fp32.
+ *   Memory:  every pointer except the weights struct itself is DEVICE memory,
+ *            owned by the caller, 16-byte aligned. The library never
+ *            allocates, frees or synchronises (except edit_attn_read_status).
+ *            Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *            default stream). Outputs must not alias inputs or the workspace.
+ *   Workspace: caller-allocated device buffer of at least the size returned by
+ *            the matching *_workspace_bytes query, 256-byte aligned. Distinct
+ *            concurrent calls need distinct workspaces.
+ *   Errors:  the return value is 0 (EDIT_OK) or a negative EDIT_ERR_* code.
+ *            Arguments are validated on the host before any launch; on a
+ *            validation error nothing is enqueued. Device-side problems (a
+ *            bounded wait that ran out) are recorded in the workspace status
+ *            word and read back with edit_attn_read_status. Kernel faults
+ *            surface at the caller's next synchronisation. Nothing traps.
+ */
+#ifndef EDIT_ATTN_H_
+#define EDIT_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EDIT_API __attribute__((visibility("default")))
+#else
+#define EDIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { EDIT_F32 = 0, EDIT_BF16 = 1 } edit_dtype;
+
+enum {
+  EDIT_OK = 0,
+  EDIT_ERR_NULL = -1,      /* a required pointer is NULL                          */
+  EDIT_ERR_SHAPE = -2,     /* B, H, W < 1; C % heads; c_red % gn_groups; N_T < 0 ...*/
+  EDIT_ERR_ALIGN = -3,     /* pointer not 16-byte aligned (workspace: 256-byte)    */
+  EDIT_ERR_DTYPE = -4,     /* unsupported dtype                                    */
+  EDIT_ERR_WORKSPACE = -5, /* workspace smaller than the query returned            */
+  EDIT_ERR_CUDA = -6,      /* a CUDA runtime/driver call or launch failed          */
+  EDIT_ERR_TIMEOUT = -7,   /* (device) a bounded wait ran out; results invalid     */
+  EDIT_ERR_UNSUPPORTED = -8 /* shape outside what the kernels are built for        */
+};
+
+/* Weights and declared constants of one EDiT layer. Shapes (row-major):
+ *   cf3_w [c_red][3][3][C]  3x3 conv C->c_red (torch [c_red,C,3,3] permuted to
+ *                           channels-last: tap (kh,kw) reads pixel (h+kh-1, w+kw-1))
+ *   cf3_b [c_red]           gn_gamma, gn_beta [c_red]
+ *   cf1_w [C][c_red]        1x1 conv c_red->C; cf1_b [C]
+ *   q_w, k_w, v_w [C][C]    Linear, torch [out][in] layout; q_b, k_b, v_b [C]
+ *   kdw_w, vdw_w [C][3][3]  depthwise stride-2 conv taps; kdw_b, vdw_b [C]
+ * Constants: gn_eps (GroupNorm, biased variance), leaky_slope, attn_eps (added
+ * to the linear-attention denominator). None is defaulted by the library. */
+typedef struct {
+  int dtype; /* edit_dtype */
+  int c_red;
+  int gn_groups;
+  float gn_eps;
+  float leaky_slope;
+  float attn_eps;
+  const void *cf3_w, *cf3_b;
+  const void *gn_gamma, *gn_beta;
+  const void *cf1_w, *cf1_b;
+  const void *q_w, *q_b;
+  const void *k_w, *k_b;
+  const void *v_w, *v_b;
+  const void *kdw_w, *kdw_b;
+  const void *vdw_w, *vdw_b;
+  void *workspace; /* device, 256-byte aligned, >= edit_attn_workspace_bytes() */
+  size_t workspace_bytes;
+} edit_attn_weights;
+
+/* Bytes of workspace edit_attn_forward needs for this shape (0 on a shape or
+ * dtype error). Host-only; no CUDA call. */
+EDIT_API size_t edit_attn_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights *w);
+
+/* One EDiT attention layer: out[B, H*W, C] from x[B, H*W, C] (equations
+ * above). Enqueues all kernels on `stream` and returns without waiting. */
+EDIT_API int edit_attn_forward(const void *x, int B, int H, int W, int C, int heads, const edit_attn_weights *w,
+                      void *out, void *stream);
+
+/* Weights of the MM-EDiT hybrid: the EDiT image-stream weights (`img`, its
+ * dtype field is the dtype of everything) plus the prompt-token projections
+ * tq_w, tk_w, tv_w [C][C] (torch Linear layout) and their biases [C]. The
+ * workspace fields of `img` are ignored; the ones here are used. */
+typedef struct {
+  edit_attn_weights img;
+  const void *tq_w, *tq_b;
+  const void *tk_w, *tk_b;
+  const void *tv_w, *tv_b;
+  void *workspace;
+  size_t workspace_bytes;
+} mmedit_weights;
+
+EDIT_API size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights *w);
+
+/* MM-EDiT hybrid attention (section "MM-EDiT", eq. (A^Hybrid)):
+ * out_img[B, H*W, C] and out_txt[B, N_T, C] from x_img[B, H*W, C] and
+ * x_txt[B, N_T, C]. N_T may be 0 (then eta = 1 and out_img is the EDiT
+ * layer; x_txt/out_txt may be NULL). */
+EDIT_API int mmedit_hybrid_forward(const void *x_img, const void *x_txt, int B, int H, int W, int N_T, int C, int heads,
+                          const mmedit_weights *w, void *out_img, void *out_txt, void *stream);
+
+/* Copy the device status word of a workspace to *status (0 = no device-side
+ * error since the last forward call on it) and synchronise `stream`. This is
+ * the only call that waits. */
+EDIT_API int edit_attn_read_status(const void *workspace, void *stream, int *status);
+
+/* Text for a status code (static storage). */
+EDIT_API const char *edit_status_string(int status);
+
+/* Byte offsets of the intermediates kept in an edit_attn_forward workspace,
+ * for inspection after the call completes (-1 when absent). Each tensor is
+ * stored in the call's dtype unless noted:
+ *   U [B,H,W,c_red]; G = LeakyReLU(GN(U)) [B,H*W,c_red]; Q [B,H*W,C];
+ *   KVp [B,H*W,2C] (Linear_K(X) | Linear_V(X) per token); K, V [B,M,C];
+ *   gn_stats fp32 [B][gn_groups][2] (mean, rstd);
+ *   Sz fp32 [B][heads][d][d+1] (S_h with z_h as the last column). */
+typedef struct {
+  int64_t status, U, G, Q, KVp, K, V, gn_stats, Sz;
+} edit_ws_layout;
+
+EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
+                               edit_ws_layout *layout);
+
+/* Measurement hooks (no counterpart on the page; used by the benchmark).
+ *
+ * edit_attn_set_stage_events: when `events` is non-NULL, the next forward
+ * calls made by this host thread record events[i] (cudaEvent_t handles
+ * created by the caller) on the call's stream at stage boundary i:
+ *   0 start, 1 K|V Linear GEMM, 2 depthwise conv, 3 KV state,
+ *   4 weight folding, 5 3x3 conv GEMM, 6 GroupNorm, 7 query GEMM,
+ *   8 apply GEMM; MM-EDiT adds 9 prompt projections, 10 image-row softmax
+ *   attention, 11 prompt-row softmax attention.
+ * `n` is the number of handles (events beyond n are not recorded). NULL
+ * clears the hook. Returns EDIT_OK or EDIT_ERR_SHAPE for n < 0.
+ *
+ * edit_attn_kernel_launches: number of kernels this host thread's forward
+ * calls have enqueued since the library was loaded. */
+enum { EDIT_STAGE_EVENTS_EDIT = 9, EDIT_STAGE_EVENTS_MM = 12 };
+
+EDIT_API int edit_attn_set_stage_events(void *const *events, int n);
+
+EDIT_API uint64_t edit_attn_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EDIT_ATTN_H_ */

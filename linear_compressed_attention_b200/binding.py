@@ -1,0 +1,247 @@
+"""ctypes binding of libedit_attn.so (include/edit_attn.h).
+
+Argument marshalling only: torch tensors are passed as device pointers, the
+stream as the current torch stream handle. Every step of the layer runs in the
+library's CUDA kernels; there is no fallback. Loading raises if the library
+has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libedit_attn.so")
+
+EDIT_F32, EDIT_BF16 = 0, 1
+WEIGHT_NAMES = ("cf3_w", "cf3_b", "gn_gamma", "gn_beta", "cf1_w", "cf1_b", "q_w", "q_b", "k_w", "k_b",
+                "v_w", "v_b", "kdw_w", "kdw_b", "vdw_w", "vdw_b")
+TEXT_NAMES = ("tq_w", "tq_b", "tk_w", "tk_b", "tv_w", "tv_b")
+EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_bytes", "mmedit_hybrid_forward",
+           "edit_attn_read_status", "edit_status_string", "edit_attn_workspace_layout",
+           "edit_attn_set_stage_events", "edit_attn_kernel_launches")
+STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
+
+
+class EditAttnWeights(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("c_red", ctypes.c_int), ("gn_groups", ctypes.c_int),
+                ("gn_eps", ctypes.c_float), ("leaky_slope", ctypes.c_float), ("attn_eps", ctypes.c_float)] + \
+               [(n, ctypes.c_void_p) for n in WEIGHT_NAMES] + \
+               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class MMEditWeights(ctypes.Structure):
+    _fields_ = [("img", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in TEXT_NAMES] + \
+               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("status", "U", "G", "Q", "KVp", "K", "V", "gn_stats", "Sz")]
+
+
+_lib = None
+
+
+def lib():
+    """Load the shared library (raises RuntimeError if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                           "(python -m linear_compressed_attention_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    i, p, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    W, MW = ctypes.POINTER(EditAttnWeights), ctypes.POINTER(MMEditWeights)
+    L.edit_attn_workspace_bytes.argtypes = [i, i, i, i, i, W]
+    L.edit_attn_workspace_bytes.restype = sz
+    L.edit_attn_forward.argtypes = [p, i, i, i, i, i, W, p, p]
+    L.edit_attn_forward.restype = i
+    L.mmedit_workspace_bytes.argtypes = [i, i, i, i, i, i, MW]
+    L.mmedit_workspace_bytes.restype = sz
+    L.mmedit_hybrid_forward.argtypes = [p, p, i, i, i, i, i, i, MW, p, p, p]
+    L.mmedit_hybrid_forward.restype = i
+    L.edit_attn_read_status.argtypes = [p, p, ctypes.POINTER(ctypes.c_int)]
+    L.edit_attn_read_status.restype = i
+    L.edit_status_string.argtypes = [i]
+    L.edit_status_string.restype = ctypes.c_char_p
+    L.edit_attn_workspace_layout.argtypes = [i, i, i, i, i, W, ctypes.POINTER(WsLayout)]
+    L.edit_attn_workspace_layout.restype = i
+    L.edit_attn_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
+    L.edit_attn_set_stage_events.restype = i
+    L.edit_attn_kernel_launches.argtypes = []
+    L.edit_attn_kernel_launches.restype = ctypes.c_uint64
+    _lib = L
+    return L
+
+
+class EditError(RuntimeError):
+    def __init__(self, code):
+        self.code = code
+        super().__init__(f"edit_attn error {code}: {status_string(code)}")
+
+
+def status_string(code: int) -> str:
+    return lib().edit_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_weights_struct(w: dict, dtype_code: int, c_red: int, gn_groups: int, gn_eps: float, leaky_slope: float,
+                        attn_eps: float, workspace=None) -> EditAttnWeights:
+    """Fill the C struct from a dict of device tensors named as in the header."""
+    s = EditAttnWeights()
+    s.dtype = dtype_code
+    s.c_red, s.gn_groups = int(c_red), int(gn_groups)
+    s.gn_eps, s.leaky_slope, s.attn_eps = float(gn_eps), float(leaky_slope), float(attn_eps)
+    for n in WEIGHT_NAMES:
+        t = w.get(n)
+        setattr(s, n, None if t is None else t.data_ptr())
+    if workspace is not None:
+        s.workspace = workspace.data_ptr()
+        s.workspace_bytes = workspace.numel() * workspace.element_size()
+    return s
+
+
+def make_mm_struct(img: EditAttnWeights, w: dict, workspace=None) -> MMEditWeights:
+    s = MMEditWeights()
+    s.img = img
+    for n in TEXT_NAMES:
+        t = w.get(n)
+        setattr(s, n, None if t is None else t.data_ptr())
+    if workspace is not None:
+        s.workspace = workspace.data_ptr()
+        s.workspace_bytes = workspace.numel() * workspace.element_size()
+    return s
+
+
+# ----------------------------------------------------------- C-ABI mirrors
+def edit_attn_workspace_bytes(B, H, W, C, heads, weights: EditAttnWeights) -> int:
+    return int(lib().edit_attn_workspace_bytes(B, H, W, C, heads, ctypes.byref(weights)))
+
+
+def edit_attn_forward(x, B, H, W, C, heads, weights: EditAttnWeights, out, stream=None) -> int:
+    """x, out: device tensors [B, H*W, C]; returns the status code (0 = OK)."""
+    return int(lib().edit_attn_forward(_ptr(x), B, H, W, C, heads, ctypes.byref(weights), _ptr(out),
+                                       _stream(stream)))
+
+
+def mmedit_workspace_bytes(B, H, W, N_T, C, heads, weights: MMEditWeights) -> int:
+    return int(lib().mmedit_workspace_bytes(B, H, W, N_T, C, heads, ctypes.byref(weights)))
+
+
+def mmedit_hybrid_forward(x_img, x_txt, B, H, W, N_T, C, heads, weights: MMEditWeights, out_img, out_txt,
+                          stream=None) -> int:
+    return int(lib().mmedit_hybrid_forward(_ptr(x_img), _ptr(x_txt), B, H, W, N_T, C, heads,
+                                           ctypes.byref(weights), _ptr(out_img), _ptr(out_txt), _stream(stream)))
+
+
+def edit_attn_read_status(workspace, stream=None) -> int:
+    st = ctypes.c_int(0)
+    rc = lib().edit_attn_read_status(_ptr(workspace), _stream(stream), ctypes.byref(st))
+    if rc != 0:
+        raise EditError(rc)
+    return int(st.value)
+
+
+def edit_attn_workspace_layout(B, H, W, C, heads, weights: EditAttnWeights) -> dict:
+    lay = WsLayout()
+    rc = lib().edit_attn_workspace_layout(B, H, W, C, heads, ctypes.byref(weights), ctypes.byref(lay))
+    if rc != 0:
+        raise EditError(rc)
+    return {n: int(getattr(lay, n)) for n, _ in WsLayout._fields_}
+
+
+_stage_keepalive = None
+
+
+def edit_attn_set_stage_events(handles) -> int:
+    """handles: list of raw cudaEvent_t values (ints), or None to clear."""
+    global _stage_keepalive
+    if handles is None:
+        _stage_keepalive = None
+        return int(lib().edit_attn_set_stage_events(None, 0))
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _stage_keepalive = arr
+    return int(lib().edit_attn_set_stage_events(arr, len(handles)))
+
+
+def edit_attn_kernel_launches() -> int:
+    return int(lib().edit_attn_kernel_launches())
+
+
+# ----------------------------------------------------------- convenience
+class EditAttention:
+    """One EDiT (or MM-EDiT) layer with weights and workspace on a CUDA device.
+
+    ``arrays`` is the dict the synthetic-input generator returns (numpy
+    float32, bf16-exact for bf16); tensors are copied to the device once.
+    """
+
+    def __init__(self, arrays: dict, B: int, H: int, W: int, C: int, heads: int, dtype: str = "bf16",
+                 n_txt: int = 0, mm: bool | None = None, device="cuda"):
+        import torch
+        self.torch = torch
+        self.B, self.H, self.W, self.C, self.heads, self.n_txt = B, H, W, C, heads, int(n_txt or 0)
+        self.mm = bool(self.n_txt) if mm is None else bool(mm)
+        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.code = EDIT_BF16 if dtype == "bf16" else EDIT_F32
+        names = WEIGHT_NAMES + (TEXT_NAMES if self.mm else ())
+        self.w = {n: torch.from_numpy(np.ascontiguousarray(arrays[n])).to(device=device, dtype=self.tdtype)
+                  for n in names}
+        self.consts = dict(c_red=arrays["c_red"], gn_groups=arrays["gn_groups"], gn_eps=arrays["gn_eps"],
+                           leaky_slope=arrays["leaky_slope"], attn_eps=arrays["attn_eps"])
+        s = make_weights_struct(self.w, self.code, **self.consts)
+        if self.mm:
+            m = make_mm_struct(s, self.w)
+            nbytes = mmedit_workspace_bytes(B, H, W, self.n_txt, C, heads, m)
+        else:
+            nbytes = edit_attn_workspace_bytes(B, H, W, C, heads, s)
+        if nbytes == 0:
+            raise ValueError("shape/dtype rejected by edit_attn_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.struct = make_weights_struct(self.w, self.code, workspace=self.workspace, **self.consts)
+        self.mm_struct = make_mm_struct(self.struct, self.w, self.workspace) if self.mm else None
+        self.layout = edit_attn_workspace_layout(B, H, W, C, heads, self.struct)
+
+    def forward(self, x, out=None, stream=None):
+        if out is None:
+            out = self.torch.empty_like(x)
+        rc = edit_attn_forward(x, self.B, self.H, self.W, self.C, self.heads, self.struct, out, stream)
+        if rc != 0:
+            raise EditError(rc)
+        return out
+
+    def forward_mm(self, x_img, x_txt, out_img=None, out_txt=None, stream=None):
+        if out_img is None:
+            out_img = self.torch.empty_like(x_img)
+        if out_txt is None and x_txt is not None:
+            out_txt = self.torch.empty_like(x_txt)
+        rc = mmedit_hybrid_forward(x_img, x_txt, self.B, self.H, self.W, self.n_txt, self.C, self.heads,
+                                   self.mm_struct, out_img, out_txt, stream)
+        if rc != 0:
+            raise EditError(rc)
+        return out_img, out_txt
+
+    def status(self, stream=None) -> int:
+        return edit_attn_read_status(self.workspace, stream)
+
+    def intermediate(self, name: str, shape, dtype=None):
+        """View of an intermediate kept in the workspace (valid after the call completes)."""
+        torch = self.torch
+        off = self.layout[name]
+        dt = dtype or self.tdtype
+        n = int(np.prod(shape))
+        es = torch.empty((), dtype=dt).element_size()
+        return self.workspace[off:off + n * es].view(dt).view(*shape)

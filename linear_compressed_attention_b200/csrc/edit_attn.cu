@@ -1,0 +1,781 @@
+// C ABI of the EDiT linear compressed attention library (include/edit_attn.h):
+// argument validation, the workspace plan, TMA tensor-map encoding and the
+// launch sequence of one EDiT layer / one MM-EDiT hybrid layer.
+//
+// Step order of one EDiT layer (bf16; fp32 uses the CUDA-core GEMM instead of
+// the tensor-core one):
+//   1. KVp = X [Wk; Wv]^T + [bk; bv]                      tensor-core GEMM
+//   2. K = ReLU(DW_k(Kp)), V = DW_v(Vp)                    depthwise stride 2
+//   3. [S_h | z_h] = sum_j K_jh^T [V_jh | 1]               split + fixed-order combine
+//   4. Wqw1 = Wq W1, bq' = Wq b1 + bq                      weight folding (see below)
+//   5. U = Conv3x3(X) (+ GroupNorm partial sums)           implicit-GEMM on tensor cores
+//   6. G = LeakyReLU(GN(U))                                fixed-order stats, elementwise
+//   7. Q = ReLU([X | G] [Wq | Wqw1]^T + bq')               tensor-core GEMM, K = C + Cr
+//   8. y = (Q_h S_h) / (Q_h z_h + eps)                     tensor-core GEMM per head
+// Step 4/7: the 1x1 conv of eq. (Q^EDiT) feeds only Linear_Q, so
+// Linear_Q(X + Conv1x1(G)) = X Wq^T + G (Wq W1)^T + (Wq b1 + bq): the same
+// FLOPs as the two GEMMs in a row, without writing and re-reading R.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "simt_kernels.cuh"
+#include "tc_gemm.cuh"
+
+using namespace edit;
+
+namespace {
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+            const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A operand: [imgs][rows][K] bf16, row stride ld elements, box 64 x 128 x 1.
+bool map_a(CUtensorMap* m, const void* base, long K, long rows, long imgs, long ld, long img_stride) {
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)imgs};
+  cuuint64_t st[2] = {(cuuint64_t)ld * 2, (cuuint64_t)img_stride * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  return encode(m, 3, base, dims, st, box);
+}
+
+// B operand: [rows][K] bf16, row stride ld elements, box 64 x box_rows.
+bool map_b(CUtensorMap* m, const void* base, long K, long rows, long ld, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t st[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  return encode(m, 2, base, dims, st, box);
+}
+
+// Conv input grid [B][H][W][C] bf16, box 64 x TW x TH x 1.
+bool map_grid(CUtensorMap* m, const void* base, int B, int H, int W, int C, int TW, int TH) {
+  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t st[3] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)TW, (cuuint32_t)TH, 1};
+  return encode(m, 4, base, dims, st, box);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------------ plan
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Plan {
+  // geometry
+  int B, H, W, C, heads, Cr, G, d, Ho, Wo, M, NT;
+  long HW;
+  bool bf16;
+  int es;  // bytes per element of activations/weights
+  int TH, TW, tiles_h, tiles_w;
+  int gn_P;       // GroupNorm partials per image
+  int kv_chunks;  // KV-state partials per (image, head)
+  int NP, KP;     // apply operand padding: [S|z] rows (N) and K
+  int bn_lin;     // tile N of the Linear GEMMs
+  // workspace offsets (bytes)
+  size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, kvpart, Sz, SzT, QKVt, total;
+};
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Host-only shape/dtype checks and the workspace layout. Returns EDIT_OK or
+// an error code; fills `pl` on success.
+int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_weights* w, Plan& pl) {
+  if (!w) return EDIT_ERR_NULL;
+  if (w->dtype != EDIT_F32 && w->dtype != EDIT_BF16) return EDIT_ERR_DTYPE;
+  if (B < 1 || H < 1 || W < 1 || C < 1 || heads < 1 || NT < 0) return EDIT_ERR_SHAPE;
+  if (C % heads != 0 || w->c_red < 1 || w->gn_groups < 1 || w->c_red % w->gn_groups != 0) return EDIT_ERR_SHAPE;
+  if (static_cast<long>(H) * W > (1L << 28) || static_cast<long>(B) * H * W > (1L << 30) || C > 65536)
+    return EDIT_ERR_SHAPE;
+  pl = Plan();
+  pl.B = B;
+  pl.H = H;
+  pl.W = W;
+  pl.C = C;
+  pl.heads = heads;
+  pl.Cr = w->c_red;
+  pl.G = w->gn_groups;
+  pl.d = C / heads;
+  pl.Ho = (H + 1) / 2;
+  pl.Wo = (W + 1) / 2;
+  pl.M = pl.Ho * pl.Wo;
+  pl.HW = static_cast<long>(H) * W;
+  pl.NT = NT;
+  pl.bf16 = w->dtype == EDIT_BF16;
+  pl.es = pl.bf16 ? 2 : 4;
+  if (pl.bf16) {
+    // Tensor-core path constraints: 64-wide k-blocks over C, Linear tiles that
+    // divide C, conv tile N = Cr (instantiated sizes), 16-byte head offsets.
+    if (C % 128 != 0) return EDIT_ERR_UNSUPPORTED;
+    if (!(pl.Cr == 64 || pl.Cr == 128 || pl.Cr == 256 || pl.Cr == 288 || pl.Cr == 384)) return EDIT_ERR_UNSUPPORTED;
+    if (pl.d % 8 != 0 || pl.d + 1 > 144) return EDIT_ERR_UNSUPPORTED;
+    pl.bn_lin = (C % 256 == 0) ? 256 : (C % 192 == 0) ? 192 : 128;
+    pl.TW = next_pow2(W) < 128 ? next_pow2(W) : 128;
+    pl.TH = 128 / pl.TW;
+    pl.tiles_h = (H + pl.TH - 1) / pl.TH;
+    pl.tiles_w = (W + pl.TW - 1) / pl.TW;
+    pl.gn_P = pl.tiles_h * pl.tiles_w * 4;
+    // [S_h | z_h] has d + 1 columns; the apply GEMM is built for N = 48, 80, 144.
+    pl.NP = (pl.d + 1 <= 48) ? 48 : (pl.d + 1 <= 80) ? 80 : 144;
+    pl.KP = (pl.d + 63) / 64 * 64;
+  } else {
+    pl.gn_P = static_cast<int>(pl.HW < 64 ? pl.HW : 64);
+  }
+  if (NT > 0 && !(pl.d == 32 || pl.d == 64 || pl.d == 72)) return EDIT_ERR_UNSUPPORTED;
+  pl.kv_chunks = pl.M / 256;
+  if (pl.kv_chunks < 1) pl.kv_chunks = 1;
+  if (pl.kv_chunks > 64) pl.kv_chunks = 64;
+
+  const size_t es = pl.es;
+  const size_t tok = static_cast<size_t>(B) * pl.HW;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  pl.status = take(256);
+  pl.U = take(tok * pl.Cr * es);
+  pl.Gb = take(tok * pl.Cr * es);
+  pl.gnpart = take(static_cast<size_t>(B) * pl.gn_P * pl.G * 2 * 4);
+  pl.gnstats = take(static_cast<size_t>(B) * pl.G * 2 * 4);
+  pl.gnss = take(static_cast<size_t>(B) * pl.Cr * 2 * 4);
+  pl.W1t = take(static_cast<size_t>(pl.Cr) * C * es);
+  pl.Wqw1 = take(static_cast<size_t>(C) * pl.Cr * es);
+  pl.bfold = take(static_cast<size_t>(C) * 4);
+  pl.Q = take(tok * C * es);
+  pl.KVp = take(tok * 2 * C * es);
+  pl.K = take(static_cast<size_t>(B) * pl.M * C * es);
+  pl.V = take(static_cast<size_t>(B) * pl.M * C * es);
+  pl.kvpart = take(static_cast<size_t>(B) * heads * pl.kv_chunks * pl.d * (pl.d + 1) * 4);
+  pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
+  pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
+  pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
+  pl.total = off;
+  return EDIT_OK;
+}
+
+int check_weights(const edit_attn_weights* w) {
+  const void* ptrs[] = {w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b, w->q_w, w->q_b,
+                        w->k_w,   w->k_b,   w->v_w,      w->v_b,     w->kdw_w, w->kdw_b, w->vdw_w, w->vdw_b};
+  for (const void* p : ptrs) {
+    if (!p) return EDIT_ERR_NULL;
+    if (!aligned(p, 16)) return EDIT_ERR_ALIGN;
+  }
+  return EDIT_OK;
+}
+
+}  // namespace
+
+namespace {
+
+// ------------------------------------------------------------ measurement hooks
+thread_local void* const* g_stage_events = nullptr;
+thread_local int g_stage_n = 0;
+thread_local uint64_t g_launches = 0;
+
+void stage_mark(int i, cudaStream_t st) {
+  if (g_stage_events && i < g_stage_n && g_stage_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), st);
+}
+
+// ------------------------------------------------------------ launchers
+int last_launch() {
+  ++g_launches;
+  return cudaGetLastError() == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
+}
+
+int grid_for(long total, int threads) {
+  long g = (total + threads - 1) / threads;
+  const long cap = static_cast<long>(num_sms()) * 16;
+  if (g > cap) g = cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+template <int BN, int NSPLIT, int STAGES, int EPI>
+int launch_tc(const TcGemmParams& p, cudaStream_t st) {
+  using Cfg = TcGemmCfg<BN, NSPLIT, STAGES>;
+  auto kern = tc_gemm_kernel<BN, NSPLIT, STAGES, EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
+  if (grid < 1) return EDIT_OK;
+  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(p);
+  return last_launch();
+}
+
+// Box rows of a B map = the MMA N of one instruction.
+int linear_chunk(int bn) { return bn; }
+int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
+
+int gemm_linear(const TcGemmParams& p, int bn, cudaStream_t st) {
+  switch (bn) {
+    case 128: return launch_tc<128, 1, 6, EPI_LINEAR>(p, st);
+    case 192: return launch_tc<192, 1, 5, EPI_LINEAR>(p, st);
+    case 256: return launch_tc<256, 1, 4, EPI_LINEAR>(p, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+int gemm_conv(const TcGemmParams& p, int cr, cudaStream_t st) {
+  switch (cr) {
+    case 64: return launch_tc<64, 1, 8, EPI_CONV>(p, st);
+    case 128: return launch_tc<128, 1, 6, EPI_CONV>(p, st);
+    case 256: return launch_tc<256, 1, 4, EPI_CONV>(p, st);
+    case 288: return launch_tc<288, 2, 4, EPI_CONV>(p, st);
+    case 384: return launch_tc<384, 2, 3, EPI_CONV>(p, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+int gemm_apply(const TcGemmParams& p, int np, cudaStream_t st) {
+  switch (np) {
+    case 48: return launch_tc<48, 1, 4, EPI_APPLY>(p, st);
+    case 80: return launch_tc<80, 1, 4, EPI_APPLY>(p, st);
+    case 144: return launch_tc<144, 1, 4, EPI_APPLY>(p, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+int ceil_div(long a, long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Plain Linear on the tensor cores: out[rows][nsrc*C] = A[rows][K] [W0; W1; W2]^T + bias.
+int tc_linear(const void* a, long rows, int K, const void* const* wts, const void* const* biases, int nsrc, int C,
+              int bn, void* out, int* status, cudaStream_t st) {
+  TcGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!map_a(&p.a0, a, K, rows, 1, K, rows * K)) return EDIT_ERR_CUDA;
+  p.a1 = p.a0;
+  CUtensorMap* bm[3] = {&p.b0, &p.b1, &p.b2};
+  for (int s = 0; s < 3; ++s)
+    if (!map_b(bm[s], wts[s < nsrc ? s : 0], K, C, K, linear_chunk(bn))) return EDIT_ERR_CUDA;
+  p.bk = p.b0;
+  p.R = static_cast<int>(rows);
+  p.m_tiles_per_img = ceil_div(rows, 128);
+  p.num_kb = K / 64;
+  p.kb_split = p.num_kb;
+  p.n_split = C;
+  p.N = nsrc * C;
+  p.num_n_tiles = ceil_div(p.N, bn);
+  p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
+  p.out = out;
+  p.ldo = static_cast<long>(nsrc) * C;
+  for (int s = 0; s < nsrc; ++s) p.bias[s] = biases[s];
+  p.status = status;
+  return gemm_linear(p, bn, st);
+}
+
+int simt_linear(const void* a, long rows, int K, const void* const* wts, const void* const* biases, int nsrc,
+                int C, void* out, cudaStream_t st) {
+  SimtGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.a0 = static_cast<const float*>(a);
+  p.K0 = K;
+  for (int s = 0; s < nsrc; ++s) {
+    p.b[s] = static_cast<const float*>(wts[s]);
+    p.bias[s] = static_cast<const float*>(biases[s]);
+  }
+  p.n_split = C;
+  p.M = static_cast<int>(rows);
+  p.N = nsrc * C;
+  p.out = static_cast<float*>(out);
+  p.ldo = nsrc * C;
+  simt_gemm_f32<<<dim3(ceil_div(p.N, 64), ceil_div(p.M, 64)), 256, 0, st>>>(p);
+  return last_launch();
+}
+
+#define EDIT_TRY(expr)        \
+  do {                        \
+    const int rc_ = (expr);   \
+    if (rc_ != EDIT_OK) return rc_; \
+  } while (0)
+
+// Steps 1-3: K, V and the per-head [S | z] (fp32) into the workspace.
+template <typename T>
+int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  const long tok = static_cast<long>(pl.B) * pl.HW;
+  const void* wts[3] = {w->k_w, w->v_w, w->k_w};
+  const void* bs[3] = {w->k_b, w->v_b, nullptr};
+  if (pl.bf16)
+    EDIT_TRY(tc_linear(x, tok, pl.C, wts, bs, 2, pl.C, pl.bn_lin, ws + pl.KVp, status, st));
+  else
+    EDIT_TRY(simt_linear(x, tok, pl.C, wts, bs, 2, pl.C, ws + pl.KVp, st));
+  stage_mark(1, st);
+  {
+    constexpr int VEC = sizeof(T) == 2 ? 8 : 1;
+    const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C / VEC);
+    dwconv_s2_kernel<T, VEC><<<grid_for(total, 256), 256, 0, st>>>(
+        reinterpret_cast<const T*>(ws + pl.KVp), pl.B, pl.H, pl.W, pl.C, static_cast<const T*>(w->kdw_w),
+        static_cast<const T*>(w->kdw_b), static_cast<const T*>(w->vdw_w), static_cast<const T*>(w->vdw_b),
+        reinterpret_cast<T*>(ws + pl.K), reinterpret_cast<T*>(ws + pl.V));
+    EDIT_TRY(last_launch());
+  }
+  stage_mark(2, st);
+  {
+    const int nb = (pl.d + 3) / 4;
+    int threads = (nb * nb + 31) / 32 * 32;
+    if (threads < pl.d) threads = (pl.d + 31) / 32 * 32;
+    const size_t smem = 2 * 32 * static_cast<size_t>(pl.d) * sizeof(float);
+    kv_state_partial_kernel<T><<<dim3(pl.kv_chunks, pl.heads, pl.B), threads, smem, st>>>(
+        reinterpret_cast<const T*>(ws + pl.K), reinterpret_cast<const T*>(ws + pl.V), pl.M, pl.C, pl.heads,
+        pl.kv_chunks, reinterpret_cast<float*>(ws + pl.kvpart));
+    EDIT_TRY(last_launch());
+    const int per_head = pl.d * (pl.d + 1);
+    const long total = static_cast<long>(pl.B) * pl.heads * per_head;
+    kv_state_combine_kernel<<<grid_for(total, 256), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.kvpart),
+                                                                   pl.kv_chunks, per_head, total,
+                                                                   reinterpret_cast<float*>(ws + pl.Sz));
+    EDIT_TRY(last_launch());
+  }
+  if (pl.bf16) {
+    const long total = static_cast<long>(pl.B) * pl.heads * pl.NP * pl.KP;
+    sz_pack_bf16_kernel<<<grid_for(total, 256), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.Sz), pl.d,
+                                                               pl.NP, pl.KP, total,
+                                                               reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT));
+    EDIT_TRY(last_launch());
+  }
+  stage_mark(3, st);
+  return EDIT_OK;
+}
+
+// Steps 4-7: Q = ReLU([X | G] [Wq | Wq W1]^T + Wq b1 + bq) into the workspace.
+template <typename T>
+int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  const long tok = static_cast<long>(pl.B) * pl.HW;
+  const int C = pl.C, Cr = pl.Cr;
+  // 4. weight folding
+  transpose_kernel<T><<<dim3(ceil_div(Cr, 32), ceil_div(C, 32)), dim3(32, 8), 0, st>>>(
+      static_cast<const T*>(w->cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t));
+  EDIT_TRY(last_launch());
+  if (pl.bf16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!map_a(&p.a0, w->q_w, C, C, 1, C, static_cast<long>(C) * C)) return EDIT_ERR_CUDA;
+    p.a1 = p.a0;
+    if (!map_b(&p.b0, ws + pl.W1t, C, Cr, C, 128)) return EDIT_ERR_CUDA;
+    p.b1 = p.b2 = p.bk = p.b0;
+    p.R = C;
+    p.m_tiles_per_img = ceil_div(C, 128);
+    p.num_kb = C / 64;
+    p.kb_split = p.num_kb;
+    p.n_split = Cr;
+    p.N = Cr;
+    p.num_n_tiles = ceil_div(Cr, 128);
+    p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
+    p.out = ws + pl.Wqw1;
+    p.ldo = Cr;
+    p.status = status;
+    EDIT_TRY(gemm_linear(p, 128, st));
+  } else {
+    SimtGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.a0 = static_cast<const float*>(w->q_w);
+    p.K0 = C;
+    p.b[0] = reinterpret_cast<const float*>(ws + pl.W1t);
+    p.n_split = Cr;
+    p.M = C;
+    p.N = Cr;
+    p.out = reinterpret_cast<float*>(ws + pl.Wqw1);
+    p.ldo = Cr;
+    simt_gemm_f32<<<dim3(ceil_div(Cr, 64), ceil_div(C, 64)), 256, 0, st>>>(p);
+    EDIT_TRY(last_launch());
+  }
+  fold_bias_kernel<T><<<C, 128, 0, st>>>(static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
+                                         static_cast<const T*>(w->cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
+  EDIT_TRY(last_launch());
+  stage_mark(4, st);
+  // 5. U = Conv3x3(X) (+ GroupNorm partials)
+  float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
+  if (pl.bf16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!map_grid(&p.a0, x, pl.B, pl.H, pl.W, C, pl.TW, pl.TH)) return EDIT_ERR_CUDA;
+    p.a1 = p.a0;
+    if (!map_b(&p.b0, w->cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr))) return EDIT_ERR_CUDA;
+    p.b1 = p.b2 = p.bk = p.b0;
+    p.num_kb = 9 * C / 64;
+    p.kb_split = p.num_kb;
+    p.kb_per_tap = C / 64;
+    p.n_split = Cr;
+    p.N = Cr;
+    p.num_n_tiles = 1;
+    p.H = pl.H;
+    p.W = pl.W;
+    p.TH = pl.TH;
+    p.TW = pl.TW;
+    p.tiles_h = pl.tiles_h;
+    p.tiles_w = pl.tiles_w;
+    p.num_tiles = pl.B * pl.tiles_h * pl.tiles_w;
+    p.out = ws + pl.U;
+    p.ldo = Cr;
+    p.bias[0] = w->cf3_b;
+    p.gn_partials = gnpart;
+    p.groups = pl.G;
+    p.cpg = Cr / pl.G;
+    p.status = status;
+    EDIT_TRY(gemm_conv(p, Cr, st));
+  } else {
+    SimtGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.a0 = static_cast<const float*>(x);
+    p.K0 = 9 * C;
+    p.conv = 1;
+    p.B = pl.B;
+    p.H = pl.H;
+    p.W = pl.W;
+    p.Cin = C;
+    p.b[0] = static_cast<const float*>(w->cf3_w);
+    p.bias[0] = static_cast<const float*>(w->cf3_b);
+    p.n_split = Cr;
+    p.M = static_cast<int>(tok);
+    p.N = Cr;
+    p.out = reinterpret_cast<float*>(ws + pl.U);
+    p.ldo = Cr;
+    simt_gemm_f32<<<dim3(ceil_div(Cr, 64), ceil_div(tok, 64)), 256, 0, st>>>(p);
+    EDIT_TRY(last_launch());
+    gn_partial_kernel<float><<<dim3(pl.gn_P, pl.B), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.U),
+                                                                  static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
+    EDIT_TRY(last_launch());
+  }
+  stage_mark(5, st);
+  // 6. G = LeakyReLU(GN(U))
+  gn_finalize_kernel<T><<<pl.B, 32, 0, st>>>(gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
+                                              static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
+                                              reinterpret_cast<float*>(ws + pl.gnstats),
+                                              reinterpret_cast<float*>(ws + pl.gnss));
+  EDIT_TRY(last_launch());
+  if (pl.bf16) {
+    const long total8 = tok * Cr / 8;
+    gn_apply_leaky_bf16x8<<<grid_for(total8, 256), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
+        w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), total8);
+  } else {
+    const long total = tok * Cr;
+    gn_apply_leaky_kernel<float><<<grid_for(total, 256), 256, 0, st>>>(
+        reinterpret_cast<const float*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
+        w->leaky_slope, reinterpret_cast<float*>(ws + pl.Gb), total);
+  }
+  EDIT_TRY(last_launch());
+  stage_mark(6, st);
+  // 7. Q
+  if (pl.bf16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!map_a(&p.a0, x, C, tok, 1, C, tok * C)) return EDIT_ERR_CUDA;
+    if (!map_a(&p.a1, ws + pl.Gb, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, w->q_w, C, C, C, linear_chunk(pl.bn_lin))) return EDIT_ERR_CUDA;
+    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, linear_chunk(pl.bn_lin))) return EDIT_ERR_CUDA;
+    p.b1 = p.b2 = p.b0;
+    p.R = static_cast<int>(tok);
+    p.m_tiles_per_img = ceil_div(tok, 128);
+    p.kb_split = C / 64;
+    p.num_kb = C / 64 + ceil_div(Cr, 64);
+    p.n_split = C;
+    p.N = C;
+    p.num_n_tiles = C / pl.bn_lin;
+    p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
+    p.out = ws + pl.Q;
+    p.ldo = C;
+    p.bias[0] = ws + pl.bfold;
+    p.bias_f32 = 1;
+    p.relu = 1;
+    p.status = status;
+    EDIT_TRY(gemm_linear(p, pl.bn_lin, st));
+  } else {
+    SimtGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.a0 = static_cast<const float*>(x);
+    p.a1 = reinterpret_cast<const float*>(ws + pl.Gb);
+    p.K0 = C;
+    p.K1 = Cr;
+    p.b[0] = static_cast<const float*>(w->q_w);
+    p.bk = reinterpret_cast<const float*>(ws + pl.Wqw1);
+    p.n_split = C;
+    p.M = static_cast<int>(tok);
+    p.N = C;
+    p.out = reinterpret_cast<float*>(ws + pl.Q);
+    p.ldo = C;
+    p.bias[0] = reinterpret_cast<const float*>(ws + pl.bfold);
+    p.relu = 1;
+    simt_gemm_f32<<<dim3(ceil_div(C, 64), ceil_div(tok, 64)), 256, 0, st>>>(p);
+    EDIT_TRY(last_launch());
+  }
+  stage_mark(7, st);
+  return EDIT_OK;
+}
+
+// Step 8: out = per-head (Q_h S_h) / (Q_h z_h + eps).
+template <typename T>
+int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  if (pl.bf16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!map_a(&p.a0, ws + pl.Q, pl.C, pl.HW, pl.B, pl.C, pl.HW * pl.C)) return EDIT_ERR_CUDA;
+    p.a1 = p.a0;
+    if (!map_b(&p.b0, ws + pl.SzT, pl.KP, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.KP, pl.NP))
+      return EDIT_ERR_CUDA;
+    p.b1 = p.b2 = p.bk = p.b0;
+    p.R = static_cast<int>(pl.HW);
+    p.m_tiles_per_img = ceil_div(pl.HW, 128);
+    p.num_kb = pl.KP / 64;
+    p.kb_split = p.num_kb;
+    p.n_split = pl.heads * pl.NP;
+    p.N = pl.C;
+    p.num_n_tiles = pl.heads;
+    p.num_tiles = pl.B * p.m_tiles_per_img * pl.heads;
+    p.d = pl.d;
+    p.heads = pl.heads;
+    p.eps = w->attn_eps;
+    p.out = out;
+    p.ldo = pl.C;
+    p.status = status;
+    return gemm_apply(p, pl.NP, st);
+  }
+  const size_t smem = static_cast<size_t>(pl.d) * (pl.d + 1) * sizeof(float);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(apply_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  apply_simt_kernel<T><<<dim3(ceil_div(pl.HW, 128), pl.heads, pl.B), 128, smem, st>>>(
+      reinterpret_cast<const T*>(ws + pl.Q), reinterpret_cast<const float*>(ws + pl.Sz), static_cast<int>(pl.HW),
+      pl.C, pl.heads, w->attn_eps, static_cast<T*>(out));
+  return last_launch();
+}
+
+template <typename T>
+int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st) {
+  if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
+  stage_mark(0, st);
+  EDIT_TRY(run_kv<T>(x, pl, w, ws, st));
+  EDIT_TRY(run_query<T>(x, pl, w, ws, st));
+  EDIT_TRY(run_apply<T>(pl, w, ws, out, st));
+  stage_mark(8, st);
+  return EDIT_OK;
+}
+
+template <typename T, int D>
+int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
+  const size_t smem = (128 * D + 128 * (D + 1)) * sizeof(float);
+  auto kern = sdpa_blend_kernel<T, D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  kern<<<dim3(ceil_div(p.Nq, 128), p.heads, B), 128, smem, st>>>(p);
+  return last_launch();
+}
+
+template <typename T>
+int sdpa(const SdpaParams& p, int B, cudaStream_t st) {
+  switch (p.d) {
+    case 32: return launch_sdpa<T, 32>(p, B, st);
+    case 64: return launch_sdpa<T, 64>(p, B, st);
+    case 72: return launch_sdpa<T, 72>(p, B, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8_t* ws,
+           void* out_img, void* out_txt, cudaStream_t st) {
+  EDIT_TRY(run_edit<T>(x_img, pl, &w->img, ws, out_img, st));
+  if (pl.NT == 0) return EDIT_OK;  // eta = 1: the image rows are the EDiT layer
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  const long trow = static_cast<long>(pl.B) * pl.NT;
+  const void* wts[3] = {w->tq_w, w->tk_w, w->tv_w};
+  const void* bs[3] = {w->tq_b, w->tk_b, w->tv_b};
+  if (pl.bf16)
+    EDIT_TRY(tc_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, pl.bn_lin, ws + pl.QKVt, status, st));
+  else
+    EDIT_TRY(simt_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, st));
+  stage_mark(9, st);
+  const double eta = static_cast<double>(pl.HW) / static_cast<double>(pl.HW + pl.NT);
+  const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
+  // image rows: eta * y + (1 - eta) * A(Q_I, K_P, V_P)
+  SdpaParams a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = ws + pl.Q;
+  a.ldq = pl.C;
+  a.k1 = qkv + pl.C;
+  a.v1 = qkv + 2 * pl.C;
+  a.ld1 = 3L * pl.C;
+  a.n1 = pl.NT;
+  a.out = out_img;
+  a.ldo = pl.C;
+  a.Nq = static_cast<int>(pl.HW);
+  a.heads = pl.heads;
+  a.d = pl.d;
+  a.w0 = static_cast<float>(eta);
+  a.w1 = static_cast<float>(1.0 - eta);
+  a.blend_in = 1;
+  EDIT_TRY(sdpa<T>(a, pl.B, st));
+  stage_mark(10, st);
+  // text rows: eta * A(Q_P, K_I, V_I) + (1 - eta) * A(Q_P, K_P, V_P)
+  SdpaParams t;
+  std::memset(&t, 0, sizeof(t));
+  t.q = qkv;
+  t.ldq = 3L * pl.C;
+  t.k1 = ws + pl.K;
+  t.v1 = ws + pl.V;
+  t.ld1 = pl.C;
+  t.n1 = pl.M;
+  t.k2 = qkv + pl.C;
+  t.v2 = qkv + 2 * pl.C;
+  t.ld2 = 3L * pl.C;
+  t.n2 = pl.NT;
+  t.out = out_txt;
+  t.ldo = pl.C;
+  t.Nq = pl.NT;
+  t.heads = pl.heads;
+  t.d = pl.d;
+  t.w1 = static_cast<float>(eta);
+  t.w2 = static_cast<float>(1.0 - eta);
+  EDIT_TRY(sdpa<T>(t, pl.B, st));
+  stage_mark(11, st);
+  return EDIT_OK;
+}
+
+int common_checks(const void* x, const void* out, const edit_attn_weights* w, void* ws, size_t ws_bytes,
+                  const Plan& pl) {
+  if (!x || !out || !ws) return EDIT_ERR_NULL;
+  EDIT_TRY(check_weights(w));
+  if (!aligned(x, 16) || !aligned(out, 16)) return EDIT_ERR_ALIGN;
+  if (!aligned(ws, 256)) return EDIT_ERR_ALIGN;
+  if (ws_bytes < pl.total) return EDIT_ERR_WORKSPACE;
+  return EDIT_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+size_t edit_attn_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights* w) {
+  Plan pl;
+  return make_plan(B, H, W, C, heads, 0, w, pl) == EDIT_OK ? pl.total : 0;
+}
+
+int edit_attn_forward(const void* x, int B, int H, int W, int C, int heads, const edit_attn_weights* w, void* out,
+                      void* stream) {
+  Plan pl;
+  EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl));
+  EDIT_TRY(common_checks(x, out, w, w->workspace, w->workspace_bytes, pl));
+  uint8_t* ws = static_cast<uint8_t*>(w->workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st) : run_edit<float>(x, pl, w, ws, out, st);
+}
+
+size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights* w) {
+  if (!w) return 0;
+  Plan pl;
+  return make_plan(B, H, W, C, heads, N_T, &w->img, pl) == EDIT_OK ? pl.total : 0;
+}
+
+int mmedit_hybrid_forward(const void* x_img, const void* x_txt, int B, int H, int W, int N_T, int C, int heads,
+                          const mmedit_weights* w, void* out_img, void* out_txt, void* stream) {
+  if (!w) return EDIT_ERR_NULL;
+  Plan pl;
+  EDIT_TRY(make_plan(B, H, W, C, heads, N_T, &w->img, pl));
+  EDIT_TRY(common_checks(x_img, out_img, &w->img, w->workspace, w->workspace_bytes, pl));
+  if (N_T > 0) {
+    if (!x_txt || !out_txt) return EDIT_ERR_NULL;
+    if (!aligned(x_txt, 16) || !aligned(out_txt, 16)) return EDIT_ERR_ALIGN;
+    const void* tp[] = {w->tq_w, w->tq_b, w->tk_w, w->tk_b, w->tv_w, w->tv_b};
+    for (const void* p : tp) {
+      if (!p) return EDIT_ERR_NULL;
+      if (!aligned(p, 16)) return EDIT_ERR_ALIGN;
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(w->workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return pl.bf16 ? run_mm<__nv_bfloat16>(x_img, x_txt, pl, w, ws, out_img, out_txt, st)
+                 : run_mm<float>(x_img, x_txt, pl, w, ws, out_img, out_txt, st);
+}
+
+int edit_attn_read_status(const void* workspace, void* stream, int* status) {
+  if (!workspace || !status) return EDIT_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(status, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return EDIT_ERR_CUDA;
+  return EDIT_OK;
+}
+
+const char* edit_status_string(int status) {
+  switch (status) {
+    case EDIT_OK: return "ok";
+    case EDIT_ERR_NULL: return "null pointer";
+    case EDIT_ERR_SHAPE: return "bad shape";
+    case EDIT_ERR_ALIGN: return "misaligned pointer";
+    case EDIT_ERR_DTYPE: return "unsupported dtype";
+    case EDIT_ERR_WORKSPACE: return "workspace too small";
+    case EDIT_ERR_CUDA: return "CUDA error";
+    case EDIT_ERR_TIMEOUT: return "device wait timed out";
+    case EDIT_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+  }
+  return "unknown status";
+}
+
+int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights* w,
+                               edit_ws_layout* layout) {
+  if (!layout) return EDIT_ERR_NULL;
+  Plan pl;
+  EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl));
+  layout->status = static_cast<int64_t>(pl.status);
+  layout->U = static_cast<int64_t>(pl.U);
+  layout->G = static_cast<int64_t>(pl.Gb);
+  layout->Q = static_cast<int64_t>(pl.Q);
+  layout->KVp = static_cast<int64_t>(pl.KVp);
+  layout->K = static_cast<int64_t>(pl.K);
+  layout->V = static_cast<int64_t>(pl.V);
+  layout->gn_stats = static_cast<int64_t>(pl.gnstats);
+  layout->Sz = static_cast<int64_t>(pl.Sz);
+  return EDIT_OK;
+}
+
+int edit_attn_set_stage_events(void* const* events, int n) {
+  if (n < 0) return EDIT_ERR_SHAPE;
+  g_stage_events = events;
+  g_stage_n = events ? n : 0;
+  return EDIT_OK;
+}
+
+uint64_t edit_attn_kernel_launches(void) { return g_launches; }
+
+}  // extern "C"

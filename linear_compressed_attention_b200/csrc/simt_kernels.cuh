@@ -1,0 +1,544 @@
+// CUDA-core kernels of the EDiT layer: the memory-bound steps (GroupNorm,
+// depthwise stride-2 conv, KV-state reduction, apply, softmax attention for
+// the prompt blocks of MM-EDiT) and an fp32 tiled GEMM used by the fp32 path
+// (fp32 storage must stay fp32 end to end, so it does not go to the bf16
+// tensor cores).
+#pragma once
+
+#include "common.cuh"
+
+namespace edit {
+
+// ====================================================================== GEMM
+// out[m, n] = act(sum_k A(m, k) * Bw(n, k) + bias(n)), fp32.
+// A(m, k): conv mode: implicit 3x3 im2col of X[B,H,W,Cin] with zero padding,
+//          k = tap * Cin + c, tap = kh * 3 + kw;
+//          else [A0 | A1] with A0 [M][K0], A1 [M][K1].
+// Bw(n, k): source s = n / n_split holds rows [s*n_split, (s+1)*n_split) of
+//          the first K0 columns; bk [N][K1] holds columns K0.. .
+struct SimtGemmParams {
+  const float* a0;
+  const float* a1;
+  int K0, K1;
+  const float* b[3];
+  const float* bk;
+  int n_split;
+  int M, N;
+  int conv, B, H, W, Cin;
+  float* out;
+  int ldo;
+  const float* bias[3];
+  int relu;
+};
+
+__device__ __forceinline__ float simt_load_a(const SimtGemmParams& p, int m, int k) {
+  if (m >= p.M || k >= p.K0 + p.K1) return 0.f;
+  if (p.conv) {
+    const int hw = p.H * p.W;
+    const int b = m / hw, r = m - b * hw;
+    const int h = r / p.W, w = r - h * p.W;
+    const int tap = k / p.Cin, c = k - tap * p.Cin;
+    const int hh = h + tap / 3 - 1, ww = w + tap % 3 - 1;
+    if (hh < 0 || hh >= p.H || ww < 0 || ww >= p.W) return 0.f;
+    return p.a0[((static_cast<long>(b) * p.H + hh) * p.W + ww) * p.Cin + c];
+  }
+  if (k < p.K0) return p.a0[static_cast<long>(m) * p.K0 + k];
+  return p.a1[static_cast<long>(m) * p.K1 + (k - p.K0)];
+}
+
+__device__ __forceinline__ float simt_load_b(const SimtGemmParams& p, int n, int k) {
+  if (n >= p.N || k >= p.K0 + p.K1) return 0.f;
+  if (k < p.K0) {
+    const int s = n / p.n_split;
+    return p.b[s][static_cast<long>(n - s * p.n_split) * p.K0 + k];
+  }
+  return p.bk[static_cast<long>(n) * p.K1 + (k - p.K0)];
+}
+
+// 64 x 64 output tile, 256 threads, 4 x 4 outputs per thread (strided by 16).
+__global__ void __launch_bounds__(256) simt_gemm_f32(SimtGemmParams p) {
+  __shared__ float As[16][65];
+  __shared__ float Bs[16][65];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  const int K = p.K0 + p.K1;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 1024; i += 256) {
+      const int r = i >> 4, kk = i & 15;
+      As[kk][r] = simt_load_a(p, m0 + r, k0 + kk);
+      Bs[kk][r] = simt_load_b(p, n0 + r, k0 + kk);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[kk][ty + 16 * i];
+        b[i] = Bs[kk][tx + 16 * i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty + 16 * i;
+    if (m >= p.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n >= p.N) continue;
+      const int s = n / p.n_split;
+      float v = acc[i][j];
+      if (p.bias[s]) v += p.bias[s][n - s * p.n_split];
+      if (p.relu) v = fmaxf(v, 0.f);
+      p.out[static_cast<long>(m) * p.ldo + n] = v;
+    }
+  }
+}
+
+// ================================================================ GroupNorm
+// Partial sums of U [B][HW][Cr] over token chunks: part[b][chunk][g][2].
+template <typename T>
+__global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int groups, int chunks,
+                                  float* __restrict__ part) {
+  const int b = blockIdx.y, chunk = blockIdx.x;
+  const int cpg = Cr / groups;
+  const int t0 = static_cast<int>((static_cast<long>(HW) * chunk) / chunks);
+  const int t1 = static_cast<int>((static_cast<long>(HW) * (chunk + 1)) / chunks);
+  __shared__ float red[32][2];
+  for (int g = 0; g < groups; ++g) {
+    float s1 = 0.f, s2 = 0.f;
+    const long cnt = static_cast<long>(t1 - t0) * cpg;
+    for (long e = threadIdx.x; e < cnt; e += blockDim.x) {
+      const long t = t0 + e / cpg;
+      const int c = g * cpg + static_cast<int>(e % cpg);
+      const float v = to_f32(U[(static_cast<long>(b) * HW + t) * Cr + c]);
+      s1 += v;
+      s2 += v * v;
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      red[w][0] = s1;
+      red[w][1] = s2;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float a = 0.f, q = 0.f;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+        a += red[i][0];
+        q += red[i][1];
+      }
+      float* o = part + ((static_cast<long>(b) * chunks + chunk) * groups + g) * 2;
+      o[0] = a;
+      o[1] = q;
+    }
+    __syncthreads();
+  }
+}
+
+// Fixed-order (deterministic) combine of the partials in fp64, then the
+// per-channel affine form of GN: scale = gamma * rstd, shift = beta - mean * scale.
+// part: [B][P][groups][2]; stats out: [B][groups][2] (mean, rstd);
+// ss out: [B][Cr][2] (scale, shift). One block per batch item.
+template <typename T>
+__global__ void gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr, long count,
+                                   float eps, const T* __restrict__ gamma, const T* __restrict__ beta,
+                                   float* __restrict__ stats, float* __restrict__ ss) {
+  const int b = blockIdx.x;
+  const int cpg = Cr / groups;
+  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+    double s1 = 0.0, s2 = 0.0;
+    for (int i = 0; i < P; ++i) {
+      const float* q = part + ((static_cast<long>(b) * P + i) * groups + g) * 2;
+      s1 += q[0];
+      s2 += q[1];
+    }
+    const double mean = s1 / static_cast<double>(count);
+    double var = s2 / static_cast<double>(count) - mean * mean;
+    if (var < 0.0) var = 0.0;
+    const double rstd = 1.0 / sqrt(var + static_cast<double>(eps));
+    stats[(b * groups + g) * 2] = static_cast<float>(mean);
+    stats[(b * groups + g) * 2 + 1] = static_cast<float>(rstd);
+    for (int c = g * cpg; c < (g + 1) * cpg; ++c) {
+      const double sc = static_cast<double>(to_f32(gamma[c])) * rstd;
+      ss[(static_cast<long>(b) * Cr + c) * 2] = static_cast<float>(sc);
+      ss[(static_cast<long>(b) * Cr + c) * 2 + 1] = static_cast<float>(static_cast<double>(to_f32(beta[c])) - mean * sc);
+    }
+  }
+}
+
+// G = LeakyReLU(scale * U + shift), elementwise over [B][HW][Cr].
+template <typename T>
+__global__ void gn_apply_leaky_kernel(const T* __restrict__ U, const float* __restrict__ ss, long HW, int Cr,
+                                      float slope, T* __restrict__ G, long total) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % Cr);
+    const long b = i / (HW * Cr);
+    const float sc = ss[(b * Cr + c) * 2], sh = ss[(b * Cr + c) * 2 + 1];
+    float v = fmaf(to_f32(U[i]), sc, sh);
+    v = v >= 0.f ? v : v * slope;
+    G[i] = from_f32<T>(v);
+  }
+}
+
+// bf16 variant, 8 channels per thread with 16-byte loads/stores (Cr % 8 == 0).
+__global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const float* __restrict__ ss, long HW,
+                                      int Cr, float slope, __nv_bfloat16* __restrict__ G, long total8) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total8;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long e = i * 8;
+    const int c = static_cast<int>(e % Cr);
+    const long b = e / (HW * Cr);
+    const uint4 raw = *reinterpret_cast<const uint4*>(U + e);
+    const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    const float4* s4 = reinterpret_cast<const float4*>(ss + (b * Cr + c) * 2);
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 s = s4[j];
+      float v0 = fmaf(__bfloat162float(u[2 * j]), s.x, s.y);
+      float v1 = fmaf(__bfloat162float(u[2 * j + 1]), s.z, s.w);
+      o[2 * j] = v0 >= 0.f ? v0 : v0 * slope;
+      o[2 * j + 1] = v1 >= 0.f ? v1 : v1 * slope;
+    }
+    uint4 out;
+    out.x = pack_bf16x2(o[0], o[1]);
+    out.y = pack_bf16x2(o[2], o[3]);
+    out.z = pack_bf16x2(o[4], o[5]);
+    out.w = pack_bf16x2(o[6], o[7]);
+    *reinterpret_cast<uint4*>(G + e) = out;
+  }
+}
+
+// ============================================================ weight folding
+// The 1x1 conv feeds only Linear_Q, so Linear_Q(X + G W1^T + b1) =
+// X Wq^T + G (Wq W1)^T + (Wq b1 + bq). dst[c][r] = sum_k Wq[c][k] W1[k][r]
+// is formed on the tensor cores from W1 transposed; this kernel transposes
+// W1 [C][Cr] -> W1t [Cr][C] and forms the folded bias (fp32).
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, T* __restrict__ dst) {
+  __shared__ T tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[static_cast<long>(r) * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[static_cast<long>(c) * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+template <typename T>
+__global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__ bq, const T* __restrict__ b1,
+                                 int C, float* __restrict__ out) {
+  const int c = blockIdx.x;
+  float s = 0.f;
+  for (int k = threadIdx.x; k < C; k += blockDim.x) s = fmaf(to_f32(wq[static_cast<long>(c) * C + k]), to_f32(b1[k]), s);
+  s = warp_sum(s);
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+    out[c] = t + to_f32(bq[c]);
+  }
+}
+
+// ====================================================== depthwise stride-2
+// KVp [B][H][W][2C] (Linear_K | Linear_V) -> K = ReLU(DW_K), V = DW_V, each
+// [B][Ho][Wo][C]; tap (a, e) of output (i, j) reads input (2i+a-1, 2j+e-1).
+template <typename T, int VEC>
+__global__ void dwconv_s2_kernel(const T* __restrict__ kvp, int B, int H, int W, int C,
+                                 const T* __restrict__ kw, const T* __restrict__ kb, const T* __restrict__ vw,
+                                 const T* __restrict__ vb, T* __restrict__ K, T* __restrict__ V) {
+  const int Ho = (H + 1) / 2, Wo = (W + 1) / 2;
+  const int C2v = 2 * C / VEC;
+  const long total = static_cast<long>(B) * Ho * Wo * C2v;
+  for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int cv = static_cast<int>(idx % C2v);
+    long pix = idx / C2v;
+    const int j = static_cast<int>(pix % Wo);
+    pix /= Wo;
+    const int i = static_cast<int>(pix % Ho);
+    const int b = static_cast<int>(pix / Ho);
+    const int ch = cv * VEC;  // channel in [0, 2C)
+    const bool isk = ch < C;
+    const int c = isk ? ch : ch - C;
+    const T* wt = isk ? kw : vw;
+    const T* bs = isk ? kb : vb;
+    float acc[VEC];
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) acc[u] = to_f32(bs[c + u]);
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const int hh = 2 * i + a - 1;
+      if (hh < 0 || hh >= H) continue;
+#pragma unroll
+      for (int e = 0; e < 3; ++e) {
+        const int ww = 2 * j + e - 1;
+        if (ww < 0 || ww >= W) continue;
+        const T* src = kvp + ((static_cast<long>(b) * H + hh) * W + ww) * (2L * C) + ch;
+        T vals[VEC];
+        if (VEC == 8 && sizeof(T) == 2) {
+          *reinterpret_cast<uint4*>(vals) = *reinterpret_cast<const uint4*>(src);
+        } else {
+#pragma unroll
+          for (int u = 0; u < VEC; ++u) vals[u] = src[u];
+        }
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) acc[u] = fmaf(to_f32(wt[(c + u) * 9 + a * 3 + e]), to_f32(vals[u]), acc[u]);
+      }
+    }
+    T* dst = (isk ? K : V) + ((static_cast<long>(b) * Ho + i) * Wo + j) * C + c;
+    T outv[VEC];
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) outv[u] = from_f32<T>(isk ? fmaxf(acc[u], 0.f) : acc[u]);
+    if (VEC == 8 && sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(outv);
+    } else {
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) dst[u] = outv[u];
+    }
+  }
+}
+
+// ================================================================ KV state
+// Partial [S_h | z_h] over a chunk of compressed tokens:
+// part[b][h][chunk][a][c], a < d, c <= d, with column d = sum_j K_ja.
+// Thread block: ceil(d/4)^2 threads (padded to a warp multiple), each owning a
+// 4 x 4 block of S; tokens staged through shared memory 32 at a time.
+template <typename T>
+__global__ void kv_state_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int M, int C, int heads,
+                                        int chunks, float* __restrict__ part) {
+  const int d = C / heads;
+  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t0 = static_cast<int>((static_cast<long>(M) * chunk) / chunks);
+  const int t1 = static_cast<int>((static_cast<long>(M) * (chunk + 1)) / chunks);
+  extern __shared__ float kv_sm[];
+  constexpr int TT = 32;
+  float* Ks = kv_sm;            // [TT][d]
+  float* Vs = kv_sm + TT * d;   // [TT][d]
+  const int nb = (d + 3) / 4;
+  const int tid = threadIdx.x;
+  const int ba = tid / nb, bc = tid % nb;
+  const bool owner = ba < nb;
+  float acc[4][4] = {};
+  float zacc = 0.f;  // threads tid < d accumulate z[tid]
+  for (int tb = t0; tb < t1; tb += TT) {
+    const int cnt = min(TT, t1 - tb);
+    for (int e = tid; e < TT * d; e += blockDim.x) {
+      const int t = e / d, c = e - t * d;
+      float kv = 0.f, vv = 0.f;
+      if (t < cnt) {
+        const long off = (static_cast<long>(b) * M + tb + t) * C + h * d + c;
+        kv = to_f32(K[off]);
+        vv = to_f32(V[off]);
+      }
+      Ks[e] = kv;
+      Vs[e] = vv;
+    }
+    __syncthreads();
+    if (owner) {
+      for (int t = 0; t < cnt; ++t) {
+        float ka[4], vc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int a = ba * 4 + u, c = bc * 4 + u;
+          ka[u] = a < d ? Ks[t * d + a] : 0.f;
+          vc[u] = c < d ? Vs[t * d + c] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(ka[u], vc[v], acc[u][v]);
+      }
+    }
+    if (tid < d)
+      for (int t = 0; t < cnt; ++t) zacc += Ks[t * d + tid];
+    __syncthreads();
+  }
+  float* o = part + ((static_cast<long>(b) * heads + h) * chunks + chunk) * d * (d + 1);
+  if (owner) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int a = ba * 4 + u, c = bc * 4 + v;
+        if (a < d && c < d) o[a * (d + 1) + c] = acc[u][v];
+      }
+  }
+  if (tid < d) o[tid * (d + 1) + d] = zacc;
+}
+
+// Fixed-order sum of the chunk partials: Sz[b][h][a][c] (fp32).
+__global__ void kv_state_combine_kernel(const float* __restrict__ part, int chunks, int per_head, long total,
+                                        float* __restrict__ Sz) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long bh = i / per_head;
+    const int e = static_cast<int>(i - bh * per_head);
+    const float* q = part + bh * chunks * per_head + e;
+    float s = 0.f;
+    for (int k = 0; k < chunks; ++k) s += q[static_cast<long>(k) * per_head];
+    Sz[i] = s;
+  }
+}
+
+// [S_h | z_h] as the bf16 B operand of the tensor-core apply:
+// SzT[(b*heads + h)*NP + c][a] = Sz[b][h][a][c] for c <= d, a < d; zero for
+// c in (d, NP) and a in [d, KP).
+__global__ void sz_pack_bf16_kernel(const float* __restrict__ Sz, int d, int NP, int KP, long total,
+                                    __nv_bfloat16* __restrict__ SzT) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int a = static_cast<int>(i % KP);
+    const long r = i / KP;
+    const int c = static_cast<int>(r % NP);
+    const long bh = r / NP;
+    float v = 0.f;
+    if (a < d && c <= d) v = Sz[(bh * d + a) * (d + 1) + c];
+    SzT[i] = __float2bfloat16_rn(v);
+  }
+}
+
+// ==================================================================== apply
+// y_ih = (Q_ih S_h) / (Q_ih . z_h + eps) on CUDA cores (fp32 path).
+// One block per (token block, head, batch); [S_h | z_h] staged in shared memory.
+template <typename T>
+__global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restrict__ Sz, int N, int C, int heads,
+                                  float eps, T* __restrict__ out) {
+  const int d = C / heads;
+  const int h = blockIdx.y, b = blockIdx.z;
+  extern __shared__ float ap_sm[];  // [d][d+1]
+  const float* src = Sz + (static_cast<long>(b) * heads + h) * d * (d + 1);
+  for (int e = threadIdx.x; e < d * (d + 1); e += blockDim.x) ap_sm[e] = src[e];
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const T* q = Q + (static_cast<long>(b) * N + n) * C + h * d;
+  T* o = out + (static_cast<long>(b) * N + n) * C + h * d;
+  float den = 0.f;
+  for (int a = 0; a < d; ++a) den = fmaf(to_f32(q[a]), ap_sm[a * (d + 1) + d], den);
+  const float inv = 1.f / (den + eps);
+  for (int c = 0; c < d; ++c) {
+    float s = 0.f;
+    for (int a = 0; a < d; ++a) s = fmaf(to_f32(q[a]), ap_sm[a * (d + 1) + c], s);
+    o[c] = from_f32<T>(s * inv);
+  }
+}
+
+// ============================================================ MM-EDiT SDPA
+// out[b, i, head] = w0 * out[b, i, head] (or 0 when `blend_in` is 0)
+//                 + w1 * softmax(q k1^T / sqrt(d)) v1 + w2 * softmax(q k2^T / sqrt(d)) v2
+// with each softmax over its own key set (k2 absent when n2 == 0). One thread
+// per (query, head); keys staged through shared memory; online softmax with
+// exp2f. q: [B][Nq][ldq]; k*, v*: [B][n*][ld*] (head h at columns h*d).
+struct SdpaParams {
+  const void* q;
+  long ldq;
+  const void* k1;
+  const void* v1;
+  long ld1;
+  int n1;
+  const void* k2;
+  const void* v2;
+  long ld2;
+  int n2;
+  void* out;
+  long ldo;
+  int Nq, heads, d;
+  float w0, w1, w2;
+  int blend_in;
+};
+
+// Accumulates w * softmax(q K^T) V over one key set into res (registers).
+// q rows live in shared memory (qs, stride D + 1), one row per thread.
+template <typename T, int D>
+__device__ __forceinline__ void sdpa_one_set(const T* kb, const T* vb, long ld, int nk, const float* qrow,
+                                             bool active, float w, float (&res)[D], float* ks, float* vs, int h) {
+  constexpr int KT = 64;
+  float m = -INFINITY, l = 0.f;
+  float acc[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) acc[c] = 0.f;
+  for (int j0 = 0; j0 < nk; j0 += KT) {
+    const int cnt = min(KT, nk - j0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < KT * D; e += blockDim.x) {
+      const int j = e / D, c = e - j * D;
+      float kv = 0.f, vv = 0.f;
+      if (j < cnt) {
+        kv = to_f32(kb[(j0 + j) * ld + h * D + c]);
+        vv = to_f32(vb[(j0 + j) * ld + h * D + c]);
+      }
+      ks[e] = kv;
+      vs[e] = vv;
+    }
+    __syncthreads();
+    if (active) {
+      for (int j = 0; j < cnt; ++j) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int c = 0; c < D; ++c) s = fmaf(qrow[c], ks[j * D + c], s);
+        const float mn = fmaxf(m, s);
+        const float corr = exp2f(m - mn);
+        const float pj = exp2f(s - mn);
+        l = l * corr + pj;
+#pragma unroll
+        for (int c = 0; c < D; ++c) acc[c] = fmaf(pj, vs[j * D + c], acc[c] * corr);
+        m = mn;
+      }
+    }
+  }
+  const float sc = l > 0.f ? w / l : 0.f;
+#pragma unroll
+  for (int c = 0; c < D; ++c) res[c] = fmaf(acc[c], sc, res[c]);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
+  extern __shared__ float sd_sm[];
+  float* ks = sd_sm;                 // [64][D]
+  float* vs = sd_sm + 64 * D;        // [64][D]
+  float* qs = sd_sm + 128 * D;       // [blockDim][D + 1]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool active = i < p.Nq;
+  const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
+  float* qrow = qs + threadIdx.x * (D + 1);
+  const T* qp = reinterpret_cast<const T*>(p.q) + (static_cast<long>(b) * p.Nq + (active ? i : 0)) * p.ldq + h * D;
+  for (int c = 0; c < D; ++c) qrow[c] = active ? to_f32(qp[c]) * qscale : 0.f;
+  float res[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) res[c] = 0.f;
+  sdpa_one_set<T, D>(reinterpret_cast<const T*>(p.k1) + static_cast<long>(b) * p.n1 * p.ld1,
+                     reinterpret_cast<const T*>(p.v1) + static_cast<long>(b) * p.n1 * p.ld1, p.ld1, p.n1, qrow,
+                     active, p.w1, res, ks, vs, h);
+  if (p.n2 > 0)
+    sdpa_one_set<T, D>(reinterpret_cast<const T*>(p.k2) + static_cast<long>(b) * p.n2 * p.ld2,
+                       reinterpret_cast<const T*>(p.v2) + static_cast<long>(b) * p.n2 * p.ld2, p.ld2, p.n2, qrow,
+                       active, p.w2, res, ks, vs, h);
+  if (!active) return;
+  T* op = reinterpret_cast<T*>(p.out) + (static_cast<long>(b) * p.Nq + i) * p.ldo + h * D;
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    float v = res[c];
+    if (p.blend_in) v = fmaf(p.w0, to_f32(op[c]), v);
+    op[c] = from_f32<T>(v);
+  }
+}
+
+}  // namespace edit

@@ -1,0 +1,122 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point the header declares, and rejects bad arguments on the host with the
+documented codes before touching the device (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_compressed_attention_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "edit_attn.h")).read()
+    return re.findall(r"^EDIT_API\s+[\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    assert set(names) == set(bd.EXPORTS)
+    for must in ("edit_attn_forward", "mmedit_hybrid_forward"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = bd.lib()
+    for n in header_functions():
+        assert hasattr(L, n), n
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def fake_struct(dtype=bd.EDIT_BF16, c_red=288, groups=32, ws_bytes=1 << 40, base=0x10000):
+    s = bd.EditAttnWeights()
+    s.dtype, s.c_red, s.gn_groups = dtype, c_red, groups
+    s.gn_eps, s.leaky_slope, s.attn_eps = 1e-5, 0.01, 1e-6
+    for k, n in enumerate(bd.WEIGHT_NAMES):
+        setattr(s, n, base + 0x1000 * (k + 1))   # never dereferenced: validation fails first
+    s.workspace = 0x100000
+    s.workspace_bytes = ws_bytes
+    return s
+
+
+def fwd(s, B=1, H=64, W=64, C=1152, heads=16, x=0x200000, out=0x400000):
+    return bd.lib().edit_attn_forward(ctypes.c_void_p(x), B, H, W, C, heads, ctypes.byref(s),
+                                      ctypes.c_void_p(out), None)
+
+
+def test_workspace_query_is_host_only_and_monotone():
+    s = fake_struct()
+    a = bd.edit_attn_workspace_bytes(1, 64, 64, 1152, 16, s)
+    b = bd.edit_attn_workspace_bytes(1, 128, 128, 1152, 16, s)
+    assert 0 < a < b
+    assert a % 256 == 0
+    assert bd.edit_attn_workspace_bytes(1, 64, 64, 1152, 7, s) == 0        # C % heads
+    f = fake_struct(dtype=bd.EDIT_F32, c_red=16, groups=4)
+    assert bd.edit_attn_workspace_bytes(1, 16, 16, 64, 2, f) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), -2), (dict(H=0), -2), (dict(W=-1), -2), (dict(heads=0), -2), (dict(heads=5), -2),
+    (dict(x=0), -1), (dict(out=0), -1), (dict(x=0x200008), -3), (dict(out=0x400004), -3),
+])
+def test_forward_rejects_bad_arguments(kw, code):
+    assert fwd(fake_struct(), **kw) == code
+
+
+def test_forward_rejects_bad_weights_and_workspace():
+    s = fake_struct()
+    s.q_w = None
+    assert fwd(s) == -1
+    s = fake_struct()
+    s.k_b = 0x10008
+    assert fwd(s) == -3
+    s = fake_struct()
+    s.dtype = 7
+    assert fwd(s) == -4
+    s = fake_struct(ws_bytes=1024)
+    assert fwd(s) == -5
+    s = fake_struct()
+    s.workspace = 0x100010          # 16- but not 256-byte aligned
+    assert fwd(s) == -3
+    s = fake_struct(c_red=100, groups=4)   # no tensor-core conv tile for this width
+    assert fwd(s) == -8
+    s = fake_struct(c_red=288, groups=5)   # groups must divide c_red
+    assert fwd(s) == -2
+    assert fwd(fake_struct(), C=1000, heads=8) == -8     # C % 128 for bf16
+
+
+def test_mm_rejects_bad_arguments():
+    m = bd.MMEditWeights()
+    m.img = fake_struct()
+    for k, n in enumerate(bd.TEXT_NAMES):
+        setattr(m, n, 0x800000 + 0x1000 * k)
+    m.workspace, m.workspace_bytes = 0x100000, 1 << 40
+    L = bd.lib()
+    call = lambda **kw: L.mmedit_hybrid_forward(  # noqa: E731
+        ctypes.c_void_p(kw.get("xi", 0x200000)), ctypes.c_void_p(kw.get("xt", 0x300000)), 1, 64, 64,
+        kw.get("nt", 333), 1536, kw.get("heads", 24), ctypes.byref(m), ctypes.c_void_p(0x400000),
+        ctypes.c_void_p(kw.get("ot", 0x500000)), None)
+    assert call(nt=-1) == -2
+    assert call(xt=0) == -1
+    assert call(ot=0x500002) == -3
+    assert call(heads=12) == -8        # d = 128: no SDPA kernel for it
+    assert bd.mmedit_workspace_bytes(1, 64, 64, 333, 1536, 24, m) > bd.mmedit_workspace_bytes(1, 64, 64, 0, 1536, 24, m)
+
+
+def test_status_strings():
+    assert bd.status_string(0) == "ok"
+    assert bd.status_string(-7) == "device wait timed out"
+    assert bd.status_string(-99) == "unknown status"
+
+
+def test_workspace_layout_offsets():
+    s = fake_struct()
+    lay = bd.edit_attn_workspace_layout(1, 64, 64, 1152, 16, s)
+    offs = [lay[k] for k in ("U", "G", "Q", "KVp", "K", "V", "gn_stats", "Sz")]
+    assert lay["status"] == 0
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs)
+    assert max(offs) < bd.edit_attn_workspace_bytes(1, 64, 64, 1152, 16, s)

@@ -1,0 +1,174 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle on the
+same seeded inputs. Error metric: max |gpu - oracle| / max |oracle| per
+output tensor; bars 1e-4 (fp32 storage) and 2e-2 (bf16 storage, fp32
+accumulation). Intermediates kept in the workspace are checked too."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.edit_oracle as O
+from linear_compressed_attention_b200 import binding as bd
+from linear_compressed_attention_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def max_rel(g, o):
+    g, o = np.asarray(g, np.float64), np.asarray(o, np.float64)
+    return float(np.max(np.abs(g - o)) / max(np.max(np.abs(o)), 1e-30))
+
+
+def gpu_layer(cfg, d):
+    layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"],
+                             n_txt=cfg.get("n_txt") or 0, mm=cfg.get("n_txt") is not None)
+    x = torch.from_numpy(d["x"]).to("cuda", layer.tdtype)
+    return layer, x
+
+
+def run_edit(cfg, d):
+    layer, x = gpu_layer(cfg, d)
+    out = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    return layer, out.float().cpu().numpy()
+
+
+def check_edit(cfg, d, intermediates=True):
+    layer, y = run_edit(cfg, d)
+    yo, it = O.edit_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"], return_intermediates=True)
+    tol = TOL[cfg["dtype"]]
+    errs = {"out": max_rel(y, yo)}
+    if intermediates:
+        B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+        N, M, dh, Cr = H * W, O.compressed_count(H, W), C // heads, cfg["c_red"]
+        f32 = torch.float32
+        errs["U"] = max_rel(layer.intermediate("U", (B, H, W, Cr)).float().cpu(), it["U"])
+        errs["Q"] = max_rel(layer.intermediate("Q", (B, N, C)).float().cpu(), it["Q"])
+        errs["K"] = max_rel(layer.intermediate("K", (B, M, C)).float().cpu(), it["K"])
+        errs["V"] = max_rel(layer.intermediate("V", (B, M, C)).float().cpu(), it["V"])
+        Sz = layer.intermediate("Sz", (B, heads, dh, dh + 1), f32).cpu().numpy()
+        errs["S"] = max_rel(Sz[..., :dh], it["S"])
+        errs["z"] = max_rel(Sz[..., dh], it["z"])
+        st = layer.intermediate("gn_stats", (B, cfg["gn_groups"], 2), f32).cpu().numpy()
+        errs["gn_mean"] = float(np.max(np.abs(st[..., 0] - it["gn_mean"])) / np.sqrt(it["gn_var"].max()))
+        errs["gn_rstd"] = max_rel(st[..., 1], 1.0 / np.sqrt(it["gn_var"] + d["gn_eps"]))
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (errs, tol)
+    return errs
+
+
+SMALL_BF16 = [
+    dict(B=2, H=6, W=5, C=128, c_red=64, gn_groups=8, heads=2),        # d = 64, odd grid, batch 2
+    dict(B=1, H=17, W=9, C=256, c_red=64, gn_groups=4, heads=4),       # ragged tiles both ways
+    dict(B=1, H=9, W=7, C=1152, c_red=288, gn_groups=32, heads=16),    # d = 72, the workload widths
+    dict(B=1, H=1, W=1, C=128, c_red=64, gn_groups=4, heads=4),        # one token, d = 32
+    dict(B=1, H=5, W=130, C=128, c_red=128, gn_groups=8, heads=1),     # W > 128, d = 128
+    dict(B=3, H=12, W=20, C=384, c_red=256, gn_groups=8, heads=6),     # d = 64, 3 images
+    dict(B=1, H=8, W=8, C=1536, c_red=384, gn_groups=32, heads=24),    # MM widths
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_BF16, ids=lambda s: "x".join(str(s[k]) for k in ("B", "H", "W", "C", "heads")))
+def test_bf16_small_shapes(shape):
+    cfg = dict(shape, dtype="bf16", seed=21, nonzero_affine=True)
+    check_edit(cfg, make_inputs(**cfg))
+
+
+SMALL_F32 = [
+    dict(B=2, H=5, W=7, C=48, c_red=12, gn_groups=3, heads=3),
+    dict(B=1, H=1, W=1, C=32, c_red=8, gn_groups=2, heads=2),
+    dict(B=1, H=11, W=4, C=72, c_red=24, gn_groups=6, heads=1),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_F32, ids=lambda s: "x".join(str(s[k]) for k in ("B", "H", "W", "C", "heads")))
+def test_fp32_small_shapes(shape):
+    cfg = dict(shape, dtype="f32", seed=22, nonzero_affine=True)
+    check_edit(cfg, make_inputs(**cfg))
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "px512_b2", "px1024", "px2048"])
+def test_workload(name):
+    cfg = dict(WORKLOADS[name])
+    errs = check_edit(cfg, make_inputs(**cfg))
+    print(name, errs)
+
+
+@pytest.mark.slow
+def test_workload_px4096_full_size():
+    """The 65,536-token layer at full size, every output element against the
+    oracle (inputs with 5% outlier tokens)."""
+    cfg = dict(WORKLOADS["px4096"])
+    errs = check_edit(cfg, make_inputs(**cfg), intermediates=False)
+    print("px4096", errs)
+
+
+def test_deterministic_and_status_clean():
+    cfg = dict(WORKLOADS["px1024"])
+    d = make_inputs(**cfg)
+    layer, x = gpu_layer(cfg, d)
+    outs = [layer.forward(x).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
+def test_shared_kv_weights_literal_reading():
+    cfg = dict(B=1, H=8, W=8, C=128, c_red=64, gn_groups=8, heads=2, dtype="bf16", seed=5)
+    d = make_inputs(**cfg)
+    d["v_w"], d["v_b"], d["vdw_w"], d["vdw_b"] = d["k_w"], d["k_b"], d["kdw_w"], d["kdw_b"]
+    layer, _ = run_edit(cfg, d)
+    K = layer.intermediate("K", (1, 16, 128)).float()
+    V = layer.intermediate("V", (1, 16, 128)).float()
+    assert torch.equal(K, torch.relu(V))
+
+
+# ------------------------------------------------------------------ MM-EDiT
+
+def check_mm(cfg, d):
+    layer, xi = gpu_layer(cfg, d)
+    nt = cfg.get("n_txt") or 0
+    xt = torch.from_numpy(d["x_txt"]).to("cuda", layer.tdtype) if nt else None
+    oi, ot = layer.forward_mm(xi, xt)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ri, rt = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, cfg["heads"])
+    tol = TOL[cfg["dtype"]]
+    errs = {"img": max_rel(oi.float().cpu().numpy(), ri)}
+    if nt:
+        errs["txt"] = max_rel(ot.float().cpu().numpy(), rt)
+    assert all(v <= tol for v in errs.values()), (errs, tol)
+    return errs
+
+
+MM_SMALL = [
+    dict(dtype="bf16", B=2, H=6, W=7, C=128, c_red=64, gn_groups=8, heads=2, n_txt=5),     # d = 64
+    dict(dtype="bf16", B=1, H=9, W=9, C=1152, c_red=288, gn_groups=32, heads=16, n_txt=70),  # d = 72
+    dict(dtype="bf16", B=1, H=4, W=4, C=128, c_red=64, gn_groups=8, heads=4, n_txt=1),     # d = 32, one prompt token
+    dict(dtype="f32", B=2, H=5, W=3, C=64, c_red=16, gn_groups=4, heads=2, n_txt=7),       # d = 32
+]
+
+
+@pytest.mark.parametrize("shape", MM_SMALL, ids=lambda s: f"{s['dtype']}-{s['C']}-{s['n_txt']}")
+def test_mm_small(shape):
+    cfg = dict(shape, seed=31, nonzero_affine=True)
+    check_mm(cfg, make_inputs(**cfg))
+
+
+def test_mm_without_prompt_tokens_is_edit():
+    cfg = dict(dtype="bf16", B=1, H=8, W=8, C=128, c_red=64, gn_groups=8, heads=2, n_txt=0, seed=32)
+    d = make_inputs(**cfg)
+    layer, xi = gpu_layer(cfg, d)
+    oi, _ = layer.forward_mm(xi, None)
+    torch.cuda.synchronize()
+    e = bd.EditAttention(d, 1, 8, 8, 128, 2, "bf16")
+    y = e.forward(xi)
+    torch.cuda.synchronize()
+    assert torch.equal(oi, y)
+
+
+def test_mm_workload():
+    cfg = dict(WORKLOADS["mm1024"])
+    print("mm1024", check_mm(cfg, make_inputs(**cfg)))
