@@ -145,11 +145,16 @@ EDIT_API const char *edit_status_string(int status);
  * for inspection after the call completes (-1 when absent). Each tensor is
  * stored in the call's dtype unless noted:
  *   U [B,H,W,c_red]; G = LeakyReLU(GN(U)) [B,H*W,c_red]; Q [B,H*W,C];
- *   KVp [B,H*W,2C] (Linear_K(X) | Linear_V(X) per token); K, V [B,M,C];
+ *   KVp [B,H*W,2C] (Linear_K(X) | Linear_V(X) per token);
+ *   K, V [B,M,C] token-major (fp32 calls and MM-EDiT calls only);
+ *   KT [B][C][Mp], VTx [B][heads][NP][Mp] channel-major (bf16 only): token
+ *     t = i*Wop + j of the compressed grid padded to Wop columns (padding
+ *     tokens are 0); row d of each VTx head block is all ones;
  *   gn_stats fp32 [B][gn_groups][2] (mean, rstd);
- *   Sz fp32 [B][heads][d][d+1] (S_h with z_h as the last column). */
+ *   Sz fp32 [B][heads][d][d+1] (S_h with z_h as the last column).
+ * Mp, Wop, NP give the padded sizes (Mp = M, Wop = ceil(W/2), NP = 0 for fp32). */
 typedef struct {
-  int64_t status, U, G, Q, KVp, K, V, gn_stats, Sz;
+  int64_t status, U, G, Q, KVp, K, V, gn_stats, Sz, KT, VTx, Mp, Wop, NP;
 } edit_ws_layout;
 
 EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,

@@ -38,7 +38,8 @@ class MMEditWeights(ctypes.Structure):
 
 
 class WsLayout(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int64) for n in ("status", "U", "G", "Q", "KVp", "K", "V", "gn_stats", "Sz")]
+    _fields_ = [(n, ctypes.c_int64) for n in ("status", "U", "G", "Q", "KVp", "K", "V", "gn_stats", "Sz", "KT",
+                                              "VTx", "Mp", "Wop", "NP")]
 
 
 _lib = None

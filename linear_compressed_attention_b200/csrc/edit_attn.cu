@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "simt_kernels.cuh"
+#include "tc_conv.cuh"
 #include "tc_gemm.cuh"
 
 using namespace edit;
@@ -74,6 +75,33 @@ bool map_b(CUtensorMap* m, const void* base, long K, long rows, long ld, int box
   return encode(m, 2, base, dims, st, box);
 }
 
+// Output of the staged epilogue: [rows][ncols] bf16 (row stride ld), box 64 x 32.
+bool map_out2d(CUtensorMap* m, const void* base, long ncols, long rows, long ld) {
+  cuuint64_t dims[2] = {(cuuint64_t)ncols, (cuuint64_t)rows};
+  cuuint64_t st[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, 32};
+  return encode(m, 2, base, dims, st, box);
+}
+
+// Conv output U [B][H][W][Cr] bf16; one warp's 32 tile rows as a box
+// 64 x bw x bh x 1 with bw = min(TW, 32), bh = 32 / bw.
+bool map_out_grid(CUtensorMap* m, const void* base, int B, int H, int W, int Cr, int TW) {
+  const int bw = TW < 32 ? TW : 32;
+  cuuint64_t dims[4] = {(cuuint64_t)Cr, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t st[3] = {(cuuint64_t)Cr * 2, (cuuint64_t)W * Cr * 2, (cuuint64_t)H * W * Cr * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)bw, (cuuint32_t)(32 / bw), 1};
+  return encode(m, 4, base, dims, st, box);
+}
+
+// Conv input patch for tap reuse: [B][H][W][C] bf16, box 64 x 130 x 3 x 1
+// (3 image rows x 130 pixels: a 128-pixel tile row plus its halo).
+bool map_patch(CUtensorMap* m, const void* base, int B, int H, int W, int C) {
+  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t st[3] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
+  cuuint32_t box[4] = {64, 130, 3, 1};
+  return encode(m, 4, base, dims, st, box);
+}
+
 // Conv input grid [B][H][W][C] bf16, box 64 x TW x TH x 1.
 bool map_grid(CUtensorMap* m, const void* base, int B, int H, int W, int C, int TW, int TH) {
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
@@ -91,6 +119,9 @@ int num_sms() {
 // ------------------------------------------------------------ plan
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Planning is host-only (no CUDA call), so chunking uses the B200 SM count.
+int num_sms_hint() { return 148; }
+
 struct Plan {
   // geometry
   int B, H, W, C, heads, Cr, G, d, Ho, Wo, M, NT;
@@ -102,8 +133,11 @@ struct Plan {
   int kv_chunks;  // KV-state partials per (image, head)
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
+  int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
+  int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
   // workspace offsets (bytes)
-  size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, kvpart, Sz, SzT, QKVt, total;
+  size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
+      total;
 };
 
 int next_pow2(int v) {
@@ -158,9 +192,21 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.gn_P = static_cast<int>(pl.HW < 64 ? pl.HW : 64);
   }
   if (NT > 0 && !(pl.d == 32 || pl.d == 64 || pl.d == 72)) return EDIT_ERR_UNSUPPORTED;
-  pl.kv_chunks = pl.M / 256;
-  if (pl.kv_chunks < 1) pl.kv_chunks = 1;
-  if (pl.kv_chunks > 64) pl.kv_chunks = 64;
+  if (pl.bf16) {
+    // Tensor-core KV state: tokens on a grid padded to 32 columns, split into
+    // chunks of kv_kb 64-token blocks so that B * heads * chunks fills the GPU.
+    pl.Wop = (pl.Wo + 31) / 32 * 32;
+    pl.Mp = pl.Ho * pl.Wop;
+    const int total_kb = (pl.Mp + 63) / 64;
+    const int want = (2 * num_sms_hint() + B * heads - 1) / (B * heads);  // chunks per (image, head)
+    pl.kv_kb = (total_kb + want - 1) / (want > 0 ? want : 1);
+    if (pl.kv_kb < 4) pl.kv_kb = 4;
+    pl.kv_chunks = (total_kb + pl.kv_kb - 1) / pl.kv_kb;
+  } else {
+    pl.kv_chunks = pl.M / 256;
+    if (pl.kv_chunks < 1) pl.kv_chunks = 1;
+    if (pl.kv_chunks > 64) pl.kv_chunks = 64;
+  }
 
   const size_t es = pl.es;
   const size_t tok = static_cast<size_t>(B) * pl.HW;
@@ -181,8 +227,12 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.bfold = take(static_cast<size_t>(C) * 4);
   pl.Q = take(tok * C * es);
   pl.KVp = take(tok * 2 * C * es);
-  pl.K = take(static_cast<size_t>(B) * pl.M * C * es);
-  pl.V = take(static_cast<size_t>(B) * pl.M * C * es);
+  // token-major K, V: the fp32 path and MM-EDiT (prompt-row attention) read them
+  const bool tokmajor = !pl.bf16 || NT > 0;
+  pl.K = tokmajor ? take(static_cast<size_t>(B) * pl.M * C * es) : 0;
+  pl.V = tokmajor ? take(static_cast<size_t>(B) * pl.M * C * es) : 0;
+  pl.KT = pl.bf16 ? take(static_cast<size_t>(B) * C * pl.Mp * 2) : 0;
+  pl.VTx = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.Mp * 2) : 0;
   pl.kvpart = take(static_cast<size_t>(B) * heads * pl.kv_chunks * pl.d * (pl.d + 1) * 4);
   pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
   pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
@@ -240,35 +290,131 @@ int launch_tc(const TcGemmParams& p, cudaStream_t st) {
   return last_launch();
 }
 
-// Box rows of a B map = the MMA N of one instruction.
-int linear_chunk(int bn) { return bn; }
-int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
+// Pair kernel: clusters of 2 CTAs on neighbouring SMs, one persistent pair per
+// co-resident cluster slot.
+template <int BN, int NSPLIT, int STAGES, int EPI>
+int launch_pair(const TcGemmParams& p, cudaStream_t st) {
+  using Cfg = TcPairCfg<BN, NSPLIT, STAGES>;
+  auto kern = tc_gemm_pair_kernel<BN, NSPLIT, STAGES, EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  if (p.num_tiles < 1) return EDIT_OK;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;  // per instantiation; same device model throughout a process
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
+    max_clusters = n;
+  }
+  const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return EDIT_ERR_CUDA;
+  return last_launch();
+}
 
-int gemm_linear(const TcGemmParams& p, int bn, cudaStream_t st) {
-  switch (bn) {
-    case 128: return launch_tc<128, 1, 6, EPI_LINEAR>(p, st);
-    case 192: return launch_tc<192, 1, 5, EPI_LINEAR>(p, st);
-    case 256: return launch_tc<256, 1, 4, EPI_LINEAR>(p, st);
+// Conv with tap reuse on CTA pairs (tiles of 128 pixels of one image row).
+template <int BN, int NSPLIT, int NB>
+int launch_conv_pair(const TcGemmParams& p, cudaStream_t st) {
+  using Cfg = ConvPairCfg<BN, NSPLIT, NB>;
+  auto kern = tc_conv_pair_kernel<BN, NSPLIT, NB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  if (p.num_tiles < 1) return EDIT_OK;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
+    max_clusters = n;
+  }
+  const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return EDIT_ERR_CUDA;
+  return last_launch();
+}
+
+int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st) {
+  p.num_tiles = (p.num_m_tiles + 1) / 2;
+  switch (cr) {
+    case 64: return launch_conv_pair<64, 1, 8>(p, st);
+    case 128: return launch_conv_pair<128, 1, 7>(p, st);
+    case 256: return launch_conv_pair<256, 1, 7>(p, st);
+    case 288: return launch_conv_pair<288, 2, 7>(p, st);
+    case 384: return launch_conv_pair<384, 2, 5>(p, st);
   }
   return EDIT_ERR_UNSUPPORTED;
 }
 
-int gemm_conv(const TcGemmParams& p, int cr, cudaStream_t st) {
+// Box rows of a B map = the MMA N of one instruction (half of it per CTA in a pair).
+int linear_chunk(int bn) { return bn; }
+int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
+
+// Linear GEMMs on CTA pairs: 256 x 256 pair tiles.
+constexpr int kPairBN = 256;
+int gemm_linear_pair(TcGemmParams& p, cudaStream_t st) {
+  const int m_pairs = (p.num_m_tiles + 1) / 2;
+  p.num_n_tiles = (p.N + kPairBN - 1) / kPairBN;
+  p.num_tiles = m_pairs * p.num_n_tiles;
+  return launch_pair<kPairBN, 1, 5, EPI_LINEAR>(p, st);
+}
+
+// Small Linear GEMMs (weight folding) on single CTAs: 128 x 128 tiles.
+int gemm_linear(const TcGemmParams& p, int bn, cudaStream_t st) {
+  if (bn == 128) return launch_tc<128, 1, 6, EPI_LINEAR>(p, st);
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+// 3x3 conv on CTA pairs: 256 tokens x Cr pair tiles.
+int gemm_conv(TcGemmParams& p, int cr, cudaStream_t st) {
+  p.num_tiles = (p.num_m_tiles + 1) / 2;
   switch (cr) {
-    case 64: return launch_tc<64, 1, 8, EPI_CONV>(p, st);
-    case 128: return launch_tc<128, 1, 6, EPI_CONV>(p, st);
-    case 256: return launch_tc<256, 1, 4, EPI_CONV>(p, st);
-    case 288: return launch_tc<288, 2, 4, EPI_CONV>(p, st);
-    case 384: return launch_tc<384, 2, 3, EPI_CONV>(p, st);
+    case 64: return launch_pair<64, 1, 9, EPI_CONV>(p, st);
+    case 128: return launch_pair<128, 1, 7, EPI_CONV>(p, st);
+    case 256: return launch_pair<256, 1, 5, EPI_CONV>(p, st);
+    case 288: return launch_pair<288, 2, 5, EPI_CONV>(p, st);
+    case 384: return launch_pair<384, 2, 4, EPI_CONV>(p, st);
   }
   return EDIT_ERR_UNSUPPORTED;
 }
 
 int gemm_apply(const TcGemmParams& p, int np, cudaStream_t st) {
   switch (np) {
-    case 48: return launch_tc<48, 1, 4, EPI_APPLY>(p, st);
-    case 80: return launch_tc<80, 1, 4, EPI_APPLY>(p, st);
-    case 144: return launch_tc<144, 1, 4, EPI_APPLY>(p, st);
+    case 48: return launch_tc<48, 1, 8, EPI_APPLY>(p, st);
+    case 80: return launch_tc<80, 1, 8, EPI_APPLY>(p, st);
+    case 144: return launch_tc<144, 1, 6, EPI_APPLY>(p, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+int gemm_kvstate(const TcGemmParams& p, int np, cudaStream_t st) {
+  switch (np) {
+    case 48: return launch_tc<48, 1, 8, EPI_KVSTATE>(p, st);
+    case 80: return launch_tc<80, 1, 8, EPI_KVSTATE>(p, st);
+    case 144: return launch_tc<144, 1, 6, EPI_KVSTATE>(p, st);
   }
   return EDIT_ERR_UNSUPPORTED;
 }
@@ -284,21 +430,22 @@ int tc_linear(const void* a, long rows, int K, const void* const* wts, const voi
   p.a1 = p.a0;
   CUtensorMap* bm[3] = {&p.b0, &p.b1, &p.b2};
   for (int s = 0; s < 3; ++s)
-    if (!map_b(bm[s], wts[s < nsrc ? s : 0], K, C, K, linear_chunk(bn))) return EDIT_ERR_CUDA;
+    if (!map_b(bm[s], wts[s < nsrc ? s : 0], K, C, K, kPairBN / 2)) return EDIT_ERR_CUDA;
+  (void)bn;
   p.bk = p.b0;
   p.R = static_cast<int>(rows);
   p.m_tiles_per_img = ceil_div(rows, 128);
+  p.num_m_tiles = p.m_tiles_per_img;
   p.num_kb = K / 64;
   p.kb_split = p.num_kb;
   p.n_split = C;
   p.N = nsrc * C;
-  p.num_n_tiles = ceil_div(p.N, bn);
-  p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
   p.out = out;
   p.ldo = static_cast<long>(nsrc) * C;
+  if (!map_out2d(&p.out_map, out, p.N, rows, p.ldo)) return EDIT_ERR_CUDA;
   for (int s = 0; s < nsrc; ++s) p.bias[s] = biases[s];
   p.status = status;
-  return gemm_linear(p, bn, st);
+  return gemm_linear_pair(p, st);
 }
 
 int simt_linear(const void* a, long rows, int K, const void* const* wts, const void* const* biases, int nsrc,
@@ -338,17 +485,52 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   else
     EDIT_TRY(simt_linear(x, tok, pl.C, wts, bs, 2, pl.C, ws + pl.KVp, st));
   stage_mark(1, st);
-  {
-    constexpr int VEC = sizeof(T) == 2 ? 8 : 1;
-    const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C / VEC);
-    dwconv_s2_kernel<T, VEC><<<grid_for(total, 256), 256, 0, st>>>(
-        reinterpret_cast<const T*>(ws + pl.KVp), pl.B, pl.H, pl.W, pl.C, static_cast<const T*>(w->kdw_w),
-        static_cast<const T*>(w->kdw_b), static_cast<const T*>(w->vdw_w), static_cast<const T*>(w->vdw_b),
-        reinterpret_cast<T*>(ws + pl.K), reinterpret_cast<T*>(ws + pl.V));
+  if (pl.bf16) {
+    __nv_bfloat16* KT = reinterpret_cast<__nv_bfloat16*>(ws + pl.KT);
+    __nv_bfloat16* VTx = reinterpret_cast<__nv_bfloat16*>(ws + pl.VTx);
+    dwconv_s2_t_kernel<<<dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64)), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(ws + pl.KVp), pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, pl.Mp, pl.NP,
+        static_cast<const __nv_bfloat16*>(w->kdw_w), static_cast<const __nv_bfloat16*>(w->kdw_b),
+        static_cast<const __nv_bfloat16*>(w->vdw_w), static_cast<const __nv_bfloat16*>(w->vdw_b), KT, VTx,
+        pl.K ? reinterpret_cast<__nv_bfloat16*>(ws + pl.K) : nullptr,
+        pl.V ? reinterpret_cast<__nv_bfloat16*>(ws + pl.V) : nullptr);
     EDIT_TRY(last_launch());
-  }
-  stage_mark(2, st);
-  {
+    const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * pl.Mp;
+    vtx_pad_rows_kernel<<<grid_for(padn, 256), 256, 0, st>>>(VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
+    EDIT_TRY(last_launch());
+    stage_mark(2, st);
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!map_a(&p.a0, KT, pl.Mp, static_cast<long>(pl.B) * pl.C, 1, pl.Mp, static_cast<long>(pl.B) * pl.C * pl.Mp))
+      return EDIT_ERR_CUDA;
+    p.a1 = p.a0;
+    if (!map_b(&p.b0, VTx, pl.Mp, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.Mp, pl.NP)) return EDIT_ERR_CUDA;
+    p.b1 = p.b2 = p.bk = p.b0;
+    p.num_kb = (pl.Mp + 63) / 64;
+    p.kb_split = p.num_kb;
+    p.kb_per_chunk = pl.kv_kb;
+    p.num_chunks = pl.kv_chunks;
+    p.num_m_tiles = pl.kv_chunks;
+    p.num_tiles = pl.B * pl.heads * pl.kv_chunks;
+    p.num_n_tiles = 1;
+    p.n_split = pl.NP;
+    p.N = pl.NP;
+    p.d = pl.d;
+    p.heads = pl.heads;
+    p.kv_rows_per_img = pl.C;
+    p.kv_part = reinterpret_cast<float*>(ws + pl.kvpart);
+    p.status = reinterpret_cast<int*>(ws + pl.status);
+    EDIT_TRY(gemm_kvstate(p, pl.NP, st));
+  } else {
+    {
+      const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C);
+      dwconv_s2_kernel<T, 1><<<grid_for(total, 256), 256, 0, st>>>(
+          reinterpret_cast<const T*>(ws + pl.KVp), pl.B, pl.H, pl.W, pl.C, static_cast<const T*>(w->kdw_w),
+          static_cast<const T*>(w->kdw_b), static_cast<const T*>(w->vdw_w), static_cast<const T*>(w->vdw_b),
+          reinterpret_cast<T*>(ws + pl.K), reinterpret_cast<T*>(ws + pl.V));
+      EDIT_TRY(last_launch());
+    }
+    stage_mark(2, st);
     const int nb = (pl.d + 3) / 4;
     int threads = (nb * nb + 31) / 32 * 32;
     if (threads < pl.d) threads = (pl.d + 31) / 32 * 32;
@@ -357,6 +539,8 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
         reinterpret_cast<const T*>(ws + pl.K), reinterpret_cast<const T*>(ws + pl.V), pl.M, pl.C, pl.heads,
         pl.kv_chunks, reinterpret_cast<float*>(ws + pl.kvpart));
     EDIT_TRY(last_launch());
+  }
+  {
     const int per_head = pl.d * (pl.d + 1);
     const long total = static_cast<long>(pl.B) * pl.heads * per_head;
     kv_state_combine_kernel<<<grid_for(total, 256), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.kvpart),
@@ -394,6 +578,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.b1 = p.b2 = p.bk = p.b0;
     p.R = C;
     p.m_tiles_per_img = ceil_div(C, 128);
+    p.num_m_tiles = p.m_tiles_per_img;
     p.num_kb = C / 64;
     p.kb_split = p.num_kb;
     p.n_split = Cr;
@@ -429,7 +614,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     std::memset(&p, 0, sizeof(p));
     if (!map_grid(&p.a0, x, pl.B, pl.H, pl.W, C, pl.TW, pl.TH)) return EDIT_ERR_CUDA;
     p.a1 = p.a0;
-    if (!map_b(&p.b0, w->cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr))) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, w->cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr) / 2)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.bk = p.b0;
     p.num_kb = 9 * C / 64;
     p.kb_split = p.num_kb;
@@ -443,15 +628,21 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.TW = pl.TW;
     p.tiles_h = pl.tiles_h;
     p.tiles_w = pl.tiles_w;
-    p.num_tiles = pl.B * pl.tiles_h * pl.tiles_w;
+    p.num_m_tiles = pl.B * pl.tiles_h * pl.tiles_w;
     p.out = ws + pl.U;
     p.ldo = Cr;
+    if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
     p.bias[0] = w->cf3_b;
     p.gn_partials = gnpart;
     p.groups = pl.G;
     p.cpg = Cr / pl.G;
     p.status = status;
-    EDIT_TRY(gemm_conv(p, Cr, st));
+    if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
+      if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
+      EDIT_TRY(gemm_conv_reuse(p, Cr, st));
+    } else {
+      EDIT_TRY(gemm_conv(p, Cr, st));
+    }
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -477,7 +668,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
   }
   stage_mark(5, st);
   // 6. G = LeakyReLU(GN(U))
-  gn_finalize_kernel<T><<<pl.B, 32, 0, st>>>(gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
+  gn_finalize_kernel<T><<<dim3(pl.G, pl.B), 256, 0, st>>>(gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
                                               static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
                                               reinterpret_cast<float*>(ws + pl.gnstats),
                                               reinterpret_cast<float*>(ws + pl.gnss));
@@ -501,24 +692,24 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     std::memset(&p, 0, sizeof(p));
     if (!map_a(&p.a0, x, C, tok, 1, C, tok * C)) return EDIT_ERR_CUDA;
     if (!map_a(&p.a1, ws + pl.Gb, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
-    if (!map_b(&p.b0, w->q_w, C, C, C, linear_chunk(pl.bn_lin))) return EDIT_ERR_CUDA;
-    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, linear_chunk(pl.bn_lin))) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, w->q_w, C, C, C, kPairBN / 2)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, kPairBN / 2)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.b0;
     p.R = static_cast<int>(tok);
     p.m_tiles_per_img = ceil_div(tok, 128);
+    p.num_m_tiles = p.m_tiles_per_img;
     p.kb_split = C / 64;
     p.num_kb = C / 64 + ceil_div(Cr, 64);
-    p.n_split = C;
+    p.n_split = 1 << 30;  // one weight source; rows past C read as zeros
     p.N = C;
-    p.num_n_tiles = C / pl.bn_lin;
-    p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
     p.out = ws + pl.Q;
     p.ldo = C;
+    if (!map_out2d(&p.out_map, ws + pl.Q, C, tok, C)) return EDIT_ERR_CUDA;
     p.bias[0] = ws + pl.bfold;
     p.bias_f32 = 1;
     p.relu = 1;
     p.status = status;
-    EDIT_TRY(gemm_linear(p, pl.bn_lin, st));
+    EDIT_TRY(gemm_linear_pair(p, st));
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -556,6 +747,7 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
     p.b1 = p.b2 = p.bk = p.b0;
     p.R = static_cast<int>(pl.HW);
     p.m_tiles_per_img = ceil_div(pl.HW, 128);
+    p.num_m_tiles = pl.B * p.m_tiles_per_img;
     p.num_kb = pl.KP / 64;
     p.kb_split = p.num_kb;
     p.n_split = pl.heads * pl.NP;
@@ -766,6 +958,13 @@ int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit
   layout->V = static_cast<int64_t>(pl.V);
   layout->gn_stats = static_cast<int64_t>(pl.gnstats);
   layout->Sz = static_cast<int64_t>(pl.Sz);
+  layout->KT = pl.KT ? static_cast<int64_t>(pl.KT) : -1;
+  layout->VTx = pl.VTx ? static_cast<int64_t>(pl.VTx) : -1;
+  layout->K = pl.K ? static_cast<int64_t>(pl.K) : -1;
+  layout->V = pl.V ? static_cast<int64_t>(pl.V) : -1;
+  layout->Mp = pl.bf16 ? pl.Mp : pl.M;
+  layout->Wop = pl.bf16 ? pl.Wop : pl.Wo;
+  layout->NP = pl.bf16 ? pl.NP : 0;
   return EDIT_OK;
 }
 

@@ -147,31 +147,45 @@ __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int g
 // Fixed-order (deterministic) combine of the partials in fp64, then the
 // per-channel affine form of GN: scale = gamma * rstd, shift = beta - mean * scale.
 // part: [B][P][groups][2]; stats out: [B][groups][2] (mean, rstd);
-// ss out: [B][Cr][2] (scale, shift). One block per batch item.
+// ss out: [B][Cr][2] (scale, shift). One block of 256 threads per (group,
+// batch item): thread t sums partials t, t+256, ... in order, then a fixed
+// shared-memory tree.
 template <typename T>
-__global__ void gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr, long count,
-                                   float eps, const T* __restrict__ gamma, const T* __restrict__ beta,
-                                   float* __restrict__ stats, float* __restrict__ ss) {
-  const int b = blockIdx.x;
+__global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr,
+                                                          long count, float eps, const T* __restrict__ gamma,
+                                                          const T* __restrict__ beta, float* __restrict__ stats,
+                                                          float* __restrict__ ss) {
+  const int g = blockIdx.x, b = blockIdx.y;
   const int cpg = Cr / groups;
-  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
-    double s1 = 0.0, s2 = 0.0;
-    for (int i = 0; i < P; ++i) {
-      const float* q = part + ((static_cast<long>(b) * P + i) * groups + g) * 2;
-      s1 += q[0];
-      s2 += q[1];
+  __shared__ double r1[256], r2[256];
+  double s1 = 0.0, s2 = 0.0;
+  for (int i = threadIdx.x; i < P; i += 256) {
+    const float2 q = *reinterpret_cast<const float2*>(part + ((static_cast<long>(b) * P + i) * groups + g) * 2);
+    s1 += q.x;
+    s2 += q.y;
+  }
+  r1[threadIdx.x] = s1;
+  r2[threadIdx.x] = s2;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      r1[threadIdx.x] += r1[threadIdx.x + w];
+      r2[threadIdx.x] += r2[threadIdx.x + w];
     }
-    const double mean = s1 / static_cast<double>(count);
-    double var = s2 / static_cast<double>(count) - mean * mean;
-    if (var < 0.0) var = 0.0;
-    const double rstd = 1.0 / sqrt(var + static_cast<double>(eps));
+    __syncthreads();
+  }
+  const double mean = r1[0] / static_cast<double>(count);
+  double var = r2[0] / static_cast<double>(count) - mean * mean;
+  if (var < 0.0) var = 0.0;
+  const double rstd = 1.0 / sqrt(var + static_cast<double>(eps));
+  if (threadIdx.x == 0) {
     stats[(b * groups + g) * 2] = static_cast<float>(mean);
     stats[(b * groups + g) * 2 + 1] = static_cast<float>(rstd);
-    for (int c = g * cpg; c < (g + 1) * cpg; ++c) {
-      const double sc = static_cast<double>(to_f32(gamma[c])) * rstd;
-      ss[(static_cast<long>(b) * Cr + c) * 2] = static_cast<float>(sc);
-      ss[(static_cast<long>(b) * Cr + c) * 2 + 1] = static_cast<float>(static_cast<double>(to_f32(beta[c])) - mean * sc);
-    }
+  }
+  for (int c = g * cpg + threadIdx.x; c < (g + 1) * cpg; c += 256) {
+    const double sc = static_cast<double>(to_f32(gamma[c])) * rstd;
+    ss[(static_cast<long>(b) * Cr + c) * 2] = static_cast<float>(sc);
+    ss[(static_cast<long>(b) * Cr + c) * 2 + 1] = static_cast<float>(static_cast<double>(to_f32(beta[c])) - mean * sc);
   }
 }
 
@@ -312,6 +326,106 @@ __global__ void dwconv_s2_kernel(const T* __restrict__ kvp, int B, int H, int W,
 #pragma unroll
       for (int u = 0; u < VEC; ++u) dst[u] = outv[u];
     }
+  }
+}
+
+// bf16 depthwise stride-2 conv with channel-major outputs for the tensor-core
+// KV state. Token index t = i * Wop + j over a padded output grid (Wop a
+// multiple of 32; columns j >= Wo are written as 0, so they add nothing to
+// S or z). Outputs:
+//   KT [B][C][Mp]               K = ReLU(DW_k(K')), channel-major
+//   VTx[B][heads][NP][Mp]       rows r < d: V = DW_v(V') of channel h*d + r
+//   Ktok, Vtok [B][Ho*Wo][C]    token-major copies (only when non-NULL)
+// Block: one output row i, 32 output columns, 64 of the 2C channels of
+// [K' | V']; the 3 x 65-pixel input patch is staged in shared memory with
+// 16-byte loads, results are transposed through shared memory so every
+// global store is a 16-byte vector.
+__global__ void __launch_bounds__(256) dwconv_s2_t_kernel(
+    const __nv_bfloat16* __restrict__ kvp, int H, int W, int C, int d, int heads, int Wop, int Mp, int NP,
+    const __nv_bfloat16* __restrict__ kw, const __nv_bfloat16* __restrict__ kb,
+    const __nv_bfloat16* __restrict__ vw, const __nv_bfloat16* __restrict__ vb, __nv_bfloat16* __restrict__ KT,
+    __nv_bfloat16* __restrict__ VTx, __nv_bfloat16* __restrict__ Ktok, __nv_bfloat16* __restrict__ Vtok) {
+  constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
+  __shared__ __align__(16) __nv_bfloat16 in_s[3][PW][CB];
+  __shared__ __align__(16) __nv_bfloat16 out_s[CB][JT + 8];
+  const int Ho = (H + 1) / 2, Wo = (W + 1) / 2;
+  const int j0 = blockIdx.x * JT, i = blockIdx.y;
+  const int nblk = 2 * C / CB;
+  const int b = blockIdx.z / nblk, cb = blockIdx.z - b * nblk;
+  const int gc0 = cb * CB;  // first channel of [K' | V']
+  const bool isk = gc0 < C;
+  const int ch0 = isk ? gc0 : gc0 - C;
+  // stage the input patch: rows 2i-1..2i+1, columns 2*j0-1 .. 2*j0+2*JT-1
+  for (int e = threadIdx.x; e < 3 * PW * (CB / 8); e += 256) {
+    const int v = e % (CB / 8);
+    const int col = (e / (CB / 8)) % PW;
+    const int a = e / (CB / 8 * PW);
+    const int hh = 2 * i + a - 1, ww = 2 * j0 + col - 1;
+    const bool in = hh >= 0 && hh < H && ww >= 0 && ww < W;
+    const __nv_bfloat16* src = in ? kvp + ((static_cast<long>(b) * H + hh) * W + ww) * (2L * C) + gc0 + v * 8 : kvp;
+    cp_async16(&in_s[a][col][v * 8], src, in ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  const int c = threadIdx.x & (CB - 1);
+  const __nv_bfloat16* wt = isk ? kw : vw;
+  float wr[9];
+#pragma unroll
+  for (int q = 0; q < 9; ++q) wr[q] = __bfloat162float(wt[(ch0 + c) * 9 + q]);
+  const float bias = __bfloat162float((isk ? kb : vb)[ch0 + c]);
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < JT / 4; ++k) {
+    const int t = (threadIdx.x >> 6) + 4 * k;
+    const int j = j0 + t;
+    float acc = bias;
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+      for (int e = 0; e < 3; ++e) acc = fmaf(wr[a * 3 + e], __bfloat162float(in_s[a][2 * t + e][c]), acc);
+    if (isk) acc = fmaxf(acc, 0.f);
+    if (j >= Wo) acc = 0.f;
+    out_s[c][t] = __float2bfloat16_rn(acc);
+  }
+  __syncthreads();
+  {  // channel-major store: 64 rows x 32 tokens, one 16-byte vector per thread
+    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
+    const int ch = ch0 + r;
+    const long t0 = static_cast<long>(i) * Wop + j0 + q * 8;
+    __nv_bfloat16* dst;
+    if (isk) {
+      dst = KT + (static_cast<long>(b) * C + ch) * Mp + t0;
+    } else {
+      const int h = ch / d, rr = ch - h * d;
+      dst = VTx + ((static_cast<long>(b) * heads + h) * NP + rr) * Mp + t0;
+    }
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&out_s[r][q * 8]);
+  }
+  __nv_bfloat16* tok = isk ? Ktok : Vtok;
+  if (tok) {  // token-major store: 32 tokens x 64 channels
+    const int t = threadIdx.x >> 3, v = threadIdx.x & 7;
+    const int j = j0 + t;
+    if (j < Wo) {
+      __align__(16) __nv_bfloat16 tmp[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) tmp[u] = out_s[v * 8 + u][t];
+      *reinterpret_cast<uint4*>(tok + ((static_cast<long>(b) * Ho + i) * Wo + j) * C + ch0 + v * 8) =
+          *reinterpret_cast<const uint4*>(tmp);
+    }
+  }
+}
+
+// Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
+// KV state also yields z = sum_j K_j) followed by zero rows.
+__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
+  const long per = static_cast<long>(NP - d) * Mp;
+  const long total = BH * per;
+  for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long bh = e / per;
+    const long rem = e - bh * per;
+    const int r = d + static_cast<int>(rem / Mp);
+    const long t = rem % Mp;
+    VTx[(bh * NP + r) * Mp + t] = __float2bfloat16_rn(r == d ? 1.f : 0.f);
   }
 }
 

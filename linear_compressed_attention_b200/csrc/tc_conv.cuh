@@ -1,0 +1,214 @@
+// ConvFusion 3x3 conv (eq. Q^EDiT, first Conv) as an implicit GEMM on CTA
+// pairs with tap reuse: for each 64-channel block the CTA loads the input
+// patch of its 128-token tile once (3 image rows x 130 pixels, zero-filled
+// outside the grid by TMA) and feeds all 9 taps from it, each tap being the
+// same 128 x 64 operand shifted by kh * 130 + kw rows inside the patch (a
+// descriptor start offset; the swizzle follows the absolute address). Only the weights
+// stream per tap. Requires tiles of 128 consecutive pixels of one image row
+// (TW = 128, TH = 1, i.e. W >= 128).
+//
+// Roles as in the pair GEMM: warp 0 producer (both CTAs), warp 1 TMEM owner
+// and (leader) MMA issuer, warps 2..5 epilogue (U store + GroupNorm partials).
+#pragma once
+
+#include "tc_gemm.cuh"
+
+namespace edit {
+
+template <int BN, int NSPLIT, int NB>
+struct ConvPairCfg {
+  static constexpr int NCHUNK = BN / NSPLIT;
+  static constexpr int BROWS = NCHUNK / 2;
+  static_assert(BN % NSPLIT == 0 && NCHUNK % 16 == 0 && NCHUNK <= 256 && (BROWS * 128) % 1024 == 0, "pair N");
+  static constexpr int PATCH_W = 130, PATCH_H = 3;
+  static constexpr int PATCH_TX = 64 * PATCH_W * PATCH_H * 2;           // bytes one patch load brings
+  static constexpr int PATCH_BYTES = (PATCH_TX + 1023) / 1024 * 1024;  // buffer size
+  static constexpr int B_BYTES = NSPLIT * BROWS * 128;                 // per CTA per tap
+  static constexpr int ACC = (2 * BN <= 512) ? 2 : 1;
+  static constexpr int TMEM_COLS = (ACC * BN <= 128) ? 128 : (ACC * BN <= 256) ? 256 : 512;
+  static constexpr int BAR_BYTES = (2 * 2 + 2 * NB + 2 * ACC) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + 2 * PATCH_BYTES + NB * B_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
+};
+
+template <int BN, int NSPLIT, int NB>
+__global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_constant__ TcGemmParams p) {
+  using Cfg = ConvPairCfg<BN, NSPLIT, NB>;
+  constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                              // 2 patch buffers
+  uint8_t* sB = smem + 2 * Cfg::PATCH_BYTES;       // NB weight stages
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + NB * Cfg::B_BYTES);
+  uint64_t* a_empty = a_full + 2;
+  uint64_t* b_full = a_empty + 2;
+  uint64_t* b_empty = b_full + NB;
+  uint64_t* tfull_bar = b_empty + NB;
+  uint64_t* tempty_bar = tfull_bar + ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + ACC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int ncb = p.kb_per_tap;  // 64-channel blocks of the input
+  const int C = ncb * 64;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int a = 0; a < ACC; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 256);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.a1);
+    tma_prefetch_desc(&p.b0);
+  }
+  if (warp == 1) tmem_alloc2(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers
+    if (lane == 0) {
+      int ai = 0, bi = 0;
+      uint32_t aph = 0, bph = 0;
+      bool ok = true;
+      for (int pt = pair; pt < p.num_tiles && ok && !*abort_flag; pt += npairs) {
+        const TileCoord tc = decode_pair_tile<EPI_CONV>(p, pt, rank);
+        for (int cb = 0; cb < ncb && ok; ++cb) {
+          if (!mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&a_full[ai], 2 * Cfg::PATCH_TX);
+          tma2_load_4d(&p.a1, mapa_shared(smem_u32(&a_full[ai]), 0), sA + ai * Cfg::PATCH_BYTES, cb * 64,
+                       tc.w0 - 1, tc.h0 - 1, tc.img);
+          if (++ai == 2) {
+            ai = 0;
+            aph ^= 1;
+          }
+          for (int tap = 0; tap < 9; ++tap) {
+            if (!mbar_wait(&b_empty[bi], bph ^ 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&b_full[bi], 2 * Cfg::B_BYTES);
+            const uint32_t bar = mapa_shared(smem_u32(&b_full[bi]), 0);
+#pragma unroll
+            for (int s = 0; s < NSPLIT; ++s)
+              tma2_load_2d(&p.b0, bar, sB + bi * Cfg::B_BYTES + s * Cfg::BROWS * 128, tap * C + cb * 64,
+                           s * NCHUNK + rank * Cfg::BROWS);
+            if (++bi == NB) {
+              bi = 0;
+              bph ^= 1;
+            }
+          }
+        }
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      int ai = 0, bi = 0, acc = 0;
+      uint32_t aph = 0, bph = 0, acc_phase = 0;
+      bool ok = true;
+      for (int pt = pair; pt < p.num_tiles && ok && !*abort_flag; pt += npairs) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int cb = 0; cb < ncb && ok; ++cb) {
+          if (!mbar_wait(&a_full[ai], aph, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t patch = smem_u32(sA + ai * Cfg::PATCH_BYTES);
+          for (int tap = 0; tap < 9; ++tap) {
+            if (!mbar_wait(&b_full[bi], bph, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int off = (tap / 3) * Cfg::PATCH_W + tap % 3;  // first patch row of this tap's operand
+            const uint32_t a_addr = patch + off * 128;
+            const uint32_t b_addr = smem_u32(sB + bi * Cfg::B_BYTES);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t adesc = sdesc_kmajor_sw128(a_addr + k * 32);
+#pragma unroll
+              for (int s = 0; s < NSPLIT; ++s) {
+                const uint64_t bdesc = sdesc_kmajor_sw128(b_addr + s * Cfg::BROWS * 128 + k * 32);
+                umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (cb | tap | k) != 0 ? 1u : 0u);
+              }
+            }
+            umma2_commit_mc(&b_empty[bi], 0x3);
+            if (++bi == NB) {
+              bi = 0;
+              bph ^= 1;
+            }
+          }
+          if (!ok) break;
+          umma2_commit_mc(&a_empty[ai], 0x3);
+          if (++ai == 2) {
+            ai = 0;
+            aph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&tfull_bar[acc], 0x3);
+        if (++acc == ACC) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int pt = pair; pt < p.num_tiles; pt += npairs) {
+      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const TileCoord tc = decode_pair_tile<EPI_CONV>(p, pt, rank);
+      const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
+      epilogue_tile<BN, EPI_CONV>(p, tc, t_row, q, lane);
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      if (++acc == ACC) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace edit

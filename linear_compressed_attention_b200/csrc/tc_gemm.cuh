@@ -12,6 +12,12 @@
 //              per-tile GroupNorm partial sums.
 //  EPI_APPLY   Linear attention apply, eq. (y_i): per head h, [num | den] =
 //              Q_h [S_h | z_h] and y = num / (den + eps) fused into the store.
+//  EPI_KVSTATE Linear attention state, eq. (y_i): per (image, head, chunk of
+//              compressed tokens) tile, D = K_h^T [V_h | 1 | 0] with the
+//              tokens as the reduction dimension (both operands stored
+//              channel-major, so K-major for the MMA); rows a < d, columns
+//              c <= d of D are a partial [S_h | z_h], written in fp32 for a
+//              fixed-order combine.
 //
 // Block: 192 threads. Warp 0 = TMA producer (one lane), warp 1 = TMEM owner
 // and MMA issuer (one lane), warps 2..5 = epilogue (tcgen05.ld of the warp's
@@ -25,7 +31,7 @@
 
 namespace edit {
 
-enum { EPI_LINEAR = 0, EPI_CONV = 1, EPI_APPLY = 2 };
+enum { EPI_LINEAR = 0, EPI_CONV = 1, EPI_APPLY = 2, EPI_KVSTATE = 3 };
 
 struct TcGemmParams {
   // A sources (3D maps [img][rows][K], box 64 x 128 x 1): a0 gives the first
@@ -36,8 +42,13 @@ struct TcGemmParams {
   // [s*n_split, (s+1)*n_split) for the first kb_split k-blocks; bk holds the
   // rest of K (single N source only). EPI_APPLY: b0 = [img*heads*BN][KP].
   CUtensorMap b0, b1, b2, bk;
+  // Output map for the staged (TMA store) epilogue of the pair kernel:
+  // EPI_LINEAR: 2D [rows][N] box 64 x 32; EPI_CONV: 4D [img][H][W][Cr] box
+  // 64 x min(TW,32) x (32/min(TW,32)) x 1. Both 128-byte swizzled.
+  CUtensorMap out_map;
   int R;            // rows per image (A)
   int m_tiles_per_img;
+  int num_m_tiles;  // real 128-row tiles (the pair kernel may add one empty tile)
   int num_kb;       // 64-wide k-blocks
   int kb_split;
   int n_split;
@@ -46,9 +57,12 @@ struct TcGemmParams {
   int num_tiles;
   // implicit-conv geometry (EPI_CONV)
   int H, W, TH, TW, tiles_h, tiles_w, kb_per_tap;
-  // apply geometry (EPI_APPLY)
+  // apply / KV-state geometry (EPI_APPLY, EPI_KVSTATE)
   int d, heads;
   float eps;
+  int kv_rows_per_img;  // EPI_KVSTATE: A rows per image (= C)
+  int kb_per_chunk, num_chunks;
+  float* kv_part;       // EPI_KVSTATE: [img][heads][num_chunks][d][d+1]
   // epilogue
   void* out;        // bf16, row (img*R + r) at out + row*ldo (+ column offset)
   long ldo;
@@ -89,13 +103,47 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 struct TileCoord {
   int m_tile, n_tile, img, r0, h0, w0;
+  int kb0, nkb;  // k-block range of this tile
 };
+
+template <int EPI>
+__device__ __forceinline__ TileCoord decode_m(const TcGemmParams& p, TileCoord t);
 
 template <int EPI>
 __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int tile) {
   TileCoord t;
+  t.kb0 = 0;
+  t.nkb = p.num_kb;
+  if (EPI == EPI_KVSTATE) {  // tile = (img * heads + head) * num_chunks + chunk
+    const int chunk = tile % p.num_chunks;
+    const int ih = tile / p.num_chunks;
+    t.img = ih / p.heads;
+    t.n_tile = ih - t.img * p.heads;
+    t.m_tile = chunk;
+    t.kb0 = chunk * p.kb_per_chunk;
+    t.nkb = min(p.kb_per_chunk, p.num_kb - t.kb0);
+    t.r0 = t.h0 = t.w0 = 0;
+    return t;
+  }
   t.m_tile = tile / p.num_n_tiles;
   t.n_tile = tile - t.m_tile * p.num_n_tiles;
+  return decode_m<EPI>(p, t);
+}
+
+// Pair tile pt of the 2-CTA kernel: CTA `rank` takes 128-row tile 2*mp + rank.
+template <int EPI>
+__device__ __forceinline__ TileCoord decode_pair_tile(const TcGemmParams& p, int pt, int rank) {
+  TileCoord t;
+  t.kb0 = 0;
+  t.nkb = p.num_kb;
+  const int mp = pt / p.num_n_tiles;
+  t.n_tile = pt - mp * p.num_n_tiles;
+  t.m_tile = 2 * mp + rank;
+  return decode_m<EPI>(p, t);
+}
+
+template <int EPI>
+__device__ __forceinline__ TileCoord decode_m(const TcGemmParams& p, TileCoord t) {
   if (EPI == EPI_CONV) {
     const int per_img = p.tiles_h * p.tiles_w;
     t.img = t.m_tile / per_img;
@@ -126,10 +174,181 @@ __device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float (&
   if (nvalid >= 16) d[1] = o1;
 }
 
+// Epilogue of one tile for the thread owning TMEM lane (row) r = q*32 + lane:
+// read the accumulator columns, apply the step's output function, store.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileCoord& tc, uint32_t t_row, int q,
+                                              int lane) {
+  const int r = q * 32 + lane;
+  long row;
+  bool valid;
+  if (EPI == EPI_CONV) {
+    const int hh = tc.h0 + r / p.TW, ww = tc.w0 + r % p.TW;
+    valid = tc.m_tile < p.num_m_tiles && hh < p.H && ww < p.W;
+    row = (static_cast<long>(tc.img) * p.H + hh) * p.W + ww;
+  } else {
+    valid = tc.m_tile < p.num_m_tiles && tc.r0 + r < p.R;
+    row = static_cast<long>(tc.img) * p.R + tc.r0 + r;
+  }
+  if (EPI == EPI_KVSTATE) {
+    const int dd = p.d;
+    float* prow = p.kv_part +
+                  ((static_cast<long>(tc.img * p.heads + tc.n_tile) * p.num_chunks + tc.m_tile) * dd + r) * (dd + 1);
+#pragma unroll 1
+    for (int c = 0; c < (dd + 16) / 16; ++c) {
+      float v[16];
+      tmem_ld16(t_row + c * 16, v);
+      if (r < dd) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (c * 16 + i <= dd) prow[c * 16 + i] = v[i];
+      }
+    }
+  } else if (EPI == EPI_APPLY) {
+    // columns 0..d-1: numerator; column d: denominator
+    float v[16];
+    tmem_ld16(t_row + (p.d / 16) * 16, v);
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i == p.d % 16) den = v[i];
+    const float inv = 1.f / (den + p.eps);
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ldo + tc.n_tile * p.d;
+#pragma unroll 1
+    for (int c = 0; c < (p.d + 15) / 16; ++c) {
+      tmem_ld16(t_row + c * 16, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] *= inv;
+      if (valid) store_bf16x16(orow + c * 16, v, p.d - c * 16);
+    }
+  } else {
+    const int n0 = tc.n_tile * BN;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ldo + n0;
+    float s1 = 0.f, s2 = 0.f;  // GroupNorm running sums of the current group
+    int g_cur = 0;
+    float* gpart = nullptr;
+    const bool gn_on = EPI == EPI_CONV && tc.m_tile < p.num_m_tiles;
+    if (gn_on) {
+      const int per_img = p.tiles_h * p.tiles_w;
+      const int t_in_img = tc.m_tile - tc.img * per_img;
+      gpart = p.gn_partials + ((static_cast<long>(tc.img) * per_img + t_in_img) * 4 + q) * p.groups * 2;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 16; ++c) {
+      const int n = n0 + c * 16;
+      float v[16];
+      tmem_ld16(t_row + c * 16, v);
+      const int src = n / p.n_split;
+      const void* bias = (src < 3 && n < p.N) ? p.bias[src] : nullptr;
+      if (bias) {
+        const int j0 = n - src * p.n_split;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j0 + i]
+                             : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
+      }
+      if (p.relu) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.f);
+      }
+      if (EPI == EPI_CONV) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int g = (c * 16 + i) / p.cpg;  // warp-uniform
+          if (g != g_cur) {
+            const float t1 = warp_sum(s1), t2 = warp_sum(s2);
+            if (lane == 0 && gn_on) {
+              gpart[g_cur * 2] = t1;
+              gpart[g_cur * 2 + 1] = t2;
+            }
+            s1 = s2 = 0.f;
+            g_cur = g;
+          }
+          const float x = valid ? v[i] : 0.f;
+          s1 += x;
+          s2 += x * x;
+        }
+      }
+      if (valid && n < p.N) store_bf16x16(orow + c * 16, v, 16);
+    }
+    if (EPI == EPI_CONV) {
+      const float t1 = warp_sum(s1), t2 = warp_sum(s2);
+      if (lane == 0 && gn_on) {
+        gpart[g_cur * 2] = t1;
+        gpart[g_cur * 2 + 1] = t2;
+      }
+    }
+  }
+}
+
+// A and B loads of k-block kb of a (1-CTA) tile into one pipeline stage.
+template <int BN, int NSPLIT, int EPI, bool PAIR>
+__device__ __forceinline__ void load_stage(const TcGemmParams& p, const TileCoord& tc, int kb, uint8_t* dA,
+                                           uint8_t* dB, uint64_t* bar, int rank) {
+  constexpr int NCHUNK = BN / NSPLIT;
+  constexpr int BROWS = PAIR ? NCHUNK / 2 : NCHUNK;  // B rows of one chunk in this CTA
+  const uint32_t bar_addr = PAIR ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar);  // pair: leader's barrier
+  // ---- A: 128 rows of this CTA's tile
+  if (EPI == EPI_CONV) {
+    const int tap = kb / p.kb_per_tap;
+    const int c0 = (kb - tap * p.kb_per_tap) * 64;
+    const int kh = tap / 3, kw = tap - 3 * (tap / 3);
+    if (PAIR)
+      tma2_load_4d(&p.a0, bar_addr, dA, c0, tc.w0 + kw - 1, tc.h0 + kh - 1, tc.img);
+    else
+      tma_load_4d(&p.a0, bar, dA, c0, tc.w0 + kw - 1, tc.h0 + kh - 1, tc.img);
+  } else {
+    const CUtensorMap* am = &p.a0;
+    int x = kb * 64, y = tc.r0, z = tc.img;
+    if (EPI == EPI_APPLY) {
+      x = tc.n_tile * p.d + kb * 64;
+    } else if (EPI == EPI_KVSTATE) {
+      x = (tc.kb0 + kb) * 64;
+      y = tc.img * p.kv_rows_per_img + tc.n_tile * p.d;
+      z = 0;
+    } else if (kb >= p.kb_split) {
+      am = &p.a1;
+      x = (kb - p.kb_split) * 64;
+    }
+    if (PAIR)
+      tma2_load_3d(am, bar_addr, dA, x, y, z);
+    else
+      tma_load_3d(am, bar, dA, x, y, z);
+  }
+  // ---- B: NSPLIT chunks of NCHUNK output columns (this CTA's half in a pair)
+#pragma unroll
+  for (int s = 0; s < NSPLIT; ++s) {
+    const CUtensorMap* bm;
+    int x, y;
+    if (EPI == EPI_APPLY || EPI == EPI_KVSTATE) {
+      bm = &p.b0;
+      x = (EPI == EPI_KVSTATE ? tc.kb0 + kb : kb) * 64;
+      y = (tc.img * p.heads + tc.n_tile) * BN + s * NCHUNK;
+    } else {
+      const int n = tc.n_tile * BN + s * NCHUNK + (PAIR ? rank * BROWS : 0);
+      if (kb >= p.kb_split) {
+        bm = &p.bk;
+        x = (kb - p.kb_split) * 64;
+        y = n;
+      } else {
+        const int src = n / p.n_split;
+        bm = src == 0 ? &p.b0 : (src == 1 ? &p.b1 : &p.b2);
+        x = kb * 64;
+        y = n - src * p.n_split;
+      }
+    }
+    uint8_t* d = dB + s * BROWS * 128;
+    if (PAIR)
+      tma2_load_2d(bm, bar_addr, d, x, y);
+    else
+      tma_load_2d(bm, bar, d, x, y);
+  }
+}
+
 template <int BN, int NSPLIT, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   using Cfg = TcGemmCfg<BN, NSPLIT, STAGES>;
-  constexpr int BM = Cfg::BM, NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
+  constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -171,41 +390,11 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
         const TileCoord tc = decode_tile<EPI>(p, tile);
-        const CUtensorMap* bmap = &p.b0;
-        int brow0;
-        if (EPI == EPI_APPLY) {
-          brow0 = (tc.img * p.heads + tc.n_tile) * BN;
-        } else {
-          const int n0 = tc.n_tile * BN;
-          const int src = n0 / p.n_split;
-          bmap = src == 0 ? &p.b0 : (src == 1 ? &p.b1 : &p.b2);
-          brow0 = n0 - src * p.n_split;
-        }
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = 0; kb < tc.nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status)) break;
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
-          uint8_t* dA = sA + stage * Cfg::A_BYTES;
-          uint8_t* dB = sB + stage * Cfg::B_BYTES;
-          if (EPI == EPI_CONV) {
-            const int tap = kb / p.kb_per_tap;
-            const int c0 = (kb - tap * p.kb_per_tap) * 64;
-            const int kh = tap / 3, kw = tap - 3 * (tap / 3);
-            tma_load_4d(&p.a0, &full_bar[stage], dA, c0, tc.w0 + kw - 1, tc.h0 + kh - 1, tc.img);
-          } else if (EPI == EPI_APPLY) {
-            tma_load_3d(&p.a0, &full_bar[stage], dA, tc.n_tile * p.d + kb * 64, tc.r0, tc.img);
-          } else if (kb < p.kb_split) {
-            tma_load_3d(&p.a0, &full_bar[stage], dA, kb * 64, tc.r0, tc.img);
-          } else {
-            tma_load_3d(&p.a1, &full_bar[stage], dA, (kb - p.kb_split) * 64, tc.r0, tc.img);
-          }
-#pragma unroll
-          for (int s = 0; s < NSPLIT; ++s) {
-            if (kb < p.kb_split)
-              tma_load_2d(bmap, &full_bar[stage], dB + s * NCHUNK * 128, kb * 64, brow0 + s * NCHUNK);
-            else
-              tma_load_2d(&p.bk, &full_bar[stage], dB + s * NCHUNK * 128, (kb - p.kb_split) * 64,
-                          brow0 + s * NCHUNK);
-          }
+          load_stage<BN, NSPLIT, EPI, false>(p, tc, kb, sA + stage * Cfg::A_BYTES, sB + stage * Cfg::B_BYTES,
+                                             &full_bar[stage], 0);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -232,8 +421,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        const int nkb = decode_tile<EPI>(p, tile).nkb;
         bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
             ok = false;
             break;
@@ -268,99 +458,14 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const TileCoord tc = decode_tile<EPI>(p, tile);
-      long row;
-      bool valid;
-      if (EPI == EPI_CONV) {
-        const int hh = tc.h0 + r / p.TW, ww = tc.w0 + r % p.TW;
-        valid = hh < p.H && ww < p.W;
-        row = (static_cast<long>(tc.img) * p.H + hh) * p.W + ww;
-      } else {
-        valid = tc.r0 + r < p.R;
-        row = static_cast<long>(tc.img) * p.R + tc.r0 + r;
-      }
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      if (EPI == EPI_APPLY) {
-        // columns 0..d-1: numerator; column d: denominator
-        float v[16];
-        tmem_ld16(t_row + (p.d / 16) * 16, v);
-        float den = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (i == p.d % 16) den = v[i];
-        const float inv = 1.f / (den + p.eps);
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ldo + tc.n_tile * p.d;
-#pragma unroll 1
-        for (int c = 0; c < (p.d + 15) / 16; ++c) {
-          tmem_ld16(t_row + c * 16, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= inv;
-          if (valid) store_bf16x16(orow + c * 16, v, p.d - c * 16);
-        }
-      } else {
-        const int n0 = tc.n_tile * BN;
-        const int src = n0 / p.n_split;
-        const void* bias = p.bias[src];
-        const int bias_off = n0 - src * p.n_split;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ldo + n0;
-        float s1 = 0.f, s2 = 0.f;  // GroupNorm running sums of the current group
-        int g_cur = 0;
-        float* gpart = nullptr;
-        if (EPI == EPI_CONV) {
-          const int per_img = p.tiles_h * p.tiles_w;
-          const int t_in_img = tc.m_tile - tc.img * per_img;
-          gpart = p.gn_partials + ((static_cast<long>(tc.img) * per_img + t_in_img) * 4 + q) * p.groups * 2;
-        }
-#pragma unroll 1
-        for (int c = 0; c < BN / 16; ++c) {
-          float v[16];
-          tmem_ld16(t_row + c * 16, v);
-          if (bias) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int j = bias_off + c * 16 + i;
-              v[i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j]
-                                 : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j]);
-            }
-          }
-          if (p.relu) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.f);
-          }
-          if (EPI == EPI_CONV) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int g = (c * 16 + i) / p.cpg;  // warp-uniform
-              if (g != g_cur) {
-                const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-                if (lane == 0) {
-                  gpart[g_cur * 2] = t1;
-                  gpart[g_cur * 2 + 1] = t2;
-                }
-                s1 = s2 = 0.f;
-                g_cur = g;
-              }
-              const float x = valid ? v[i] : 0.f;
-              s1 += x;
-              s2 += x * x;
-            }
-          }
-          if (valid && n0 + c * 16 < p.N) store_bf16x16(orow + c * 16, v, 16);
-        }
-        if (EPI == EPI_CONV) {
-          const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-          if (lane == 0) {
-            gpart[g_cur * 2] = t1;
-            gpart[g_cur * 2 + 1] = t2;
-          }
-        }
-      }
+      epilogue_tile<BN, EPI>(p, tc, t_row, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == ACC) {
@@ -375,6 +480,284 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ===================================================================== pairs
+// Two-SM version (cta_group::2, cluster of 2): pair tile = 256 rows (128 per
+// CTA) x BN columns. Each CTA loads its own 128 A rows and half of each B
+// chunk into its own shared memory; TMA completion is counted on the
+// leader's (rank 0) full barrier; the leader's single thread issues the
+// M = 256 MMAs and multicasts each commit to both CTAs' barriers; each CTA's
+// epilogue drains its own TMEM rows and arrives on the leader's TMEM-empty
+// barrier (256 arrivals). Per CTA, shared-memory operand traffic per MMA
+// column is half that of the 1-CTA kernel.
+template <int BN, int NSPLIT, int STAGES>
+struct TcPairCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int NCHUNK = BN / NSPLIT;  // MMA N
+  static constexpr int BROWS = NCHUNK / 2;    // B rows per chunk per CTA
+  static_assert(BN % NSPLIT == 0 && NCHUNK % 16 == 0 && NCHUNK <= 256 && (BROWS * 128) % 1024 == 0, "pair N");
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = NSPLIT * BROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+  static constexpr int ACC = (2 * BN <= 512) ? 2 : 1;
+  static constexpr int TMEM_COLS = (ACC * BN <= 128) ? 128 : (ACC * BN <= 256) ? 256 : 512;
+  static_assert(ACC * BN <= 512, "TMEM");
+  static constexpr int STG_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x (32 rows x 128 B)
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
+};
+
+// Staged epilogue (EPI_LINEAR / EPI_CONV): per 64-column chunk, one 64-wide
+// TMEM load, bias / ReLU / GroupNorm partials in registers, a 128B-swizzled
+// 32 x 128-byte staging block per warp (double-buffered), and one TMA tensor
+// store of the block, so global writes leave the SM as full lines.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, const TileCoord& tc, uint32_t t_row,
+                                                     int q, int lane, uint8_t* stg, int& sbuf) {
+  const int r = q * 32 + lane;
+  const bool real = tc.m_tile < p.num_m_tiles;
+  bool valid;
+  if (EPI == EPI_CONV) {
+    const int hh = tc.h0 + r / p.TW, ww = tc.w0 + r % p.TW;
+    valid = real && hh < p.H && ww < p.W;
+  } else {
+    valid = real && tc.r0 + r < p.R;
+  }
+  const int n0 = tc.n_tile * BN;
+  float s1 = 0.f, s2 = 0.f;  // GroupNorm running sums of the current group
+  int g_cur = 0;
+  float* gpart = nullptr;
+  const bool gn_on = EPI == EPI_CONV && real;
+  if (gn_on) {
+    const int per_img = p.tiles_h * p.tiles_w;
+    const int t_in_img = tc.m_tile - tc.img * per_img;
+    gpart = p.gn_partials + ((static_cast<long>(tc.img) * per_img + t_in_img) * 4 + q) * p.groups * 2;
+  }
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    float v[64];
+    tmem_ld64(t_row + c0, v);
+#pragma unroll
+    for (int g16 = 0; g16 < 4; ++g16) {
+      const int col = c0 + 16 * g16;
+      const int n = n0 + col;
+      const int src = n / p.n_split;
+      const void* bias = (col < BN && src < 3 && n < p.N) ? p.bias[src] : nullptr;
+      if (bias) {
+        const int j0 = n - src * p.n_split;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[16 * g16 + i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j0 + i]
+                                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
+      }
+    }
+    if (p.relu) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+    }
+    if (EPI == EPI_CONV) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const int col = c0 + i;
+        if (col < BN) {                      // warp-uniform
+          const int g = col / p.cpg;
+          if (g != g_cur) {
+            const float t1 = warp_sum(s1), t2 = warp_sum(s2);
+            if (lane == 0 && gn_on) {
+              gpart[g_cur * 2] = t1;
+              gpart[g_cur * 2 + 1] = t2;
+            }
+            s1 = s2 = 0.f;
+            g_cur = g;
+          }
+          const float x = valid ? v[i] : 0.f;
+          s1 += x;
+          s2 += x * x;
+        }
+      }
+    }
+    // stage this warp's 32 rows x 64 columns (bf16) in 128B-swizzled order
+    if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
+    __syncwarp();
+    uint8_t* buf = stg + sbuf * 4096;
+    uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 128);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint4 o;
+      o.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      o.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      o.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      o.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      rowp[j ^ (lane & 7)] = o;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && real) {
+      if (EPI == EPI_CONV) {
+        const int r0w = q * 32;
+        const int ws = tc.w0 + r0w % p.TW, hs = tc.h0 + r0w / p.TW;
+        if (ws < p.W && hs < p.H) tma_store_4d(&p.out_map, buf, c0, ws, hs, tc.img);
+      } else {
+        if (tc.r0 + q * 32 < p.R) tma_store_2d(&p.out_map, buf, n0 + c0, tc.img * p.R + tc.r0 + q * 32);
+      }
+      bulk_commit();
+    }
+    sbuf ^= 1;
+  }
+  if (EPI == EPI_CONV) {
+    const float t1 = warp_sum(s1), t2 = warp_sum(s2);
+    if (lane == 0 && gn_on) {
+      gpart[g_cur * 2] = t1;
+      gpart[g_cur * 2 + 1] = t2;
+    }
+  }
+}
+
+template <int BN, int NSPLIT, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_constant__ TcGemmParams p) {
+  using Cfg = TcPairCfg<BN, NSPLIT, STAGES>;
+  constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* stg_base = sB + STAGES * Cfg::B_BYTES;  // 1024-byte aligned
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + ACC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < ACC; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 256);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.a0);
+    tma_prefetch_desc(&p.b0);
+  }
+  if (warp == 1) tmem_alloc2(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int pt = pair; pt < p.num_tiles && !*abort_flag; pt += npairs) {
+        const TileCoord tc = decode_pair_tile<EPI>(p, pt, rank);
+        for (int kb = 0; kb < tc.nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status)) break;
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
+          load_stage<BN, NSPLIT, EPI, true>(p, tc, kb, sA + stage * Cfg::A_BYTES, sB + stage * Cfg::B_BYTES,
+                                            &full_bar[stage], rank);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int pt = pair; pt < p.num_tiles && !*abort_flag; pt += npairs) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t adesc = sdesc_kmajor_sw128(a_addr + k * 32);
+#pragma unroll
+            for (int s = 0; s < NSPLIT; ++s) {
+              const uint64_t bdesc = sdesc_kmajor_sw128(b_addr + s * Cfg::BROWS * 128 + k * 32);
+              umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+            }
+          }
+          umma2_commit_mc(&empty_bar[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&tfull_bar[acc], 0x3);
+        if (++acc == ACC) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    uint8_t* stg = stg_base + q * 8192;
+    int sbuf = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int pt = pair; pt < p.num_tiles; pt += npairs) {
+      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const TileCoord tc = decode_pair_tile<EPI>(p, pt, rank);
+      const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
+      epilogue_tile_staged<BN, EPI>(p, tc, t_row, q, lane, stg, sbuf);
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      if (++acc == ACC) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    if (lane == 0) bulk_wait_all();  // staged stores finished before shared memory is released
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

@@ -115,7 +115,9 @@ def test_status_strings():
 def test_workspace_layout_offsets():
     s = fake_struct()
     lay = bd.edit_attn_workspace_layout(1, 64, 64, 1152, 16, s)
-    offs = [lay[k] for k in ("U", "G", "Q", "KVp", "K", "V", "gn_stats", "Sz")]
+    offs = [lay[k] for k in ("U", "G", "Q", "KVp", "KT", "VTx", "gn_stats", "Sz")]
+    assert lay["K"] == -1 and lay["V"] == -1          # bf16 EDiT keeps K, V channel-major only
+    assert lay["Mp"] == 32 * 32 and lay["Wop"] == 32 and lay["NP"] == 80
     assert lay["status"] == 0
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)

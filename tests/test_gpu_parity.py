@@ -35,6 +35,25 @@ def run_edit(cfg, d):
     return layer, out.float().cpu().numpy()
 
 
+def get_kv(layer, cfg):
+    """K, V [B, M, C] from the workspace (token-major copy or the channel-major
+    tensor-core operands, which also carry the ones row and zero padding)."""
+    B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+    Ho, Wo, dh = (H + 1) // 2, (W + 1) // 2, C // heads
+    M = Ho * Wo
+    lay = layer.layout
+    if lay["K"] >= 0:
+        return (layer.intermediate("K", (B, M, C)).float().cpu(), layer.intermediate("V", (B, M, C)).float().cpu())
+    Mp, Wop, NP = lay["Mp"], lay["Wop"], lay["NP"]
+    KT = layer.intermediate("KT", (B, C, Ho, Wop)).float().cpu()
+    VTx = layer.intermediate("VTx", (B, heads, NP, Ho, Wop)).float().cpu()
+    assert torch.all(KT[..., Wo:] == 0) and torch.all(VTx[:, :, :dh, :, Wo:] == 0)
+    assert torch.all(VTx[:, :, dh] == 1) and torch.all(VTx[:, :, dh + 1:] == 0)
+    K = KT[..., :Wo].reshape(B, C, M).transpose(1, 2)
+    V = VTx[:, :, :dh, :, :Wo].reshape(B, C, M).transpose(1, 2)
+    return K, V
+
+
 def check_edit(cfg, d, intermediates=True):
     layer, y = run_edit(cfg, d)
     yo, it = O.edit_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"], return_intermediates=True)
@@ -46,8 +65,9 @@ def check_edit(cfg, d, intermediates=True):
         f32 = torch.float32
         errs["U"] = max_rel(layer.intermediate("U", (B, H, W, Cr)).float().cpu(), it["U"])
         errs["Q"] = max_rel(layer.intermediate("Q", (B, N, C)).float().cpu(), it["Q"])
-        errs["K"] = max_rel(layer.intermediate("K", (B, M, C)).float().cpu(), it["K"])
-        errs["V"] = max_rel(layer.intermediate("V", (B, M, C)).float().cpu(), it["V"])
+        Kg, Vg = get_kv(layer, cfg)
+        errs["K"] = max_rel(Kg, it["K"])
+        errs["V"] = max_rel(Vg, it["V"])
         Sz = layer.intermediate("Sz", (B, heads, dh, dh + 1), f32).cpu().numpy()
         errs["S"] = max_rel(Sz[..., :dh], it["S"])
         errs["z"] = max_rel(Sz[..., dh], it["z"])
@@ -120,8 +140,7 @@ def test_shared_kv_weights_literal_reading():
     d = make_inputs(**cfg)
     d["v_w"], d["v_b"], d["vdw_w"], d["vdw_b"] = d["k_w"], d["k_b"], d["kdw_w"], d["kdw_b"]
     layer, _ = run_edit(cfg, d)
-    K = layer.intermediate("K", (1, 16, 128)).float()
-    V = layer.intermediate("V", (1, 16, 128)).float()
+    K, V = get_kv(layer, cfg)
     assert torch.equal(K, torch.relu(V))
 
 
