@@ -71,7 +71,8 @@ enum {
   EDIT_ERR_WORKSPACE = -5, /* workspace smaller than the query returned            */
   EDIT_ERR_CUDA = -6,      /* a CUDA runtime/driver call or launch failed          */
   EDIT_ERR_TIMEOUT = -7,   /* (device) a bounded wait ran out; results invalid     */
-  EDIT_ERR_UNSUPPORTED = -8 /* shape outside what the kernels are built for        */
+  EDIT_ERR_UNSUPPORTED = -8, /* shape outside what the kernels are built for       */
+  EDIT_ERR_SCRATCH = -9     /* request needs more than the library's fixed scratch */
 };
 
 /* Weights and declared constants of one EDiT layer. Shapes (row-major):
@@ -179,6 +180,37 @@ enum { EDIT_STAGE_EVENTS_EDIT = 9, EDIT_STAGE_EVENTS_MM = 12 };
 EDIT_API int edit_attn_set_stage_events(void *const *events, int n);
 
 EDIT_API uint64_t edit_attn_kernel_launches(void);
+
+/* Linear attention step without any caller-provided scratch (the paper has
+ * no counterpart; this is a deployment convenience).
+ *
+ * Some callers cannot allocate device memory at the point where they run the
+ * layer: code running inside a framework's memory pool that forbids ad-hoc
+ * cudaMalloc, plugins handed only their input and output buffers, or hosts
+ * that must not grow device memory after start-up. For them this entry point
+ * computes y from q, k, v exactly like the last step of edit_attn_forward
+ * (per head: S = sum_j k_j^T v_j, z = sum_j k_j, y_i = q_i S / (q_i z + eps))
+ * using a scratch array compiled into the library instead of a workspace.
+ *
+ *   q, out [B, N, C]; k, v [B, M, C] (device, dtype `dtype`, 16-byte aligned);
+ *   heads divide C; the call is asynchronous on `stream`.
+ *
+ * The scratch is a static device array of EDIT_NOALLOC_SCRATCH_BYTES bytes
+ * that every GPU which loads the library keeps until the process exits. A
+ * call needs B * heads * d * (d + 1) * 4 bytes for two chunks of partial sums
+ * plus the combined [S | z] (d = C / heads, at least 3 such blocks in all);
+ * larger requests return EDIT_ERR_SCRATCH without launching anything. The
+ * library never calls cudaMalloc, cudaFree or any allocating routine here.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's
+ * contents (every value a call reads is written earlier in the same call), so
+ * calls whose kernels may overlap on the GPU (different streams without
+ * ordering) race on it: order them on one stream. */
+#define EDIT_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+EDIT_API int edit_linear_attention_noalloc(const void *q, const void *k, const void *v, int B, int N, int M, int C,
+                                           int heads, int dtype, float attn_eps, void *out, void *stream);
 
 #ifdef __cplusplus
 }

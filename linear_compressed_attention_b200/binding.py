@@ -21,7 +21,7 @@ WEIGHT_NAMES = ("cf3_w", "cf3_b", "gn_gamma", "gn_beta", "cf1_w", "cf1_b", "q_w"
 TEXT_NAMES = ("tq_w", "tq_b", "tk_w", "tk_b", "tv_w", "tv_b")
 EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_bytes", "mmedit_hybrid_forward",
            "edit_attn_read_status", "edit_status_string", "edit_attn_workspace_layout",
-           "edit_attn_set_stage_events", "edit_attn_kernel_launches")
+           "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc")
 STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
 
 
@@ -74,6 +74,8 @@ def lib():
     L.edit_attn_set_stage_events.restype = i
     L.edit_attn_kernel_launches.argtypes = []
     L.edit_attn_kernel_launches.restype = ctypes.c_uint64
+    L.edit_linear_attention_noalloc.argtypes = [p, p, p, i, i, i, i, i, i, ctypes.c_float, p, p]
+    L.edit_linear_attention_noalloc.restype = i
     _lib = L
     return L
 
@@ -180,6 +182,13 @@ def edit_attn_set_stage_events(handles) -> int:
 
 def edit_attn_kernel_launches() -> int:
     return int(lib().edit_attn_kernel_launches())
+
+
+def edit_linear_attention_noalloc(q, k, v, B, N, M, C, heads, dtype_code, attn_eps, out, stream=None) -> int:
+    """Linear attention step with the library's static scratch (no workspace);
+    q, out [B, N, C], k, v [B, M, C] device tensors. Returns the status code."""
+    return int(lib().edit_linear_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), B, N, M, C, heads, dtype_code,
+                                                   float(attn_eps), _ptr(out), _stream(stream)))
 
 
 # ----------------------------------------------------------- convenience

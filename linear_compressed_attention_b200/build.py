@@ -7,9 +7,10 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "edit_attn.cu")
+SRCS = [os.path.join(PKG, "csrc", "edit_attn.cu"), os.path.join(PKG, "csrc", "edit_noalloc.cu")]
 OUT = os.path.join(PKG, "libedit_attn.so")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("edit_attn.cu", "common.cuh", "tc_gemm.cuh", "simt_kernels.cuh")]
+DEPS = [os.path.join(PKG, "csrc", f) for f in ("edit_attn.cu", "edit_noalloc.cu", "common.cuh", "tc_gemm.cuh",
+                                                "tc_conv.cuh", "simt_kernels.cuh")]
 DEPS.append(os.path.join(ROOT, "include", "edit_attn.h"))
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -33,7 +34,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
     tmp = OUT + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-o", tmp, SRC]
+    cmd = [nvcc(), *NVCC_FLAGS, "-o", tmp, *SRCS]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)

@@ -940,6 +940,7 @@ const char* edit_status_string(int status) {
     case EDIT_ERR_CUDA: return "CUDA error";
     case EDIT_ERR_TIMEOUT: return "device wait timed out";
     case EDIT_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+    case EDIT_ERR_SCRATCH: return "request exceeds the library's fixed scratch";
   }
   return "unknown status";
 }

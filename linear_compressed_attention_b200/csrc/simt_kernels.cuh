@@ -8,6 +8,7 @@
 #include "common.cuh"
 
 namespace edit {
+namespace {  // internal linkage: each translation unit that uses these keeps its own copy
 
 // ====================================================================== GEMM
 // out[m, n] = act(sum_k A(m, k) * Bw(n, k) + bias(n)), fp32.
@@ -655,4 +656,5 @@ __global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
   }
 }
 
+}  // namespace
 }  // namespace edit

@@ -122,3 +122,14 @@ def test_workspace_layout_offsets():
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)
     assert max(offs) < bd.edit_attn_workspace_bytes(1, 64, 64, 1152, 16, s)
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch():
+    L = bd.lib()
+    p = lambda a: ctypes.c_void_p(a)  # noqa: E731  (never dereferenced: rejected before any launch)
+    # 64 images x 16 heads x 72 x 73 x 4 B per block > the fixed scratch
+    rc = L.edit_linear_attention_noalloc(p(0x1000), p(0x2000), p(0x3000), 64, 4096, 1024, 1152, 16, bd.EDIT_BF16,
+                                         ctypes.c_float(1e-6), p(0x4000), None)
+    assert rc == -9 and bd.status_string(rc) == "request exceeds the library's fixed scratch"
+    assert L.edit_linear_attention_noalloc(None, p(0x2000), p(0x3000), 1, 8, 4, 64, 2, 0, ctypes.c_float(1e-6),
+                                           p(0x4000), None) == -1
