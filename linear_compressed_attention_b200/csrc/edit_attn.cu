@@ -130,6 +130,7 @@ struct Plan {
   int es;  // bytes per element of activations/weights
   int TH, TW, tiles_h, tiles_w;
   int gn_P;       // GroupNorm partials per image
+  int gn_chunk;   // bf16: tokens per GroupNorm partial
   int kv_chunks;  // KV-state partials per (image, head)
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
@@ -184,7 +185,8 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.TH = 128 / pl.TW;
     pl.tiles_h = (H + pl.TH - 1) / pl.TH;
     pl.tiles_w = (W + pl.TW - 1) / pl.TW;
-    pl.gn_P = pl.tiles_h * pl.tiles_w * 4;
+    pl.gn_chunk = 32;  // tokens per GroupNorm partial (many blocks: the pass is latency-bound otherwise)
+    pl.gn_P = static_cast<int>((pl.HW + pl.gn_chunk - 1) / pl.gn_chunk);
     // [S_h | z_h] has d + 1 columns; the apply GEMM is built for N = 48, 80, 144.
     pl.NP = (pl.d + 1 <= 48) ? 48 : (pl.d + 1 <= 80) ? 80 : 144;
     pl.KP = (pl.d + 63) / 64 * 64;
@@ -358,10 +360,11 @@ int launch_conv_pair(const TcGemmParams& p, cudaStream_t st) {
 }
 
 int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st) {
+  p.num_n_tiles = 1;
   p.num_tiles = (p.num_m_tiles + 1) / 2;
   switch (cr) {
     case 64: return launch_conv_pair<64, 1, 8>(p, st);
-    case 128: return launch_conv_pair<128, 1, 7>(p, st);
+    case 128: return launch_conv_pair<128, 1, 8>(p, st);
     case 256: return launch_conv_pair<256, 1, 7>(p, st);
     case 288: return launch_conv_pair<288, 2, 7>(p, st);
     case 384: return launch_conv_pair<384, 2, 5>(p, st);
@@ -633,16 +636,26 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.ldo = Cr;
     if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
     p.bias[0] = w->cf3_b;
-    p.gn_partials = gnpart;
-    p.groups = pl.G;
-    p.cpg = Cr / pl.G;
     p.status = status;
     if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
       if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
+
       EDIT_TRY(gemm_conv_reuse(p, Cr, st));
     } else {
       EDIT_TRY(gemm_conv(p, Cr, st));
     }
+    if ((Cr / pl.G) >= 8) {
+      const int nvec = Cr / 8;
+      const int kt = 256 / nvec > 0 ? 256 / nvec : 1;
+      const int threads = kt * nvec;
+      gn_stats_bf16_kernel<<<dim3(pl.gn_P, pl.B), threads, threads * 4 * sizeof(float), st>>>(
+          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_chunk,
+          pl.gn_P, gnpart);
+    } else {
+      gn_partial_kernel<__nv_bfloat16><<<dim3(pl.gn_P, pl.B), 256, 0, st>>>(
+          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
+    }
+    EDIT_TRY(last_launch());
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));

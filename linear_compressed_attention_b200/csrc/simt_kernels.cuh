@@ -145,6 +145,62 @@ __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int g
   }
 }
 
+// bf16 GroupNorm partial sums with 16-byte loads: thread (kt, v) reads the 8
+// channels 8v..8v+7 of tokens t0 + kt, t0 + kt + KT, ... of its chunk; with at
+// least 8 channels per group those 8 channels touch at most two groups, so
+// each thread keeps two (sum, sum of squares) pairs. The block then sums the
+// per-thread pairs of each group in a fixed order (vector, then kt) in fp64.
+// U [B][HW][Cr]; part[b][chunk][g][2]; blockDim = KT * (Cr / 8) threads.
+__global__ void gn_stats_bf16_kernel(const __nv_bfloat16* __restrict__ U, int HW, int Cr, int groups,
+                                     int chunk_tokens, int chunks, float* __restrict__ part) {
+  extern __shared__ float gs_red[];  // [KT * nvec][4]
+  const int b = blockIdx.y, chunk = blockIdx.x;
+  const int nvec = Cr / 8, KT = blockDim.x / nvec;
+  const int cpg = Cr / groups;
+  const int t = threadIdx.x;
+  if (t < KT * nvec) {
+    const int v = t % nvec, kt = t / nvec;
+    const int c0 = v * 8, g0 = c0 / cpg;
+    const int t0 = chunk * chunk_tokens;
+    const int t1 = min(HW, t0 + chunk_tokens);
+    float a0 = 0.f, q0 = 0.f, a1 = 0.f, q1 = 0.f;
+    for (int tok = t0 + kt; tok < t1; tok += KT) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(U + (static_cast<long>(b) * HW + tok) * Cr + c0);
+      const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float x = __bfloat162float(u[j]);
+        if ((c0 + j) / cpg == g0) {
+          a0 += x;
+          q0 = fmaf(x, x, q0);
+        } else {
+          a1 += x;
+          q1 = fmaf(x, x, q1);
+        }
+      }
+    }
+    gs_red[t * 4 + 0] = a0;
+    gs_red[t * 4 + 1] = q0;
+    gs_red[t * 4 + 2] = a1;
+    gs_red[t * 4 + 3] = q1;
+  }
+  __syncthreads();
+  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+    double s1 = 0.0, s2 = 0.0;
+    const int vlo = (g * cpg) / 8, vhi = ((g + 1) * cpg - 1) / 8;
+    for (int v = vlo; v <= vhi; ++v) {
+      const int slot = ((v * 8) / cpg == g) ? 0 : 2;
+      for (int kt = 0; kt < KT; ++kt) {
+        s1 += gs_red[(kt * nvec + v) * 4 + slot];
+        s2 += gs_red[(kt * nvec + v) * 4 + slot + 1];
+      }
+    }
+    float* o = part + ((static_cast<long>(b) * chunks + chunk) * groups + g) * 2;
+    o[0] = static_cast<float>(s1);
+    o[1] = static_cast<float>(s2);
+  }
+}
+
 // Fixed-order (deterministic) combine of the partials in fp64, then the
 // per-channel affine form of GN: scale = gamma * rstd, shift = beta - mean * scale.
 // part: [B][P][groups][2]; stats out: [B][groups][2] (mean, rstd);

@@ -5,10 +5,12 @@
 // same 128 x 64 operand shifted by kh * 130 + kw rows inside the patch (a
 // descriptor start offset; the swizzle follows the absolute address). Only the weights
 // stream per tap. Requires tiles of 128 consecutive pixels of one image row
-// (TW = 128, TH = 1, i.e. W >= 128).
+// (TW = 128, TH = 1, i.e. W >= 128). The epilogue only adds the bias and
+// stores U (GroupNorm statistics are a separate pass over U), so the
+// non-overlapped epilogue of the single TMEM accumulator stays short.
 //
 // Roles as in the pair GEMM: warp 0 producer (both CTAs), warp 1 TMEM owner
-// and (leader) MMA issuer, warps 2..5 epilogue (U store + GroupNorm partials).
+// and (leader) MMA issuer, warps 2..5 epilogue (bias + U store).
 #pragma once
 
 #include "tc_gemm.cuh"
@@ -26,8 +28,9 @@ struct ConvPairCfg {
   static constexpr int B_BYTES = NSPLIT * BROWS * 128;                 // per CTA per tap
   static constexpr int ACC = (2 * BN <= 512) ? 2 : 1;
   static constexpr int TMEM_COLS = (ACC * BN <= 128) ? 128 : (ACC * BN <= 256) ? 256 : 512;
+  static constexpr int STG_BYTES = 0;  // U is small: direct 16-byte stores, no staging
   static constexpr int BAR_BYTES = (2 * 2 + 2 * NB + 2 * ACC) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + 2 * PATCH_BYTES + NB * B_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + 2 * PATCH_BYTES + NB * B_BYTES + STG_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
 };
@@ -40,7 +43,7 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                              // 2 patch buffers
   uint8_t* sB = smem + 2 * Cfg::PATCH_BYTES;       // NB weight stages
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + NB * Cfg::B_BYTES);
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + NB * Cfg::B_BYTES + Cfg::STG_BYTES);
   uint64_t* a_empty = a_full + 2;
   uint64_t* b_full = a_empty + 2;
   uint64_t* b_empty = b_full + NB;
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
 #pragma unroll
             for (int s = 0; s < NSPLIT; ++s)
               tma2_load_2d(&p.b0, bar, sB + bi * Cfg::B_BYTES + s * Cfg::BROWS * 128, tap * C + cb * 64,
-                           s * NCHUNK + rank * Cfg::BROWS);
+                           tc.n_tile * BN + s * NCHUNK + rank * Cfg::BROWS);
             if (++bi == NB) {
               bi = 0;
               bph ^= 1;

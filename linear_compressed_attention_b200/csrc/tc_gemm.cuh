@@ -8,8 +8,7 @@
 //  EPI_CONV    ConvFusion 3x3 conv as an implicit GEMM over the token grid
 //              (K = 9 * C_in, one shifted TMA box per tap; the box's
 //              out-of-grid rows/columns are zero-filled by TMA, which is
-//              exactly the conv's zero padding): + bias, bf16 store of U and
-//              per-tile GroupNorm partial sums.
+//              exactly the conv's zero padding): + bias, bf16 store of U.
 //  EPI_APPLY   Linear attention apply, eq. (y_i): per head h, [num | den] =
 //              Q_h [S_h | z_h] and y = num / (den + eps) fused into the store.
 //  EPI_KVSTATE Linear attention state, eq. (y_i): per (image, head, chunk of
@@ -69,8 +68,6 @@ struct TcGemmParams {
   const void* bias[3];
   int bias_f32;
   int relu;
-  float* gn_partials;  // EPI_CONV: [img][tiles_per_img][4][groups][2]
-  int groups, cpg;
   int* status;
 };
 
@@ -224,58 +221,29 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileC
   } else {
     const int n0 = tc.n_tile * BN;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ldo + n0;
-    float s1 = 0.f, s2 = 0.f;  // GroupNorm running sums of the current group
-    int g_cur = 0;
-    float* gpart = nullptr;
-    const bool gn_on = EPI == EPI_CONV && tc.m_tile < p.num_m_tiles;
-    if (gn_on) {
-      const int per_img = p.tiles_h * p.tiles_w;
-      const int t_in_img = tc.m_tile - tc.img * per_img;
-      gpart = p.gn_partials + ((static_cast<long>(tc.img) * per_img + t_in_img) * 4 + q) * p.groups * 2;
-    }
 #pragma unroll 1
-    for (int c = 0; c < BN / 16; ++c) {
-      const int n = n0 + c * 16;
-      float v[16];
-      tmem_ld16(t_row + c * 16, v);
-      const int src = n / p.n_split;
-      const void* bias = (src < 3 && n < p.N) ? p.bias[src] : nullptr;
-      if (bias) {
-        const int j0 = n - src * p.n_split;
+    for (int c0 = 0; c0 < BN; c0 += 64) {
+      float v[64];
+      tmem_ld64(t_row + c0, v);  // columns past BN belong to nobody here and are not used
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          v[i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j0 + i]
-                             : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
-      }
-      if (p.relu) {
+      for (int g16 = 0; g16 < 4; ++g16) {
+        const int col = c0 + 16 * g16;
+        const int n = n0 + col;
+        if (col >= BN) continue;
+        const int src = n / p.n_split;
+        const void* bias = (src < 3 && n < p.N) ? p.bias[src] : nullptr;
+        if (bias) {
+          const int j0 = n - src * p.n_split;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.f);
-      }
-      if (EPI == EPI_CONV) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int g = (c * 16 + i) / p.cpg;  // warp-uniform
-          if (g != g_cur) {
-            const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-            if (lane == 0 && gn_on) {
-              gpart[g_cur * 2] = t1;
-              gpart[g_cur * 2 + 1] = t2;
-            }
-            s1 = s2 = 0.f;
-            g_cur = g;
-          }
-          const float x = valid ? v[i] : 0.f;
-          s1 += x;
-          s2 += x * x;
+          for (int i = 0; i < 16; ++i)
+            v[16 * g16 + i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j0 + i]
+                                          : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
         }
-      }
-      if (valid && n < p.N) store_bf16x16(orow + c * 16, v, 16);
-    }
-    if (EPI == EPI_CONV) {
-      const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-      if (lane == 0 && gn_on) {
-        gpart[g_cur * 2] = t1;
-        gpart[g_cur * 2 + 1] = t2;
+        if (p.relu) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = fmaxf(v[16 * g16 + i], 0.f);
+        }
+        if (valid && n < p.N) store_bf16x16(orow + col, *reinterpret_cast<const float(*)[16]>(&v[16 * g16]), 16);
       }
     }
   }
@@ -512,31 +480,14 @@ struct TcPairCfg {
 };
 
 // Staged epilogue (EPI_LINEAR / EPI_CONV): per 64-column chunk, one 64-wide
-// TMEM load, bias / ReLU / GroupNorm partials in registers, a 128B-swizzled
+// TMEM load, bias / ReLU in registers, a 128B-swizzled
 // 32 x 128-byte staging block per warp (double-buffered), and one TMA tensor
 // store of the block, so global writes leave the SM as full lines.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, const TileCoord& tc, uint32_t t_row,
                                                      int q, int lane, uint8_t* stg, int& sbuf) {
-  const int r = q * 32 + lane;
   const bool real = tc.m_tile < p.num_m_tiles;
-  bool valid;
-  if (EPI == EPI_CONV) {
-    const int hh = tc.h0 + r / p.TW, ww = tc.w0 + r % p.TW;
-    valid = real && hh < p.H && ww < p.W;
-  } else {
-    valid = real && tc.r0 + r < p.R;
-  }
   const int n0 = tc.n_tile * BN;
-  float s1 = 0.f, s2 = 0.f;  // GroupNorm running sums of the current group
-  int g_cur = 0;
-  float* gpart = nullptr;
-  const bool gn_on = EPI == EPI_CONV && real;
-  if (gn_on) {
-    const int per_img = p.tiles_h * p.tiles_w;
-    const int t_in_img = tc.m_tile - tc.img * per_img;
-    gpart = p.gn_partials + ((static_cast<long>(tc.img) * per_img + t_in_img) * 4 + q) * p.groups * 2;
-  }
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 64) {
     float v[64];
@@ -559,27 +510,6 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
     }
-    if (EPI == EPI_CONV) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int col = c0 + i;
-        if (col < BN) {                      // warp-uniform
-          const int g = col / p.cpg;
-          if (g != g_cur) {
-            const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-            if (lane == 0 && gn_on) {
-              gpart[g_cur * 2] = t1;
-              gpart[g_cur * 2 + 1] = t2;
-            }
-            s1 = s2 = 0.f;
-            g_cur = g;
-          }
-          const float x = valid ? v[i] : 0.f;
-          s1 += x;
-          s2 += x * x;
-        }
-      }
-    }
     // stage this warp's 32 rows x 64 columns (bf16) in 128B-swizzled order
     if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
     __syncwarp();
@@ -600,20 +530,13 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
       if (EPI == EPI_CONV) {
         const int r0w = q * 32;
         const int ws = tc.w0 + r0w % p.TW, hs = tc.h0 + r0w / p.TW;
-        if (ws < p.W && hs < p.H) tma_store_4d(&p.out_map, buf, c0, ws, hs, tc.img);
+        if (ws < p.W && hs < p.H) tma_store_4d(&p.out_map, buf, n0 + c0, ws, hs, tc.img);
       } else {
         if (tc.r0 + q * 32 < p.R) tma_store_2d(&p.out_map, buf, n0 + c0, tc.img * p.R + tc.r0 + q * 32);
       }
       bulk_commit();
     }
     sbuf ^= 1;
-  }
-  if (EPI == EPI_CONV) {
-    const float t1 = warp_sum(s1), t2 = warp_sum(s2);
-    if (lane == 0 && gn_on) {
-      gpart[g_cur * 2] = t1;
-      gpart[g_cur * 2 + 1] = t2;
-    }
   }
 }
 
