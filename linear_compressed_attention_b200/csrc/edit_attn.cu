@@ -49,14 +49,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+enum Swz { SWZ_NONE = 0, SWZ_64 = 64, SWZ_128 = 128 };
+
 bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-            const cuuint32_t* box) {
+            const cuuint32_t* box, int swz = SWZ_128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = swz == SWZ_128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swz == SWZ_64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Apply output: out [img][R][C] bf16, unswizzled box d x 32 x 1 (one head of
+// 32 rows per store).
+bool map_out_heads(CUtensorMap* m, const void* base, long C, long R, long imgs, int d) {
+  cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)R, (cuuint64_t)imgs};
+  cuuint64_t st[2] = {(cuuint64_t)C * 2, (cuuint64_t)R * C * 2};
+  cuuint32_t box[3] = {(cuuint32_t)d, 32, 1};
+  return encode(m, 3, base, dims, st, box, SWZ_NONE);
 }
 
 // A operand: [imgs][rows][K] bf16, row stride ld elements, box 64 x 128 x 1.
@@ -280,10 +294,10 @@ int grid_for(long total, int threads) {
   return static_cast<int>(g < 1 ? 1 : g);
 }
 
-template <int BN, int NSPLIT, int STAGES, int EPI>
+template <int BN, int NSPLIT, int STAGES, int EPI, int STG = 0>
 int launch_tc(const TcGemmParams& p, cudaStream_t st) {
-  using Cfg = TcGemmCfg<BN, NSPLIT, STAGES>;
-  auto kern = tc_gemm_kernel<BN, NSPLIT, STAGES, EPI>;
+  using Cfg = TcGemmCfg<BN, NSPLIT, STAGES, STG>;
+  auto kern = tc_gemm_kernel<BN, NSPLIT, STAGES, EPI, STG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
     return EDIT_ERR_CUDA;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
@@ -404,11 +418,12 @@ int gemm_conv(TcGemmParams& p, int cr, cudaStream_t st) {
   return EDIT_ERR_UNSUPPORTED;
 }
 
+// Apply: staging of 4 warps x 2 buffers x (32 rows x d bf16); d <= 40 / 72 / 136 for NP 48 / 80 / 144.
 int gemm_apply(const TcGemmParams& p, int np, cudaStream_t st) {
   switch (np) {
-    case 48: return launch_tc<48, 1, 8, EPI_APPLY>(p, st);
-    case 80: return launch_tc<80, 1, 8, EPI_APPLY>(p, st);
-    case 144: return launch_tc<144, 1, 6, EPI_APPLY>(p, st);
+    case 48: return launch_tc<48, 1, 8, EPI_APPLY, 8 * 32 * 40 * 2>(p, st);
+    case 80: return launch_tc<80, 1, 6, EPI_APPLY, 8 * 32 * 72 * 2>(p, st);
+    case 144: return launch_tc<144, 1, 4, EPI_APPLY, 8 * 32 * 136 * 2>(p, st);
   }
   return EDIT_ERR_UNSUPPORTED;
 }
@@ -491,13 +506,38 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   if (pl.bf16) {
     __nv_bfloat16* KT = reinterpret_cast<__nv_bfloat16*>(ws + pl.KT);
     __nv_bfloat16* VTx = reinterpret_cast<__nv_bfloat16*>(ws + pl.VTx);
-    dwconv_s2_t_kernel<<<dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64)), 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(ws + pl.KVp), pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, pl.Mp, pl.NP,
-        static_cast<const __nv_bfloat16*>(w->kdw_w), static_cast<const __nv_bfloat16*>(w->kdw_b),
-        static_cast<const __nv_bfloat16*>(w->vdw_w), static_cast<const __nv_bfloat16*>(w->vdw_b), KT, VTx,
-        pl.K ? reinterpret_cast<__nv_bfloat16*>(ws + pl.K) : nullptr,
-        pl.V ? reinterpret_cast<__nv_bfloat16*>(ws + pl.V) : nullptr);
-    EDIT_TRY(last_launch());
+    {
+      DwTmaMaps mp;
+      std::memset(&mp, 0, sizeof(mp));
+      const long C2 = 2L * pl.C;
+      cuuint64_t d_in[4] = {(cuuint64_t)C2, (cuuint64_t)pl.W, (cuuint64_t)pl.H, (cuuint64_t)pl.B};
+      cuuint64_t s_in[3] = {(cuuint64_t)C2 * 2, (cuuint64_t)pl.W * C2 * 2, (cuuint64_t)pl.H * pl.W * C2 * 2};
+      cuuint32_t b_in[4] = {64, 65, 3, 1};
+      cuuint64_t d_kt[2] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.B * pl.C};
+      cuuint64_t s_kt[1] = {(cuuint64_t)pl.Mp * 2};
+      cuuint32_t b_kt[2] = {32, 64};
+      cuuint64_t d_vt[3] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.NP, (cuuint64_t)pl.B * pl.heads};
+      cuuint64_t s_vt[2] = {(cuuint64_t)pl.Mp * 2, (cuuint64_t)pl.NP * pl.Mp * 2};
+      cuuint32_t b_vt[3] = {32, 8, 1};
+      if (!encode(&mp.in, 4, ws + pl.KVp, d_in, s_in, b_in, SWZ_NONE) ||
+          !encode(&mp.kt, 2, KT, d_kt, s_kt, b_kt, SWZ_64) || !encode(&mp.vtx, 3, VTx, d_vt, s_vt, b_vt, SWZ_64))
+        return EDIT_ERR_CUDA;
+      const int tokmajor = pl.K ? 1 : 0;
+      if (tokmajor) {
+        cuuint64_t d_t[4] = {(cuuint64_t)pl.C, (cuuint64_t)pl.Wo, (cuuint64_t)pl.Ho, (cuuint64_t)pl.B};
+        cuuint64_t s_t[3] = {(cuuint64_t)pl.C * 2, (cuuint64_t)pl.Wo * pl.C * 2,
+                             (cuuint64_t)pl.Ho * pl.Wo * pl.C * 2};
+        cuuint32_t b_t[4] = {64, 32, 1, 1};
+        if (!encode(&mp.ktok, 4, ws + pl.K, d_t, s_t, b_t, SWZ_NONE) ||
+            !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
+          return EDIT_ERR_CUDA;
+      }
+      dwconv_s2_tma_kernel<<<dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64)), 256, 0, st>>>(
+          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
+          static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
+          static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
+      EDIT_TRY(last_launch());
+    }
     const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * pl.Mp;
     vtx_pad_rows_kernel<<<grid_for(padn, 256), 256, 0, st>>>(VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
     EDIT_TRY(last_launch());
@@ -687,10 +727,12 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
                                               reinterpret_cast<float*>(ws + pl.gnss));
   EDIT_TRY(last_launch());
   if (pl.bf16) {
-    const long total8 = tok * Cr / 8;
-    gn_apply_leaky_bf16x8<<<grid_for(total8, 256), 256, 0, st>>>(
+    const int nvec = Cr / 8;
+    const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
+    const int threads = per_block * nvec;
+    gn_apply_leaky_bf16x8<<<grid_for(tok, per_block), threads, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-        w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), total8);
+        w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
   } else {
     const long total = tok * Cr;
     gn_apply_leaky_kernel<float><<<grid_for(total, 256), 256, 0, st>>>(
@@ -772,6 +814,7 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
     p.eps = w->attn_eps;
     p.out = out;
     p.ldo = pl.C;
+    if (!map_out_heads(&p.out_map, out, pl.C, pl.HW, pl.B, pl.d)) return EDIT_ERR_CUDA;
     p.status = status;
     return gemm_apply(p, pl.NP, st);
   }

@@ -262,24 +262,40 @@ __global__ void gn_apply_leaky_kernel(const T* __restrict__ U, const float* __re
 }
 
 // bf16 variant, 8 channels per thread with 16-byte loads/stores (Cr % 8 == 0).
+// Thread t always handles channel vector t % (Cr/8) (blockDim a multiple of
+// Cr/8), so its scale/shift stay in registers across the tokens it visits.
 __global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const float* __restrict__ ss, long HW,
-                                      int Cr, float slope, __nv_bfloat16* __restrict__ G, long total8) {
-  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total8;
-       i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long e = i * 8;
-    const int c = static_cast<int>(e % Cr);
-    const long b = e / (HW * Cr);
+                                      int Cr, float slope, __nv_bfloat16* __restrict__ G, long tokens) {
+  const int nvec = Cr / 8;
+  const int per_block = blockDim.x / nvec;
+  const int v = threadIdx.x % nvec, kt = threadIdx.x / nvec;
+  if (kt >= per_block) return;
+  const int c = v * 8;
+  long b_cur = -1;
+  float sc[8], sh[8];
+  for (long tok = static_cast<long>(blockIdx.x) * per_block + kt; tok < tokens;
+       tok += static_cast<long>(gridDim.x) * per_block) {
+    const long b = tok / HW;
+    if (b != b_cur) {
+      const float4* s4 = reinterpret_cast<const float4*>(ss + (b * Cr + c) * 2);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 q = s4[j];
+        sc[2 * j] = q.x;
+        sh[2 * j] = q.y;
+        sc[2 * j + 1] = q.z;
+        sh[2 * j + 1] = q.w;
+      }
+      b_cur = b;
+    }
+    const long e = tok * Cr + c;
     const uint4 raw = *reinterpret_cast<const uint4*>(U + e);
     const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
-    const float4* s4 = reinterpret_cast<const float4*>(ss + (b * Cr + c) * 2);
     float o[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 s = s4[j];
-      float v0 = fmaf(__bfloat162float(u[2 * j]), s.x, s.y);
-      float v1 = fmaf(__bfloat162float(u[2 * j + 1]), s.z, s.w);
-      o[2 * j] = v0 >= 0.f ? v0 : v0 * slope;
-      o[2 * j + 1] = v1 >= 0.f ? v1 : v1 * slope;
+    for (int j = 0; j < 8; ++j) {
+      const float y = fmaf(__bfloat162float(u[j]), sc[j], sh[j]);
+      o[j] = y >= 0.f ? y : y * slope;
     }
     uint4 out;
     out.x = pack_bf16x2(o[0], o[1]);
@@ -468,6 +484,119 @@ __global__ void __launch_bounds__(256) dwconv_s2_t_kernel(
       *reinterpret_cast<uint4*>(tok + ((static_cast<long>(b) * Ho + i) * Wo + j) * C + ch0 + v * 8) =
           *reinterpret_cast<const uint4*>(tmp);
     }
+  }
+}
+
+// TMA version of the channel-major depthwise conv (same outputs as
+// dwconv_s2_t_kernel): the 3 x 65-pixel, 64-channel input patch arrives in one
+// tensor load (zero-filled outside the grid). Thread (tg, c) computes the 8
+// consecutive output tokens 8*tg .. 8*tg+7 of channel c (51 patch reads for
+// 72 taps) and writes them as one 16-byte chunk of the channel-major block,
+// placed with the 64-byte swizzle (chunk j of row r at j ^ ((r >> 1) & 3)) so
+// the 16-byte writes of a warp hit distinct banks; the tensor stores undo the
+// swizzle. KT leaves as one 64-row x 32-token block, VTx as eight 8-row
+// blocks (a head boundary never splits one since d % 8 == 0), and the
+// token-major copies (MM-EDiT) as one 32-token x 64-channel block clipped at
+// the end of the output row. The load wait is bounded (status on timeout).
+struct DwTmaMaps {
+  CUtensorMap in;    // KVp as [B][H][W][2C], box 64 x 65 x 3 x 1, no swizzle
+  CUtensorMap kt;    // KT as [B*C][Mp], box 32 x 64, 64-byte swizzle
+  CUtensorMap vtx;   // VTx as [B*heads][NP][Mp], box 32 x 8 x 1, 64-byte swizzle
+  CUtensorMap ktok;  // K as [B][Ho][Wo][C], box 64 x 32 x 1 x 1, no swizzle (MM only)
+  CUtensorMap vtok;  // V likewise
+};
+
+__global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constant__ DwTmaMaps m, int H, int W, int C,
+                                                            int d, int heads, int Wop,
+                                                            const __nv_bfloat16* __restrict__ kw,
+                                                            const __nv_bfloat16* __restrict__ kb,
+                                                            const __nv_bfloat16* __restrict__ vw,
+                                                            const __nv_bfloat16* __restrict__ vb, int tokmajor,
+                                                            int* status) {
+  constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
+  __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
+  __shared__ __align__(128) __nv_bfloat16 in_s[3][PW][CB];
+  __shared__ __align__(128) __nv_bfloat16 tok_s[JT][CB];    // [token][channel]
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const int Wo = (W + 1) / 2;
+  const int j0 = blockIdx.x * JT, i = blockIdx.y;
+  const int nblk = 2 * C / CB;
+  const int b = blockIdx.z / nblk, cb = blockIdx.z - b * nblk;
+  const int gc0 = cb * CB;
+  const bool isk = gc0 < C;
+  const int ch0 = isk ? gc0 : gc0 - C;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&m.in);
+    mbar_arrive_expect_tx(&bar, 3 * PW * CB * 2);
+    tma_load_4d(&m.in, &bar, &in_s[0][0][0], gc0, 2 * j0 - 1, 2 * i - 1, b);
+  }
+  const int c = threadIdx.x & (CB - 1);
+  const int tg = threadIdx.x >> 6;  // tokens 8*tg .. 8*tg + 7
+  const __nv_bfloat16* wt = isk ? kw : vw;
+  float wr[9];
+#pragma unroll
+  for (int q = 0; q < 9; ++q) wr[q] = __bfloat162float(wt[(ch0 + c) * 9 + q]);
+  const float bias = __bfloat162float((isk ? kb : vb)[ch0 + c]);
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, status);
+  if (ok) {
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = bias;
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+#pragma unroll
+      for (int col = 0; col < 17; ++col) {  // patch columns 16*tg + col
+        const float x = __bfloat162float(in_s[a][16 * tg + col][c]);
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+          const int t2 = col - e;  // output 2t + e == col
+          if (t2 >= 0 && (t2 & 1) == 0 && t2 / 2 < 8) acc[t2 / 2] = fmaf(wr[a * 3 + e], x, acc[t2 / 2]);
+        }
+      }
+    }
+    float o[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      float v = isk ? fmaxf(acc[t], 0.f) : acc[t];
+      o[t] = (j0 + 8 * tg + t >= Wo) ? 0.f : v;
+    }
+    uint4 pk;
+    pk.x = pack_bf16x2(o[0], o[1]);
+    pk.y = pack_bf16x2(o[2], o[3]);
+    pk.z = pack_bf16x2(o[4], o[5]);
+    pk.w = pack_bf16x2(o[6], o[7]);
+    // row c (64 bytes = 4 chunks), chunk tg, 64-byte swizzle
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out_s) + c * 64 + 16 * (tg ^ ((c >> 1) & 3))) = pk;
+    if (tokmajor) {
+      const __nv_bfloat16* ob = reinterpret_cast<const __nv_bfloat16*>(&pk);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) tok_s[8 * tg + t][c] = ob[t];
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0 && ok) {
+    const int t0 = i * Wop + j0;
+    if (isk) {
+      tma_store_2d(&m.kt, out_s, t0, b * C + ch0);
+    } else {
+#pragma unroll 1
+      for (int g = 0; g < CB / 8; ++g) {
+        const int ch = ch0 + 8 * g;
+        const int h = ch / d, rr = ch - h * d;
+        tma_store_3d(&m.vtx, out_s + 8 * g * JT, t0, rr, b * heads + h);
+      }
+    }
+    if (tokmajor && j0 < Wo) tma_store_4d(isk ? &m.ktok : &m.vtok, &tok_s[0][0], ch0, j0, i, b);
+    bulk_commit();
+    bulk_wait_all();
   }
 }
 

@@ -71,7 +71,7 @@ struct TcGemmParams {
   int* status;
 };
 
-template <int BN, int NSPLIT, int STAGES>
+template <int BN, int NSPLIT, int STAGES, int STG = 0>
 struct TcGemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int NCHUNK = BN / NSPLIT;
@@ -84,11 +84,14 @@ struct TcGemmCfg {
   static constexpr int TMEM_COLS = (ACC * BN <= 32) ? 32 : (ACC * BN <= 64) ? 64 : (ACC * BN <= 128) ? 128
                                    : (ACC * BN <= 256) ? 256 : 512;
   static_assert(ACC * BN <= 512, "TMEM");
+  static constexpr int STG_BYTES = STG;  // epilogue staging (EPI_APPLY)
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * ACC) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NCHUNK);
 };
+
+
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
@@ -249,6 +252,49 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileC
   }
 }
 
+// Apply epilogue with staged TMA stores: per warp, 32 rows x d outputs of one
+// head in a dense [32][d] bf16 block (2 buffers, 32*d*2 bytes each), written
+// by one 3D tensor store into out [img][R][C] at column head * d.
+template <int BN>
+__device__ __forceinline__ void epilogue_apply_staged(const TcGemmParams& p, const TileCoord& tc, uint32_t t_row,
+                                                      int q, int lane, uint8_t* stg, int& sbuf) {
+  const int d = p.d;
+  float v[64];
+  float dv[16];
+  tmem_ld16(t_row + (d / 16) * 16, dv);  // the denominator column d
+  float den = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (i == d % 16) den = dv[i];
+  const float inv = 1.f / (den + p.eps);
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  uint8_t* buf = stg + sbuf * (32 * d * 2);
+  uint4* rowp = reinterpret_cast<uint4*>(buf + lane * d * 2);
+#pragma unroll 1
+  for (int c0 = 0; c0 < d; c0 += 64) {
+    tmem_ld64(t_row + c0, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (c0 + 8 * j < d) {
+        uint4 o;
+        o.x = pack_bf16x2(v[8 * j + 0] * inv, v[8 * j + 1] * inv);
+        o.y = pack_bf16x2(v[8 * j + 2] * inv, v[8 * j + 3] * inv);
+        o.z = pack_bf16x2(v[8 * j + 4] * inv, v[8 * j + 5] * inv);
+        o.w = pack_bf16x2(v[8 * j + 6] * inv, v[8 * j + 7] * inv);
+        rowp[c0 / 8 + j] = o;
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && tc.m_tile < p.num_m_tiles && tc.r0 + q * 32 < p.R) {
+    tma_store_3d(&p.out_map, buf, tc.n_tile * d, tc.r0 + q * 32, tc.img);
+    bulk_commit();
+  }
+  sbuf ^= 1;
+}
+
 // A and B loads of k-block kb of a (1-CTA) tile into one pipeline stage.
 template <int BN, int NSPLIT, int EPI, bool PAIR>
 __device__ __forceinline__ void load_stage(const TcGemmParams& p, const TileCoord& tc, int kb, uint8_t* dA,
@@ -313,15 +359,16 @@ __device__ __forceinline__ void load_stage(const TcGemmParams& p, const TileCoor
   }
 }
 
-template <int BN, int NSPLIT, int STAGES, int EPI>
+template <int BN, int NSPLIT, int STAGES, int EPI, int STG = 0>
 __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
-  using Cfg = TcGemmCfg<BN, NSPLIT, STAGES>;
+  using Cfg = TcGemmCfg<BN, NSPLIT, STAGES, STG>;
   constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_BYTES);
+  uint8_t* stg_base = sB + STAGES * Cfg::B_BYTES;  // 1024-byte aligned
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;
   uint64_t* tempty_bar = tfull_bar + ACC;
@@ -426,6 +473,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* stg = stg_base + q * (STG / 4);
+    int sbuf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -433,13 +482,20 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       tc_fence_after();
       const TileCoord tc = decode_tile<EPI>(p, tile);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_tile<BN, EPI>(p, tc, t_row, q, lane);
+      if (EPI == EPI_APPLY && STG > 0)
+        epilogue_apply_staged<BN>(p, tc, t_row, q, lane, stg, sbuf);
+      else
+        epilogue_tile<BN, EPI>(p, tc, t_row, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == ACC) {
         acc = 0;
         acc_phase ^= 1;
       }
+    }
+    if (STG > 0) {
+      if (lane == 0) bulk_wait_all();  // staged stores finished before shared memory is released
+      __syncwarp();
     }
   }
 
