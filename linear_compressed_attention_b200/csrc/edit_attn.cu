@@ -136,6 +136,10 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Planning is host-only (no CUDA call), so chunking uses the B200 SM count.
 int num_sms_hint() { return 148; }
 
+// Most conv pair tiles ever split in the last wave (at most half of the
+// co-resident pairs).
+constexpr int kConvMaxSplit = 40;
+
 struct Plan {
   // geometry
   int B, H, W, C, heads, Cr, G, d, Ho, Wo, M, NT;
@@ -152,7 +156,7 @@ struct Plan {
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      total;
+      fixpart, total;
 };
 
 int next_pow2(int v) {
@@ -253,6 +257,8 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
   pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
   pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
+  // fp32 halves of the conv tiles split in the last wave (tap-reuse conv only)
+  pl.fixpart = (pl.bf16 && pl.TW == 128) ? take(static_cast<size_t>(kConvMaxSplit) * 4 * 128 * pl.Cr * 4) : 0;
   pl.total = off;
   return EDIT_OK;
 }
@@ -342,7 +348,7 @@ int launch_pair(const TcGemmParams& p, cudaStream_t st) {
 
 // Conv with tap reuse on CTA pairs (tiles of 128 pixels of one image row).
 template <int BN, int NSPLIT, int NB>
-int launch_conv_pair(const TcGemmParams& p, cudaStream_t st) {
+int launch_conv_pair(TcGemmParams& p, cudaStream_t st, bool* split_out) {
   using Cfg = ConvPairCfg<BN, NSPLIT, NB>;
   auto kern = tc_conv_pair_kernel<BN, NSPLIT, NB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
@@ -367,21 +373,33 @@ int launch_conv_pair(const TcGemmParams& p, cudaStream_t st) {
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
     max_clusters = n;
   }
+  // Last partial wave at most half full: split its tiles over the input-channel
+  // blocks into two half items each, so every pair has work in that wave.
+  const int T = p.num_tiles;
+  const int R = T % max_clusters;
+  p.split_first = T;
+  p.split_count = 0;
+  if (T > max_clusters && R > 0 && 2 * R <= max_clusters && R <= kConvMaxSplit && p.fix_part && p.kb_per_tap >= 2) {
+    p.split_first = T - R;
+    p.split_count = R;
+    p.num_tiles = T + R;  // items
+  }
+  *split_out = p.split_count > 0;
   const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return EDIT_ERR_CUDA;
   return last_launch();
 }
 
-int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st) {
+int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st, bool* split) {
   p.num_n_tiles = 1;
   p.num_tiles = (p.num_m_tiles + 1) / 2;
   switch (cr) {
-    case 64: return launch_conv_pair<64, 1, 8>(p, st);
-    case 128: return launch_conv_pair<128, 1, 8>(p, st);
-    case 256: return launch_conv_pair<256, 1, 7>(p, st);
-    case 288: return launch_conv_pair<288, 2, 7>(p, st);
-    case 384: return launch_conv_pair<384, 2, 5>(p, st);
+    case 64: return launch_conv_pair<64, 1, 8>(p, st, split);
+    case 128: return launch_conv_pair<128, 1, 8>(p, st, split);
+    case 256: return launch_conv_pair<256, 1, 7>(p, st, split);
+    case 288: return launch_conv_pair<288, 2, 7>(p, st, split);
+    case 384: return launch_conv_pair<384, 2, 5>(p, st, split);
   }
   return EDIT_ERR_UNSUPPORTED;
 }
@@ -538,7 +556,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
           static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
       EDIT_TRY(last_launch());
     }
-    const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * pl.Mp;
+    const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
     vtx_pad_rows_kernel<<<grid_for(padn, 256), 256, 0, st>>>(VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
     EDIT_TRY(last_launch());
     stage_mark(2, st);
@@ -679,8 +697,16 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.status = status;
     if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
       if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
-
-      EDIT_TRY(gemm_conv_reuse(p, Cr, st));
+      p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
+      bool split = false;
+      EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
+      if (split) {
+        const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
+        conv_fixup_kernel<<<grid_for(total, 256), 256, 0, st>>>(
+            p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
+            static_cast<const __nv_bfloat16*>(w->cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+        EDIT_TRY(last_launch());
+      }
     } else {
       EDIT_TRY(gemm_conv(p, Cr, st));
     }

@@ -601,17 +601,54 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
 }
 
 // Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
-// KV state also yields z = sum_j K_j) followed by zero rows.
+// KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
+// (Mp % 8 == 0).
 __global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
-  const long per = static_cast<long>(NP - d) * Mp;
-  const long total = BH * per;
+  const int vpr = Mp / 8;                   // vectors per row
+  const int rows = NP - d;
+  const long total = static_cast<long>(BH) * rows * vpr;
+  const __nv_bfloat162 one2 = __floats2bfloat162_rn(1.f, 1.f);
+  const uint32_t onew = *reinterpret_cast<const uint32_t*>(&one2);
   for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long bh = e / per;
-    const long rem = e - bh * per;
-    const int r = d + static_cast<int>(rem / Mp);
-    const long t = rem % Mp;
-    VTx[(bh * NP + r) * Mp + t] = __float2bfloat16_rn(r == d ? 1.f : 0.f);
+    const long ri = e / vpr;
+    const int v = static_cast<int>(e - ri * vpr);
+    const long bh = ri / rows;
+    const int r = d + static_cast<int>(ri - bh * rows);
+    const uint32_t w = r == d ? onew : 0u;
+    *reinterpret_cast<uint4*>(VTx + (bh * NP + r) * Mp + 8L * v) = make_uint4(w, w, w, w);
+  }
+}
+
+// Sum of the two fp32 halves of each split conv tile plus the bias -> U (bf16),
+// 4 channels per thread (Cr % 4 == 0). Tile t of the pair grid: CTA `rank`
+// holds 128-pixel tile 2t + rank (one image-row segment of 128 pixels).
+// part [split][half][rank][128][Cr].
+__global__ void conv_fixup_kernel(const float* __restrict__ part, int split_first, int split_count, int tiles_w,
+                                  int tiles_h, int H, int W, int Cr, const __nv_bfloat16* __restrict__ bias,
+                                  int num_m_tiles, __nv_bfloat16* __restrict__ U) {
+  const int cv = Cr / 4;
+  const int total = split_count * 2 * 128 * cv;
+  const int per = 2 * 128 * Cr;  // one split tile, one half
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int c = (e % cv) * 4;
+    const int rr = e / cv;  // (split, rank, row)
+    const int row = rr & 127;
+    const int rank = (rr >> 7) & 1;
+    const int sp = rr >> 8;
+    const int m_tile = 2 * (split_first + sp) + rank;
+    if (m_tile >= num_m_tiles) continue;
+    const int per_img = tiles_h * tiles_w;
+    const int img = m_tile / per_img, u = m_tile - img * per_img;
+    const int hh = u / tiles_w, ww = (u % tiles_w) * 128 + row;
+    if (hh >= H || ww >= W) continue;
+    const int off = (rank * 128 + row) * Cr + c;
+    const float4 a = *reinterpret_cast<const float4*>(part + (2 * sp) * per + off);
+    const float4 b = *reinterpret_cast<const float4*>(part + (2 * sp + 1) * per + off);
+    __nv_bfloat16* dst = U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c;
+    const uint2 o = make_uint2(pack_bf16x2(a.x + b.x + __bfloat162float(bias[c]), a.y + b.y + __bfloat162float(bias[c + 1])),
+                               pack_bf16x2(a.z + b.z + __bfloat162float(bias[c + 2]), a.w + b.w + __bfloat162float(bias[c + 3])));
+    *reinterpret_cast<uint2*>(dst) = o;
   }
 }
 

@@ -35,6 +35,28 @@ struct ConvPairCfg {
   static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
 };
 
+// Work item `it`: a whole pair tile, or (for the last partial wave) one half of
+// a pair tile's input-channel blocks.
+struct ConvItem {
+  int pt, cb0, cb1, half;  // half = -1: whole tile
+};
+__device__ __forceinline__ ConvItem conv_item(const TcGemmParams& p, int it, int ncb) {
+  ConvItem c;
+  if (it < p.split_first) {
+    c.pt = it;
+    c.cb0 = 0;
+    c.cb1 = ncb;
+    c.half = -1;
+  } else {
+    const int k = it - p.split_first;
+    c.pt = p.split_first + k / 2;
+    c.half = k & 1;
+    c.cb0 = c.half ? ncb / 2 : 0;
+    c.cb1 = c.half ? ncb : ncb / 2;
+  }
+  return c;
+}
+
 template <int BN, int NSPLIT, int NB>
 __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_constant__ TcGemmParams p) {
   using Cfg = ConvPairCfg<BN, NSPLIT, NB>;
@@ -90,9 +112,10 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
       int ai = 0, bi = 0;
       uint32_t aph = 0, bph = 0;
       bool ok = true;
-      for (int pt = pair; pt < p.num_tiles && ok && !*abort_flag; pt += npairs) {
-        const TileCoord tc = decode_pair_tile<EPI_CONV>(p, pt, rank);
-        for (int cb = 0; cb < ncb && ok; ++cb) {
+      for (int it = pair; it < p.num_tiles && ok && !*abort_flag; it += npairs) {
+        const ConvItem ci = conv_item(p, it, ncb);
+        const TileCoord tc = decode_pair_tile<EPI_CONV>(p, ci.pt, rank);
+        for (int cb = ci.cb0; cb < ci.cb1 && ok; ++cb) {
           if (!mbar_wait(&a_empty[ai], aph ^ 1, abort_flag, p.status)) {
             ok = false;
             break;
@@ -135,11 +158,12 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
       int ai = 0, bi = 0, acc = 0;
       uint32_t aph = 0, bph = 0, acc_phase = 0;
       bool ok = true;
-      for (int pt = pair; pt < p.num_tiles && ok && !*abort_flag; pt += npairs) {
+      for (int it = pair; it < p.num_tiles && ok && !*abort_flag; it += npairs) {
+        const ConvItem ci = conv_item(p, it, ncb);
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int cb = 0; cb < ncb && ok; ++cb) {
+        for (int cb = ci.cb0; cb < ci.cb1 && ok; ++cb) {
           if (!mbar_wait(&a_full[ai], aph, abort_flag, p.status)) {
             ok = false;
             break;
@@ -160,7 +184,7 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
 #pragma unroll
               for (int s = 0; s < NSPLIT; ++s) {
                 const uint64_t bdesc = sdesc_kmajor_sw128(b_addr + s * Cfg::BROWS * 128 + k * 32);
-                umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (cb | tap | k) != 0 ? 1u : 0u);
+                umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (cb != ci.cb0 || tap | k) ? 1u : 0u);
               }
             }
             umma2_commit_mc(&b_empty[bi], 0x3);
@@ -191,12 +215,27 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int pt = pair; pt < p.num_tiles; pt += npairs) {
+    for (int it = pair; it < p.num_tiles; it += npairs) {
       if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const TileCoord tc = decode_pair_tile<EPI_CONV>(p, pt, rank);
+      const ConvItem ci = conv_item(p, it, ncb);
+      const TileCoord tc = decode_pair_tile<EPI_CONV>(p, ci.pt, rank);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_tile<BN, EPI_CONV>(p, tc, t_row, q, lane);
+      if (ci.half < 0) {
+        epilogue_tile<BN, EPI_CONV>(p, tc, t_row, q, lane);
+      } else {  // fp32 partial of this half, row q*32 + lane
+        float* prow = p.fix_part + ((((static_cast<long>(ci.pt - p.split_first) * 2 + ci.half) * 2 + rank) * 128) +
+                                    q * 32 + lane) * p.N;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          float v[64];
+          tmem_ld64(t_row + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + 4 * j < BN)
+              *reinterpret_cast<float4*>(prow + c0 + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader0 + acc * 8);
       if (++acc == ACC) {

@@ -61,6 +61,11 @@ struct TcGemmParams {
   float eps;
   int kv_rows_per_img;  // EPI_KVSTATE: A rows per image (= C)
   int kb_per_chunk, num_chunks;
+  // tap-reuse conv: pair tiles [split_first, split_first + split_count) run as
+  // two half items over the input-channel blocks, writing fp32 partials to
+  // fix_part [split tile][half][rank][128][N] (summed with the bias afterwards)
+  int split_first, split_count;
+  float* fix_part;
   float* kv_part;       // EPI_KVSTATE: [img][heads][num_chunks][d][d+1]
   // epilogue
   void* out;        // bf16, row (img*R + r) at out + row*ldo (+ column offset)
