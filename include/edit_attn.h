@@ -167,9 +167,13 @@ EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, c
  * calls made by this host thread record events[i] (cudaEvent_t handles
  * created by the caller) on the call's stream at stage boundary i:
  *   0 start, 1 K|V Linear GEMM, 2 depthwise conv, 3 KV state,
- *   4 weight folding, 5 3x3 conv GEMM, 6 GroupNorm, 7 query GEMM,
- *   8 apply GEMM; MM-EDiT adds 9 prompt projections, 10 image-row softmax
- *   attention, 11 prompt-row softmax attention.
+ *   4 weight folding, 5 3x3 conv GEMM (the conv kernel alone), 6 GroupNorm
+ *   (statistics, finalize, apply; plus the conv's last-wave fixup when
+ *   used), 7 query GEMM, 8 apply GEMM; MM-EDiT adds 9 prompt projections,
+ *   10 image-row softmax attention, 11 prompt-row softmax attention.
+ * Recording events between kernels serialises the programmatic overlap of
+ * consecutive kernels at those points, so timed steps are fastest without
+ * the hook.
  * `n` is the number of handles (events beyond n are not recorded). NULL
  * clears the hook. Returns EDIT_OK or EDIT_ERR_SHAPE for n < 0.
  *

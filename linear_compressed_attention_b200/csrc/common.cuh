@@ -43,6 +43,14 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ----------------------------------------------------------------- PDL
+// Programmatic dependent launch: every kernel of the library calls this before
+// touching memory written by the kernel before it in the stream (a no-op when
+// launched without the programmatic-serialization attribute). No kernel
+// signals its dependents early, so a dependent grid launches only as the
+// previous grid's blocks exit.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----------------------------------------------------------------- mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -92,17 +100,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
-}
-
-// ----------------------------------------------------------------- cp.async
-// 16-byte global -> shared copy; src_bytes = 0 writes zeros (no global read).
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- TMA

@@ -21,6 +21,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "simt_kernels.cuh"
@@ -288,6 +289,25 @@ void stage_mark(int i, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------ launchers
+// Every library kernel launches with programmatic stream serialization: it may
+// start while the previous kernel drains and waits in pdl_wait() for that
+// kernel's memory. Errors surface through cudaGetLastError in last_launch().
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 int last_launch() {
   ++g_launches;
   return cudaGetLastError() == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
@@ -308,7 +328,7 @@ int launch_tc(const TcGemmParams& p, cudaStream_t st) {
     return EDIT_ERR_CUDA;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
   if (grid < 1) return EDIT_OK;
-  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(p);
+  launch_pdl(kern, dim3(grid), dim3(192), Cfg::SMEM_BYTES, st, p);
   return last_launch();
 }
 
@@ -323,16 +343,18 @@ int launch_pair(const TcGemmParams& p, cudaStream_t st) {
   if (p.num_tiles < 1) return EDIT_OK;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   static int max_clusters = 0;  // per instantiation; same device model throughout a process
   if (max_clusters == 0) {
     cfg.gridDim = dim3(2 * 74, 1, 1);
@@ -356,16 +378,18 @@ int launch_conv_pair(TcGemmParams& p, cudaStream_t st, bool* split_out) {
   if (p.num_tiles < 1) return EDIT_OK;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   static int max_clusters = 0;
   if (max_clusters == 0) {
     cfg.gridDim = dim3(2 * 74, 1, 1);
@@ -499,7 +523,7 @@ int simt_linear(const void* a, long rows, int K, const void* const* wts, const v
   p.N = nsrc * C;
   p.out = static_cast<float*>(out);
   p.ldo = nsrc * C;
-  simt_gemm_f32<<<dim3(ceil_div(p.N, 64), ceil_div(p.M, 64)), 256, 0, st>>>(p);
+  launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(p.N, 64), ceil_div(p.M, 64))), dim3(256), 0, st, p);
   return last_launch();
 }
 
@@ -550,14 +574,14 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
             !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
           return EDIT_ERR_CUDA;
       }
-      dwconv_s2_tma_kernel<<<dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64)), 256, 0, st>>>(
+      launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64))), dim3(256), 0, st, 
           mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
           static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
           static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
       EDIT_TRY(last_launch());
     }
     const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
-    vtx_pad_rows_kernel<<<grid_for(padn, 256), 256, 0, st>>>(VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
+    launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
     EDIT_TRY(last_launch());
     stage_mark(2, st);
     TcGemmParams p;
@@ -585,7 +609,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   } else {
     {
       const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C);
-      dwconv_s2_kernel<T, 1><<<grid_for(total, 256), 256, 0, st>>>(
+      launch_pdl(dwconv_s2_kernel<T, 1>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
           reinterpret_cast<const T*>(ws + pl.KVp), pl.B, pl.H, pl.W, pl.C, static_cast<const T*>(w->kdw_w),
           static_cast<const T*>(w->kdw_b), static_cast<const T*>(w->vdw_w), static_cast<const T*>(w->vdw_b),
           reinterpret_cast<T*>(ws + pl.K), reinterpret_cast<T*>(ws + pl.V));
@@ -596,7 +620,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
     int threads = (nb * nb + 31) / 32 * 32;
     if (threads < pl.d) threads = (pl.d + 31) / 32 * 32;
     const size_t smem = 2 * 32 * static_cast<size_t>(pl.d) * sizeof(float);
-    kv_state_partial_kernel<T><<<dim3(pl.kv_chunks, pl.heads, pl.B), threads, smem, st>>>(
+    launch_pdl(kv_state_partial_kernel<T>, dim3(dim3(pl.kv_chunks, pl.heads, pl.B)), dim3(threads), smem, st, 
         reinterpret_cast<const T*>(ws + pl.K), reinterpret_cast<const T*>(ws + pl.V), pl.M, pl.C, pl.heads,
         pl.kv_chunks, reinterpret_cast<float*>(ws + pl.kvpart));
     EDIT_TRY(last_launch());
@@ -604,14 +628,14 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   {
     const int per_head = pl.d * (pl.d + 1);
     const long total = static_cast<long>(pl.B) * pl.heads * per_head;
-    kv_state_combine_kernel<<<grid_for(total, 256), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.kvpart),
+    launch_pdl(kv_state_combine_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.kvpart),
                                                                    pl.kv_chunks, per_head, total,
                                                                    reinterpret_cast<float*>(ws + pl.Sz));
     EDIT_TRY(last_launch());
   }
   if (pl.bf16) {
     const long total = static_cast<long>(pl.B) * pl.heads * pl.NP * pl.KP;
-    sz_pack_bf16_kernel<<<grid_for(total, 256), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.Sz), pl.d,
+    launch_pdl(sz_pack_bf16_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.Sz), pl.d,
                                                                pl.NP, pl.KP, total,
                                                                reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT));
     EDIT_TRY(last_launch());
@@ -627,7 +651,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
   const long tok = static_cast<long>(pl.B) * pl.HW;
   const int C = pl.C, Cr = pl.Cr;
   // 4. weight folding
-  transpose_kernel<T><<<dim3(ceil_div(Cr, 32), ceil_div(C, 32)), dim3(32, 8), 0, st>>>(
+  launch_pdl(transpose_kernel<T>, dim3(dim3(ceil_div(Cr, 32), ceil_div(C, 32))), dim3(dim3(32, 8)), 0, st, 
       static_cast<const T*>(w->cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t));
   EDIT_TRY(last_launch());
   if (pl.bf16) {
@@ -661,10 +685,10 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.N = Cr;
     p.out = reinterpret_cast<float*>(ws + pl.Wqw1);
     p.ldo = Cr;
-    simt_gemm_f32<<<dim3(ceil_div(Cr, 64), ceil_div(C, 64)), 256, 0, st>>>(p);
+    launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(C, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
-  fold_bias_kernel<T><<<C, 128, 0, st>>>(static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
+  launch_pdl(fold_bias_kernel<T>, dim3(C), dim3(128), 0, st, static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
                                          static_cast<const T*>(w->cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
   EDIT_TRY(last_launch());
   stage_mark(4, st);
@@ -700,25 +724,27 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
       p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
       bool split = false;
       EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
+      stage_mark(5, st);
       if (split) {
         const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
-        conv_fixup_kernel<<<grid_for(total, 256), 256, 0, st>>>(
+        launch_pdl(conv_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, 
             p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
             static_cast<const __nv_bfloat16*>(w->cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
         EDIT_TRY(last_launch());
       }
     } else {
       EDIT_TRY(gemm_conv(p, Cr, st));
+      stage_mark(5, st);
     }
     if ((Cr / pl.G) >= 8) {
       const int nvec = Cr / 8;
       const int kt = 256 / nvec > 0 ? 256 / nvec : 1;
       const int threads = kt * nvec;
-      gn_stats_bf16_kernel<<<dim3(pl.gn_P, pl.B), threads, threads * 4 * sizeof(float), st>>>(
+      launch_pdl(gn_stats_bf16_kernel, dim3(dim3(pl.gn_P, pl.B)), dim3(threads), threads * 4 * sizeof(float), st, 
           reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_chunk,
           pl.gn_P, gnpart);
     } else {
-      gn_partial_kernel<__nv_bfloat16><<<dim3(pl.gn_P, pl.B), 256, 0, st>>>(
+      launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, 
           reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
     }
     EDIT_TRY(last_launch());
@@ -739,15 +765,15 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.N = Cr;
     p.out = reinterpret_cast<float*>(ws + pl.U);
     p.ldo = Cr;
-    simt_gemm_f32<<<dim3(ceil_div(Cr, 64), ceil_div(tok, 64)), 256, 0, st>>>(p);
+    launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(tok, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
-    gn_partial_kernel<float><<<dim3(pl.gn_P, pl.B), 256, 0, st>>>(reinterpret_cast<const float*>(ws + pl.U),
+    stage_mark(5, st);
+    launch_pdl(gn_partial_kernel<float>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.U),
                                                                   static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
     EDIT_TRY(last_launch());
   }
-  stage_mark(5, st);
   // 6. G = LeakyReLU(GN(U))
-  gn_finalize_kernel<T><<<dim3(pl.G, pl.B), 256, 0, st>>>(gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
+  launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
                                               static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
                                               reinterpret_cast<float*>(ws + pl.gnstats),
                                               reinterpret_cast<float*>(ws + pl.gnss));
@@ -756,12 +782,12 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     const int nvec = Cr / 8;
     const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
     const int threads = per_block * nvec;
-    gn_apply_leaky_bf16x8<<<grid_for(tok, per_block), threads, 0, st>>>(
+    launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(threads), 0, st, 
         reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
         w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
   } else {
     const long total = tok * Cr;
-    gn_apply_leaky_kernel<float><<<grid_for(total, 256), 256, 0, st>>>(
+    launch_pdl(gn_apply_leaky_kernel<float>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
         reinterpret_cast<const float*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
         w->leaky_slope, reinterpret_cast<float*>(ws + pl.Gb), total);
   }
@@ -807,7 +833,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.ldo = C;
     p.bias[0] = reinterpret_cast<const float*>(ws + pl.bfold);
     p.relu = 1;
-    simt_gemm_f32<<<dim3(ceil_div(C, 64), ceil_div(tok, 64)), 256, 0, st>>>(p);
+    launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(C, 64), ceil_div(tok, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
   stage_mark(7, st);
@@ -848,7 +874,7 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(apply_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EDIT_ERR_CUDA;
-  apply_simt_kernel<T><<<dim3(ceil_div(pl.HW, 128), pl.heads, pl.B), 128, smem, st>>>(
+  launch_pdl(apply_simt_kernel<T>, dim3(dim3(ceil_div(pl.HW, 128), pl.heads, pl.B)), dim3(128), smem, st, 
       reinterpret_cast<const T*>(ws + pl.Q), reinterpret_cast<const float*>(ws + pl.Sz), static_cast<int>(pl.HW),
       pl.C, pl.heads, w->attn_eps, static_cast<T*>(out));
   return last_launch();
@@ -871,7 +897,7 @@ int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
   auto kern = sdpa_blend_kernel<T, D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EDIT_ERR_CUDA;
-  kern<<<dim3(ceil_div(p.Nq, 128), p.heads, B), 128, smem, st>>>(p);
+  launch_pdl(kern, dim3(dim3(ceil_div(p.Nq, 128), p.heads, B)), dim3(128), smem, st, p);
   return last_launch();
 }
 

@@ -58,6 +58,7 @@ __device__ __forceinline__ float simt_load_b(const SimtGemmParams& p, int n, int
 
 // 64 x 64 output tile, 256 threads, 4 x 4 outputs per thread (strided by 16).
 __global__ void __launch_bounds__(256) simt_gemm_f32(SimtGemmParams p) {
+  pdl_wait();
   __shared__ float As[16][65];
   __shared__ float Bs[16][65];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(256) simt_gemm_f32(SimtGemmParams p) {
 template <typename T>
 __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int groups, int chunks,
                                   float* __restrict__ part) {
+  pdl_wait();
   const int b = blockIdx.y, chunk = blockIdx.x;
   const int cpg = Cr / groups;
   const int t0 = static_cast<int>((static_cast<long>(HW) * chunk) / chunks);
@@ -153,6 +155,7 @@ __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int g
 // U [B][HW][Cr]; part[b][chunk][g][2]; blockDim = KT * (Cr / 8) threads.
 __global__ void gn_stats_bf16_kernel(const __nv_bfloat16* __restrict__ U, int HW, int Cr, int groups,
                                      int chunk_tokens, int chunks, float* __restrict__ part) {
+  pdl_wait();
   extern __shared__ float gs_red[];  // [KT * nvec][4]
   const int b = blockIdx.y, chunk = blockIdx.x;
   const int nvec = Cr / 8, KT = blockDim.x / nvec;
@@ -212,6 +215,7 @@ __global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restric
                                                           long count, float eps, const T* __restrict__ gamma,
                                                           const T* __restrict__ beta, float* __restrict__ stats,
                                                           float* __restrict__ ss) {
+  pdl_wait();
   const int g = blockIdx.x, b = blockIdx.y;
   const int cpg = Cr / groups;
   __shared__ double r1[256], r2[256];
@@ -250,6 +254,7 @@ __global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restric
 template <typename T>
 __global__ void gn_apply_leaky_kernel(const T* __restrict__ U, const float* __restrict__ ss, long HW, int Cr,
                                       float slope, T* __restrict__ G, long total) {
+  pdl_wait();
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(i % Cr);
@@ -266,6 +271,7 @@ __global__ void gn_apply_leaky_kernel(const T* __restrict__ U, const float* __re
 // Cr/8), so its scale/shift stay in registers across the tokens it visits.
 __global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const float* __restrict__ ss, long HW,
                                       int Cr, float slope, __nv_bfloat16* __restrict__ G, long tokens) {
+  pdl_wait();
   const int nvec = Cr / 8;
   const int per_block = blockDim.x / nvec;
   const int v = threadIdx.x % nvec, kt = threadIdx.x / nvec;
@@ -313,6 +319,7 @@ __global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const
 // W1 [C][Cr] -> W1t [Cr][C] and forms the folded bias (fp32).
 template <typename T>
 __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, T* __restrict__ dst) {
+  pdl_wait();
   __shared__ T tile[32][33];
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -329,6 +336,7 @@ __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, 
 template <typename T>
 __global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__ bq, const T* __restrict__ b1,
                                  int C, float* __restrict__ out) {
+  pdl_wait();
   const int c = blockIdx.x;
   float s = 0.f;
   for (int k = threadIdx.x; k < C; k += blockDim.x) s = fmaf(to_f32(wq[static_cast<long>(c) * C + k]), to_f32(b1[k]), s);
@@ -350,6 +358,7 @@ template <typename T, int VEC>
 __global__ void dwconv_s2_kernel(const T* __restrict__ kvp, int B, int H, int W, int C,
                                  const T* __restrict__ kw, const T* __restrict__ kb, const T* __restrict__ vw,
                                  const T* __restrict__ vb, T* __restrict__ K, T* __restrict__ V) {
+  pdl_wait();
   const int Ho = (H + 1) / 2, Wo = (W + 1) / 2;
   const int C2v = 2 * C / VEC;
   const long total = static_cast<long>(B) * Ho * Wo * C2v;
@@ -402,91 +411,6 @@ __global__ void dwconv_s2_kernel(const T* __restrict__ kvp, int B, int H, int W,
   }
 }
 
-// bf16 depthwise stride-2 conv with channel-major outputs for the tensor-core
-// KV state. Token index t = i * Wop + j over a padded output grid (Wop a
-// multiple of 32; columns j >= Wo are written as 0, so they add nothing to
-// S or z). Outputs:
-//   KT [B][C][Mp]               K = ReLU(DW_k(K')), channel-major
-//   VTx[B][heads][NP][Mp]       rows r < d: V = DW_v(V') of channel h*d + r
-//   Ktok, Vtok [B][Ho*Wo][C]    token-major copies (only when non-NULL)
-// Block: one output row i, 32 output columns, 64 of the 2C channels of
-// [K' | V']; the 3 x 65-pixel input patch is staged in shared memory with
-// 16-byte loads, results are transposed through shared memory so every
-// global store is a 16-byte vector.
-__global__ void __launch_bounds__(256) dwconv_s2_t_kernel(
-    const __nv_bfloat16* __restrict__ kvp, int H, int W, int C, int d, int heads, int Wop, int Mp, int NP,
-    const __nv_bfloat16* __restrict__ kw, const __nv_bfloat16* __restrict__ kb,
-    const __nv_bfloat16* __restrict__ vw, const __nv_bfloat16* __restrict__ vb, __nv_bfloat16* __restrict__ KT,
-    __nv_bfloat16* __restrict__ VTx, __nv_bfloat16* __restrict__ Ktok, __nv_bfloat16* __restrict__ Vtok) {
-  constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
-  __shared__ __align__(16) __nv_bfloat16 in_s[3][PW][CB];
-  __shared__ __align__(16) __nv_bfloat16 out_s[CB][JT + 8];
-  const int Ho = (H + 1) / 2, Wo = (W + 1) / 2;
-  const int j0 = blockIdx.x * JT, i = blockIdx.y;
-  const int nblk = 2 * C / CB;
-  const int b = blockIdx.z / nblk, cb = blockIdx.z - b * nblk;
-  const int gc0 = cb * CB;  // first channel of [K' | V']
-  const bool isk = gc0 < C;
-  const int ch0 = isk ? gc0 : gc0 - C;
-  // stage the input patch: rows 2i-1..2i+1, columns 2*j0-1 .. 2*j0+2*JT-1
-  for (int e = threadIdx.x; e < 3 * PW * (CB / 8); e += 256) {
-    const int v = e % (CB / 8);
-    const int col = (e / (CB / 8)) % PW;
-    const int a = e / (CB / 8 * PW);
-    const int hh = 2 * i + a - 1, ww = 2 * j0 + col - 1;
-    const bool in = hh >= 0 && hh < H && ww >= 0 && ww < W;
-    const __nv_bfloat16* src = in ? kvp + ((static_cast<long>(b) * H + hh) * W + ww) * (2L * C) + gc0 + v * 8 : kvp;
-    cp_async16(&in_s[a][col][v * 8], src, in ? 16u : 0u);
-  }
-  cp_async_wait_all();
-  const int c = threadIdx.x & (CB - 1);
-  const __nv_bfloat16* wt = isk ? kw : vw;
-  float wr[9];
-#pragma unroll
-  for (int q = 0; q < 9; ++q) wr[q] = __bfloat162float(wt[(ch0 + c) * 9 + q]);
-  const float bias = __bfloat162float((isk ? kb : vb)[ch0 + c]);
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < JT / 4; ++k) {
-    const int t = (threadIdx.x >> 6) + 4 * k;
-    const int j = j0 + t;
-    float acc = bias;
-#pragma unroll
-    for (int a = 0; a < 3; ++a)
-#pragma unroll
-      for (int e = 0; e < 3; ++e) acc = fmaf(wr[a * 3 + e], __bfloat162float(in_s[a][2 * t + e][c]), acc);
-    if (isk) acc = fmaxf(acc, 0.f);
-    if (j >= Wo) acc = 0.f;
-    out_s[c][t] = __float2bfloat16_rn(acc);
-  }
-  __syncthreads();
-  {  // channel-major store: 64 rows x 32 tokens, one 16-byte vector per thread
-    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
-    const int ch = ch0 + r;
-    const long t0 = static_cast<long>(i) * Wop + j0 + q * 8;
-    __nv_bfloat16* dst;
-    if (isk) {
-      dst = KT + (static_cast<long>(b) * C + ch) * Mp + t0;
-    } else {
-      const int h = ch / d, rr = ch - h * d;
-      dst = VTx + ((static_cast<long>(b) * heads + h) * NP + rr) * Mp + t0;
-    }
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&out_s[r][q * 8]);
-  }
-  __nv_bfloat16* tok = isk ? Ktok : Vtok;
-  if (tok) {  // token-major store: 32 tokens x 64 channels
-    const int t = threadIdx.x >> 3, v = threadIdx.x & 7;
-    const int j = j0 + t;
-    if (j < Wo) {
-      __align__(16) __nv_bfloat16 tmp[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) tmp[u] = out_s[v * 8 + u][t];
-      *reinterpret_cast<uint4*>(tok + ((static_cast<long>(b) * Ho + i) * Wo + j) * C + ch0 + v * 8) =
-          *reinterpret_cast<const uint4*>(tmp);
-    }
-  }
-}
-
 // TMA version of the channel-major depthwise conv (same outputs as
 // dwconv_s2_t_kernel): the 3 x 65-pixel, 64-channel input patch arrives in one
 // tensor load (zero-filled outside the grid). Thread (tg, c) computes the 8
@@ -513,6 +437,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
                                                             const __nv_bfloat16* __restrict__ vw,
                                                             const __nv_bfloat16* __restrict__ vb, int tokmajor,
                                                             int* status) {
+  pdl_wait();
   constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
   __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
   __shared__ __align__(128) __nv_bfloat16 in_s[3][PW][CB];
@@ -604,6 +529,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
 // KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
 // (Mp % 8 == 0).
 __global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
+  pdl_wait();
   const int vpr = Mp / 8;                   // vectors per row
   const int rows = NP - d;
   const long total = static_cast<long>(BH) * rows * vpr;
@@ -627,6 +553,7 @@ __global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int
 __global__ void conv_fixup_kernel(const float* __restrict__ part, int split_first, int split_count, int tiles_w,
                                   int tiles_h, int H, int W, int Cr, const __nv_bfloat16* __restrict__ bias,
                                   int num_m_tiles, __nv_bfloat16* __restrict__ U) {
+  pdl_wait();
   const int cv = Cr / 4;
   const int total = split_count * 2 * 128 * cv;
   const int per = 2 * 128 * Cr;  // one split tile, one half
@@ -660,6 +587,7 @@ __global__ void conv_fixup_kernel(const float* __restrict__ part, int split_firs
 template <typename T>
 __global__ void kv_state_partial_kernel(const T* __restrict__ K, const T* __restrict__ V, int M, int C, int heads,
                                         int chunks, float* __restrict__ part) {
+  pdl_wait();
   const int d = C / heads;
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t0 = static_cast<int>((static_cast<long>(M) * chunk) / chunks);
@@ -723,6 +651,7 @@ __global__ void kv_state_partial_kernel(const T* __restrict__ K, const T* __rest
 // Fixed-order sum of the chunk partials: Sz[b][h][a][c] (fp32).
 __global__ void kv_state_combine_kernel(const float* __restrict__ part, int chunks, int per_head, long total,
                                         float* __restrict__ Sz) {
+  pdl_wait();
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
     const long bh = i / per_head;
@@ -739,6 +668,7 @@ __global__ void kv_state_combine_kernel(const float* __restrict__ part, int chun
 // c in (d, NP) and a in [d, KP).
 __global__ void sz_pack_bf16_kernel(const float* __restrict__ Sz, int d, int NP, int KP, long total,
                                     __nv_bfloat16* __restrict__ SzT) {
+  pdl_wait();
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
     const int a = static_cast<int>(i % KP);
@@ -757,6 +687,7 @@ __global__ void sz_pack_bf16_kernel(const float* __restrict__ Sz, int d, int NP,
 template <typename T>
 __global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restrict__ Sz, int N, int C, int heads,
                                   float eps, T* __restrict__ out) {
+  pdl_wait();
   const int d = C / heads;
   const int h = blockIdx.y, b = blockIdx.z;
   extern __shared__ float ap_sm[];  // [d][d+1]
@@ -847,6 +778,7 @@ __device__ __forceinline__ void sdpa_one_set(const T* kb, const T* vb, long ld, 
 
 template <typename T, int D>
 __global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
+  pdl_wait();
   extern __shared__ float sd_sm[];
   float* ks = sd_sm;                 // [64][D]
   float* vs = sd_sm + 64 * D;        // [64][D]

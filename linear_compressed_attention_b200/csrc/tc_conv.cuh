@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs of this grid are ready past this point
 
   if (warp == 0) {
     // ------------------------------------------------------------ producers

@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs of this grid are ready past this point
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -642,6 +643,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
   cluster_sync_all();  // both CTAs' barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs of this grid are ready past this point
 
   if (warp == 0) {
     // ------------------------------------------------------------ producers (both CTAs)
