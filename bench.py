@@ -35,14 +35,16 @@ STAGES = ["kv_linear", "dwconv_s2", "kv_state", "fold_weights", "conv3x3", "grou
 # conv's last-wave fixup)
 DOMINANT = "conv3x3"   # largest FLOP share of the layer (40%)
 
-# DRAM traffic of the dominant kernel from an ncu capture (profiles/), valid
-# only while the kernel sources are unchanged (hash of tc_gemm.cuh + common.cuh).
-TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the dominant kernel, from the ncu capture summarised in
+# profiles/conv3x3_px4096.md; reported only while the kernel's sources are the
+# ones that capture measured (hash of tc_conv.cuh + tc_gemm.cuh + common.cuh).
+TRAFFIC = {"src_sha": "f3b2f953d4bfebb8", "bytes_per_launch": 159513344 + 25180160}
 
 
 def kernel_src_sha():
     h = hashlib.sha256()
-    for f in ("tc_gemm.cuh", "common.cuh"):
+    for f in ("tc_conv.cuh", "tc_gemm.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "linear_compressed_attention_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
