@@ -441,9 +441,10 @@ int gemm_linear_pair(TcGemmParams& p, cudaStream_t st) {
   return launch_pair<kPairBN, 1, 5, EPI_LINEAR>(p, st);
 }
 
-// Small Linear GEMMs (weight folding) on single CTAs: 128 x 128 tiles.
+// Small Linear GEMMs (weight folding) on single CTAs: 128 x 32 tiles, so the
+// 1152 x 288 product spreads over 81 SMs.
 int gemm_linear(const TcGemmParams& p, int bn, cudaStream_t st) {
-  if (bn == 128) return launch_tc<128, 1, 6, EPI_LINEAR>(p, st);
+  if (bn == 32) return launch_tc<32, 1, 8, EPI_LINEAR>(p, st);
   return EDIT_ERR_UNSUPPORTED;
 }
 
@@ -581,7 +582,8 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
       EDIT_TRY(last_launch());
     }
     const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
-    launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP, pl.Mp);
+    launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP,
+               pl.Mp, reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT), pl.KP);
     EDIT_TRY(last_launch());
     stage_mark(2, st);
     TcGemmParams p;
@@ -628,16 +630,15 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   {
     const int per_head = pl.d * (pl.d + 1);
     const long total = static_cast<long>(pl.B) * pl.heads * per_head;
-    launch_pdl(kv_state_combine_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.kvpart),
-                                                                   pl.kv_chunks, per_head, total,
-                                                                   reinterpret_cast<float*>(ws + pl.Sz));
-    EDIT_TRY(last_launch());
-  }
-  if (pl.bf16) {
-    const long total = static_cast<long>(pl.B) * pl.heads * pl.NP * pl.KP;
-    launch_pdl(sz_pack_bf16_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.Sz), pl.d,
-                                                               pl.NP, pl.KP, total,
-                                                               reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT));
+    if (pl.bf16) {
+      launch_pdl(kv_state_combine_pack_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st,
+                 reinterpret_cast<const float*>(ws + pl.kvpart), pl.kv_chunks, pl.d, pl.NP, pl.KP, total,
+                 reinterpret_cast<float*>(ws + pl.Sz), reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT));
+    } else {
+      launch_pdl(kv_state_combine_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st,
+                 reinterpret_cast<const float*>(ws + pl.kvpart), pl.kv_chunks, per_head, total,
+                 reinterpret_cast<float*>(ws + pl.Sz));
+    }
     EDIT_TRY(last_launch());
   }
   stage_mark(3, st);
@@ -659,7 +660,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     std::memset(&p, 0, sizeof(p));
     if (!map_a(&p.a0, w->q_w, C, C, 1, C, static_cast<long>(C) * C)) return EDIT_ERR_CUDA;
     p.a1 = p.a0;
-    if (!map_b(&p.b0, ws + pl.W1t, C, Cr, C, 128)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, ws + pl.W1t, C, Cr, C, 32)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.bk = p.b0;
     p.R = C;
     p.m_tiles_per_img = ceil_div(C, 128);
@@ -668,12 +669,12 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.kb_split = p.num_kb;
     p.n_split = Cr;
     p.N = Cr;
-    p.num_n_tiles = ceil_div(Cr, 128);
+    p.num_n_tiles = ceil_div(Cr, 32);
     p.num_tiles = p.m_tiles_per_img * p.num_n_tiles;
     p.out = ws + pl.Wqw1;
     p.ldo = Cr;
     p.status = status;
-    EDIT_TRY(gemm_linear(p, 128, st));
+    EDIT_TRY(gemm_linear(p, 32, st));
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -688,7 +689,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(C, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
-  launch_pdl(fold_bias_kernel<T>, dim3(C), dim3(128), 0, st, static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
+  launch_pdl(fold_bias_kernel<T>, dim3(ceil_div(C, 8)), dim3(256), 0, st, static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
                                          static_cast<const T*>(w->cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
   EDIT_TRY(last_launch());
   stage_mark(4, st);

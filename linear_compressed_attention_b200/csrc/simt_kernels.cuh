@@ -207,28 +207,29 @@ __global__ void gn_stats_bf16_kernel(const __nv_bfloat16* __restrict__ U, int HW
 // Fixed-order (deterministic) combine of the partials in fp64, then the
 // per-channel affine form of GN: scale = gamma * rstd, shift = beta - mean * scale.
 // part: [B][P][groups][2]; stats out: [B][groups][2] (mean, rstd);
-// ss out: [B][Cr][2] (scale, shift). One block of 256 threads per (group,
-// batch item): thread t sums partials t, t+256, ... in order, then a fixed
-// shared-memory tree.
+// ss out: [B][Cr][2] (scale, shift). A block of up to 256 threads handles one
+// (group, image): thread t sums partials t, t+blockDim, ... in order, then a
+// fixed shared-memory tree (blockDim a power of two).
 template <typename T>
-__global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr,
-                                                          long count, float eps, const T* __restrict__ gamma,
-                                                          const T* __restrict__ beta, float* __restrict__ stats,
-                                                          float* __restrict__ ss) {
-  pdl_wait();
-  const int g = blockIdx.x, b = blockIdx.y;
+__device__ void gn_finalize_body(const float* __restrict__ part, int P, int groups, int Cr, long count, float eps,
+                                 const T* __restrict__ gamma, const T* __restrict__ beta, float* __restrict__ stats,
+                                 float* __restrict__ ss, int g, int b, double* r1, double* r2) {
   const int cpg = Cr / groups;
-  __shared__ double r1[256], r2[256];
+  const int nt = blockDim.x >= 256 ? 256 : 128;
   double s1 = 0.0, s2 = 0.0;
-  for (int i = threadIdx.x; i < P; i += 256) {
-    const float2 q = *reinterpret_cast<const float2*>(part + ((static_cast<long>(b) * P + i) * groups + g) * 2);
-    s1 += q.x;
-    s2 += q.y;
-  }
-  r1[threadIdx.x] = s1;
-  r2[threadIdx.x] = s2;
+  if (threadIdx.x < nt)
+    for (int i = threadIdx.x; i < P; i += nt) {
+      const float2 q = *reinterpret_cast<const float2*>(part + ((static_cast<long>(b) * P + i) * groups + g) * 2);
+      s1 += q.x;
+      s2 += q.y;
+    }
   __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
+  if (threadIdx.x < nt) {
+    r1[threadIdx.x] = s1;
+    r2[threadIdx.x] = s2;
+  }
+  __syncthreads();
+  for (int w = nt / 2; w > 0; w >>= 1) {
     if (threadIdx.x < w) {
       r1[threadIdx.x] += r1[threadIdx.x + w];
       r2[threadIdx.x] += r2[threadIdx.x + w];
@@ -243,11 +244,22 @@ __global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restric
     stats[(b * groups + g) * 2] = static_cast<float>(mean);
     stats[(b * groups + g) * 2 + 1] = static_cast<float>(rstd);
   }
-  for (int c = g * cpg + threadIdx.x; c < (g + 1) * cpg; c += 256) {
+  for (int c = g * cpg + threadIdx.x; c < (g + 1) * cpg; c += blockDim.x) {
     const double sc = static_cast<double>(to_f32(gamma[c])) * rstd;
     ss[(static_cast<long>(b) * Cr + c) * 2] = static_cast<float>(sc);
     ss[(static_cast<long>(b) * Cr + c) * 2 + 1] = static_cast<float>(static_cast<double>(to_f32(beta[c])) - mean * sc);
   }
+  __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr,
+                                                          long count, float eps, const T* __restrict__ gamma,
+                                                          const T* __restrict__ beta, float* __restrict__ stats,
+                                                          float* __restrict__ ss) {
+  pdl_wait();
+  __shared__ double r1[256], r2[256];
+  gn_finalize_body<T>(part, P, groups, Cr, count, eps, gamma, beta, stats, ss, blockIdx.x, blockIdx.y, r1, r2);
 }
 
 // G = LeakyReLU(scale * U + shift), elementwise over [B][HW][Cr].
@@ -333,22 +345,29 @@ __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, 
   }
 }
 
+// bq' = Wq b1 + bq, one warp per output row (fp32).
 template <typename T>
 __global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__ bq, const T* __restrict__ b1,
                                  int C, float* __restrict__ out) {
   pdl_wait();
-  const int c = blockIdx.x;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= C) return;
   float s = 0.f;
-  for (int k = threadIdx.x; k < C; k += blockDim.x) s = fmaf(to_f32(wq[static_cast<long>(c) * C + k]), to_f32(b1[k]), s);
-  s = warp_sum(s);
-  __shared__ float red[32];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
-    out[c] = t + to_f32(bq[c]);
+  if (sizeof(T) == 2 && (C & 7) == 0) {  // 8 elements per 16-byte load
+    for (int k = lane * 8; k < C; k += 256) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(wq + static_cast<long>(row) * C + k);
+      const uint4 bv = *reinterpret_cast<const uint4*>(b1 + k);
+      const T* w8 = reinterpret_cast<const T*>(&wv);
+      const T* b8 = reinterpret_cast<const T*>(&bv);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s = fmaf(to_f32(w8[j]), to_f32(b8[j]), s);
+    }
+  } else {
+    for (int k = lane; k < C; k += 32) s = fmaf(to_f32(wq[static_cast<long>(row) * C + k]), to_f32(b1[k]), s);
   }
+  s = warp_sum(s);
+  if (lane == 0) out[row] = s + to_f32(bq[row]);
 }
 
 // ====================================================== depthwise stride-2
@@ -528,8 +547,18 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
 // Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
 // KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
 // (Mp % 8 == 0).
-__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
+__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp,
+                                    __nv_bfloat16* __restrict__ SzT, int KP) {
   pdl_wait();
+  // also the zero padding of the apply operand SzT [BH][NP][KP]: rows c in
+  // (d, NP) and columns a in [d, KP) of rows c <= d (the combine fills the rest)
+  const long szn = static_cast<long>(BH) * NP * KP;
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < szn;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int a = static_cast<int>(i % KP);
+    const int c = static_cast<int>((i / KP) % NP);
+    if (c > d || a >= d) SzT[i] = __float2bfloat16_rn(0.f);
+  }
   const int vpr = Mp / 8;                   // vectors per row
   const int rows = NP - d;
   const long total = static_cast<long>(BH) * rows * vpr;
@@ -663,21 +692,24 @@ __global__ void kv_state_combine_kernel(const float* __restrict__ part, int chun
   }
 }
 
-// [S_h | z_h] as the bf16 B operand of the tensor-core apply:
-// SzT[(b*heads + h)*NP + c][a] = Sz[b][h][a][c] for c <= d, a < d; zero for
-// c in (d, NP) and a in [d, KP).
-__global__ void sz_pack_bf16_kernel(const float* __restrict__ Sz, int d, int NP, int KP, long total,
-                                    __nv_bfloat16* __restrict__ SzT) {
+// Same fixed-order combine, also writing [S_h | z_h] as the bf16 B operand of
+// the tensor-core apply: SzT[(b*heads + h)*NP + c][a] = Sz[b][h][a][c] for
+// c <= d, a < d. The zero padding of SzT (c in (d, NP), a in [d, KP)) is
+// written by vtx_pad_rows_kernel.
+__global__ void kv_state_combine_pack_kernel(const float* __restrict__ part, int chunks, int d, int NP, int KP,
+                                             long total, float* __restrict__ Sz, __nv_bfloat16* __restrict__ SzT) {
   pdl_wait();
+  const int per_head = d * (d + 1);
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const int a = static_cast<int>(i % KP);
-    const long r = i / KP;
-    const int c = static_cast<int>(r % NP);
-    const long bh = r / NP;
-    float v = 0.f;
-    if (a < d && c <= d) v = Sz[(bh * d + a) * (d + 1) + c];
-    SzT[i] = __float2bfloat16_rn(v);
+    const long bh = i / per_head;
+    const int e = static_cast<int>(i - bh * per_head);
+    const int a = e / (d + 1), c = e - a * (d + 1);
+    const float* q = part + bh * chunks * per_head + e;
+    float s = 0.f;
+    for (int k = 0; k < chunks; ++k) s += q[static_cast<long>(k) * per_head];
+    Sz[i] = s;
+    SzT[(bh * NP + c) * KP + a] = __float2bfloat16_rn(s);
   }
 }
 

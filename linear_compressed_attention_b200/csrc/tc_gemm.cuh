@@ -232,7 +232,13 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileC
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 64) {
       float v[64];
-      tmem_ld64(t_row + c0, v);  // columns past BN belong to nobody here and are not used
+      if (c0 + 64 <= BN || BN >= 256) {
+        tmem_ld64(t_row + c0, v);  // (BN >= 256: columns past BN are still inside the 512-column allocation)
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (c0 + 16 * j < BN) tmem_ld16(t_row + c0 + 16 * j, *reinterpret_cast<float(*)[16]>(&v[16 * j]));
+      }
 #pragma unroll
       for (int g16 = 0; g16 < 4; ++g16) {
         const int col = c0 + 16 * g16;
