@@ -136,7 +136,13 @@ EDIT_API int mmedit_hybrid_forward(const void *x_img, const void *x_txt, int B, 
 
 /* Copy the device status word of a workspace to *status (0 = no device-side
  * error since the last forward call on it) and synchronise `stream`. This is
- * the only call that waits. */
+ * the only call that waits. When a tensor-core kernel's bounded wait ran out
+ * (EDIT_ERR_TIMEOUT), the seven int32 words after the status word (offset
+ * layout.status + 4) name the first wait that gave up: site (2: MMA issuer
+ * waiting for a free accumulator, 3: MMA issuer waiting for operands,
+ * 10 + w: producer warp w waiting for a free stage, 20 + 10 r + q: epilogue
+ * warp q of pair rank r waiting for an accumulator), block, tile, k-block (or
+ * tiles done), stage or accumulator, barrier parity, globaltimer low bits. */
 EDIT_API int edit_attn_read_status(const void *workspace, void *stream, int *status);
 
 /* Text for a status code (static storage). */

@@ -43,6 +43,22 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Where a bounded wait gave up: the first waiter that timed out fills
+// status[1..7] with (site, block, tile, k-block, stage, parity, globaltimer
+// low bits); the words sit in the workspace's status block next to the
+// status word and are read back when EDIT_ERR_TIMEOUT is reported.
+__device__ __forceinline__ void record_wait_site(int* status, int site, int tile, int kb, int stage, int parity) {
+  int* w = status + 1;
+  if (status && atomicCAS(w, 0, site) == 0) {
+    w[1] = static_cast<int>(blockIdx.x);
+    w[2] = tile;
+    w[3] = kb;
+    w[4] = stage;
+    w[5] = parity;
+    w[6] = static_cast<int>(globaltimer_ns() & 0x7fffffff);
+  }
+}
+
 // ----------------------------------------------------------------- PDL
 // Programmatic dependent launch: every kernel of the library calls this before
 // touching memory written by the kernel before it in the stream (a no-op when
@@ -88,7 +104,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Returns false when the
 // block was aborted (by this waiter's timeout or by another role's).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, int* timed_out = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -97,6 +113,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (globaltimer_ns() - t0 > EDIT_WAIT_TIMEOUT_NS) {
       *abort_flag = 1;
       record_status(status, EDIT_ERR_TIMEOUT);
+      if (timed_out) *timed_out = 1;
       return false;
     }
   }

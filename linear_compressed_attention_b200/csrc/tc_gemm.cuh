@@ -99,9 +99,10 @@ struct TcGemmCfg {
 
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          int* timed_out = nullptr) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, timed_out) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
 }
@@ -684,12 +685,18 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int pt = pair; pt < p.num_tiles && !*abort_flag; pt += npairs) {
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        int to = 0;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status, &to)) {
+          if (to) record_wait_site(p.status, 2, pt, -1, acc, acc_phase ^ 1);
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
+          int to = 0;
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status, &to)) {
+            if (to) record_wait_site(p.status, 3, pt, kb, stage, phase);
             ok = false;
             break;
           }
@@ -726,16 +733,21 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     uint8_t* stg = stg_base + q * 8192;
     int sbuf = 0;
-    int acc = 0;
+    int acc = 0, ntile_done = 0;
     uint32_t acc_phase = 0;
     for (int pt = pair; pt < p.num_tiles; pt += npairs) {
-      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status)) break;
+      int to = 0;
+      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status, &to)) {
+        if (lane == 0 && to) record_wait_site(p.status, 20 + rank * 10 + (warp & 3), pt, ntile_done, acc, acc_phase);
+        break;
+      }
       tc_fence_after();
       const TileCoord tc = decode_pair_tile<EPI>(p, pt, rank);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
       epilogue_tile_staged<BN, EPI>(p, tc, t_row, q, lane, stg, sbuf);
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      ++ntile_done;
       if (++acc == ACC) {
         acc = 0;
         acc_phase ^= 1;
