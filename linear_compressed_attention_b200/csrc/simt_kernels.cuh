@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
     }
     if (tokmajor && j0 < Wo) tma_store_4d(isk ? &m.ktok : &m.vtok, &tok_s[0][0], ch0, j0, i, b);
     bulk_commit();
-    bulk_wait_all();
+    bulk_wait_read<0>();  // shared memory may be released once the stores have read it
   }
 }
 

@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       }
     }
     if (STG > 0) {
-      if (lane == 0) bulk_wait_all();  // staged stores finished before shared memory is released
+      if (lane == 0) bulk_wait_read<0>();  // staged stores have read shared memory before it is released
       __syncwarp();
     }
   }
@@ -753,7 +753,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
         acc_phase ^= 1;
       }
     }
-    if (lane == 0) bulk_wait_all();  // staged stores finished before shared memory is released
+    if (lane == 0) bulk_wait_read<0>();  // staged stores have read shared memory before it is released
     __syncwarp();
   }
 
