@@ -140,6 +140,7 @@ EDIT_API int mmedit_hybrid_forward(const void *x_img, const void *x_txt, int B, 
  * (EDIT_ERR_TIMEOUT), the seven int32 words after the status word (offset
  * layout.status + 4) name the first wait that gave up: site (2: MMA issuer
  * waiting for a free accumulator, 3: MMA issuer waiting for operands,
+ * 4: conv MMA issuer waiting for its input patch,
  * 10 + w: producer warp w waiting for a free stage, 20 + 10 r + q: epilogue
  * warp q of pair rank r waiting for an accumulator), block, tile, k-block (or
  * tiles done), stage or accumulator, barrier parity, globaltimer low bits. */

@@ -385,7 +385,7 @@ int launch_conv_pair(TcGemmParams& p, cudaStream_t st, bool* split_out) {
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(conv_threads(NSPLIT), 1, 1);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -421,9 +421,9 @@ int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st, bool* split) {
   switch (cr) {
     case 64: return launch_conv_pair<64, 1, 8>(p, st, split);
     case 128: return launch_conv_pair<128, 1, 8>(p, st, split);
-    case 256: return launch_conv_pair<256, 1, 7>(p, st, split);
-    case 288: return launch_conv_pair<288, 2, 7>(p, st, split);
-    case 384: return launch_conv_pair<384, 2, 5>(p, st, split);
+    case 256: return launch_conv_pair<256, 1, 5>(p, st, split);
+    case 288: return launch_conv_pair<288, 2, 5>(p, st, split);
+    case 384: return launch_conv_pair<384, 2, 3>(p, st, split);
   }
   return EDIT_ERR_UNSUPPORTED;
 }

@@ -6,11 +6,17 @@
 // descriptor start offset; the swizzle follows the absolute address). Only the weights
 // stream per tap. Requires tiles of 128 consecutive pixels of one image row
 // (TW = 128, TH = 1, i.e. W >= 128). The epilogue only adds the bias and
-// stores U (GroupNorm statistics are a separate pass over U), so the
-// non-overlapped epilogue of the single TMEM accumulator stays short.
+// stores U through 128B-swizzled shared-memory blocks and TMA tensor stores
+// (GroupNorm statistics are a separate pass over U), so the non-overlapped
+// epilogue of the single TMEM accumulator stays short.
 //
-// Roles as in the pair GEMM: warp 0 producer (both CTAs), warp 1 TMEM owner
-// and (leader) MMA issuer, warps 2..5 epilogue (bias + U store).
+// Roles: warp 0 producer (both CTAs), warp 1 TMEM owner and (leader) MMA
+// issuer of output chunk 0, warps 2..5 epilogue (bias + staged U store), and
+// with NSPLIT > 1 warps 6.. issue the MMAs of chunks 1.. (leader). One issuing
+// thread per accumulator chunk: a tcgen05.mma costs its issuing thread tens of
+// cycles, more than an N = 144 MMA leaves between issues when one thread
+// feeds two accumulators. Every issuer waits on the same operand barriers
+// and commits to the shared empty / TMEM-full barriers (NSPLIT arrivals).
 #pragma once
 
 #include "tc_gemm.cuh"
@@ -28,7 +34,7 @@ struct ConvPairCfg {
   static constexpr int B_BYTES = NSPLIT * BROWS * 128;                 // per CTA per tap
   static constexpr int ACC = (2 * BN <= 512) ? 2 : 1;
   static constexpr int TMEM_COLS = (ACC * BN <= 128) ? 128 : (ACC * BN <= 256) ? 256 : 512;
-  static constexpr int STG_BYTES = 0;  // U is small: direct 16-byte stores, no staging
+  static constexpr int STG_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x (32 rows x 128 B)
   static constexpr int BAR_BYTES = (2 * 2 + 2 * NB + 2 * ACC) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 + 2 * PATCH_BYTES + NB * B_BYTES + STG_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -57,8 +63,10 @@ __device__ __forceinline__ ConvItem conv_item(const TcGemmParams& p, int it, int
   return c;
 }
 
+constexpr int conv_threads(int nsplit) { return 192 + 32 * (nsplit - 1); }
+
 template <int BN, int NSPLIT, int NB>
-__global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(conv_threads(NSPLIT), 1) tc_conv_pair_kernel(const __grid_constant__ TcGemmParams p) {
   using Cfg = ConvPairCfg<BN, NSPLIT, NB>;
   constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
   extern __shared__ uint8_t smem_raw[];
@@ -83,14 +91,14 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_empty[i], NSPLIT);
     }
     for (int i = 0; i < NB; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
+      mbar_init(&b_empty[i], NSPLIT);
     }
     for (int a = 0; a < ACC; ++a) {
-      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tfull_bar[a], NSPLIT);
       mbar_init(&tempty_bar[a], 256);
     }
     *abort_flag = 0;
@@ -153,41 +161,43 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
+  } else if (warp == 1 || warp >= 6) {
+    // ------------------------------------------------------------ MMA issuers (leader), one per chunk
     if (leader && lane == 0) {
+      const int sc = warp == 1 ? 0 : warp - 5;  // output chunk of this thread
       int ai = 0, bi = 0, acc = 0;
       uint32_t aph = 0, bph = 0, acc_phase = 0;
       bool ok = true;
       for (int it = pair; it < p.num_tiles && ok && !*abort_flag; it += npairs) {
         const ConvItem ci = conv_item(p, it, ncb);
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        int to = 0;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag, p.status, &to)) {
+          if (to) record_wait_site(p.status, 2, ci.pt, -1, acc, acc_phase ^ 1);
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * BN + sc * NCHUNK;
         for (int cb = ci.cb0; cb < ci.cb1 && ok; ++cb) {
-          if (!mbar_wait(&a_full[ai], aph, abort_flag, p.status)) {
+          if (!mbar_wait(&a_full[ai], aph, abort_flag, p.status, &to)) {
+            if (to) record_wait_site(p.status, 4, ci.pt, cb, ai, aph);
             ok = false;
             break;
           }
           const uint32_t patch = smem_u32(sA + ai * Cfg::PATCH_BYTES);
           for (int tap = 0; tap < 9; ++tap) {
-            if (!mbar_wait(&b_full[bi], bph, abort_flag, p.status)) {
+            if (!mbar_wait(&b_full[bi], bph, abort_flag, p.status, &to)) {
+              if (to) record_wait_site(p.status, 3, ci.pt, cb, bi, bph);
               ok = false;
               break;
             }
             tc_fence_after();
+            // descriptors of k-step k are the k = 0 ones plus 32 bytes (2 in the address field) per step
             const int off = (tap / 3) * Cfg::PATCH_W + tap % 3;  // first patch row of this tap's operand
-            const uint32_t a_addr = patch + off * 128;
-            const uint32_t b_addr = smem_u32(sB + bi * Cfg::B_BYTES);
+            const uint64_t adesc = sdesc_kmajor_sw128(patch + off * 128);
+            const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + bi * Cfg::B_BYTES) + sc * Cfg::BROWS * 128);
+            const uint32_t first = (cb != ci.cb0 || tap != 0) ? 1u : 0u;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t adesc = sdesc_kmajor_sw128(a_addr + k * 32);
-#pragma unroll
-              for (int s = 0; s < NSPLIT; ++s) {
-                const uint64_t bdesc = sdesc_kmajor_sw128(b_addr + s * Cfg::BROWS * 128 + k * 32);
-                umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (cb != ci.cb0 || tap | k) ? 1u : 0u);
-              }
-            }
+            for (int k = 0; k < 4; ++k) umma2_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, Cfg::IDESC, k ? 1u : first);
             umma2_commit_mc(&b_empty[bi], 0x3);
             if (++bi == NB) {
               bi = 0;
@@ -214,6 +224,8 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    uint8_t* stg = sB + NB * Cfg::B_BYTES + q * 8192;  // 1024-byte aligned staging of this warp
+    int sbuf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = pair; it < p.num_tiles; it += npairs) {
@@ -223,7 +235,7 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
       const TileCoord tc = decode_pair_tile<EPI_CONV>(p, ci.pt, rank);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
       if (ci.half < 0) {
-        epilogue_tile<BN, EPI_CONV>(p, tc, t_row, q, lane);
+        epilogue_tile_staged<BN, EPI_CONV>(p, tc, t_row, q, lane, stg, sbuf);
       } else {  // fp32 partial of this half, row q*32 + lane
         float* prow = p.fix_part + ((((static_cast<long>(ci.pt - p.split_first) * 2 + ci.half) * 2 + rank) * 128) +
                                     q * 32 + lane) * p.N;
@@ -244,6 +256,8 @@ __global__ void __launch_bounds__(192, 1) tc_conv_pair_kernel(const __grid_const
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_read<0>();  // staged stores have read shared memory before it is released
+    __syncwarp();
   }
 
   tc_fence_before();
