@@ -350,7 +350,7 @@ int launch_pair(const TcGemmParams& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(pair_threads(NSPLIT), 1, 1);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -434,11 +434,15 @@ int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
 
 // Linear GEMMs on CTA pairs: 256 x 256 pair tiles.
 constexpr int kPairBN = 256;
+// One N = 256 MMA per k-step: the linear projections are bound by operand
+// ingest, and two 128-column chunks would halve the weight box height.
+constexpr int kPairNS = 1;
+constexpr int kPairBox = kPairBN / (2 * kPairNS);  // B rows per CTA per chunk
 int gemm_linear_pair(TcGemmParams& p, cudaStream_t st) {
   const int m_pairs = (p.num_m_tiles + 1) / 2;
   p.num_n_tiles = (p.N + kPairBN - 1) / kPairBN;
   p.num_tiles = m_pairs * p.num_n_tiles;
-  return launch_pair<kPairBN, 1, 5, EPI_LINEAR>(p, st);
+  return launch_pair<kPairBN, kPairNS, 5, EPI_LINEAR>(p, st);
 }
 
 // Small Linear GEMMs (weight folding) on single CTAs: 128 x 32 tiles, so the
@@ -491,7 +495,7 @@ int tc_linear(const void* a, long rows, int K, const void* const* wts, const voi
   p.a1 = p.a0;
   CUtensorMap* bm[3] = {&p.b0, &p.b1, &p.b2};
   for (int s = 0; s < 3; ++s)
-    if (!map_b(bm[s], wts[s < nsrc ? s : 0], K, C, K, kPairBN / 2)) return EDIT_ERR_CUDA;
+    if (!map_b(bm[s], wts[s < nsrc ? s : 0], K, C, K, kPairBox)) return EDIT_ERR_CUDA;
   (void)bn;
   p.bk = p.b0;
   p.R = static_cast<int>(rows);
@@ -800,8 +804,8 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     std::memset(&p, 0, sizeof(p));
     if (!map_a(&p.a0, x, C, tok, 1, C, tok * C)) return EDIT_ERR_CUDA;
     if (!map_a(&p.a1, ws + pl.Gb, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
-    if (!map_b(&p.b0, w->q_w, C, C, C, kPairBN / 2)) return EDIT_ERR_CUDA;
-    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, kPairBN / 2)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, w->q_w, C, C, C, kPairBox)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, kPairBox)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.b0;
     p.R = static_cast<int>(tok);
     p.m_tiles_per_img = ceil_div(tok, 128);

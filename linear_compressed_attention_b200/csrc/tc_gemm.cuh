@@ -609,8 +609,14 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
   }
 }
 
+// One MMA-issuing thread per output chunk (warp 1: chunk 0, warps 6..: chunks
+// 1..): a tcgen05.mma costs its issuing thread tens of cycles, so one thread
+// cannot keep several short MMAs per k-step back to back. Every issuer waits
+// on the same full barriers; empty and TMEM-full barriers take NSPLIT commits.
+constexpr int pair_threads(int nsplit) { return 192 + 32 * (nsplit - 1); }
+
 template <int BN, int NSPLIT, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(const __grid_constant__ TcGemmParams p) {
   using Cfg = TcPairCfg<BN, NSPLIT, STAGES>;
   constexpr int NCHUNK = Cfg::NCHUNK, ACC = Cfg::ACC;
   extern __shared__ uint8_t smem_raw[];
@@ -632,10 +638,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&empty_bar[s], NSPLIT);
     }
     for (int a = 0; a < ACC; ++a) {
-      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tfull_bar[a], NSPLIT);
       mbar_init(&tempty_bar[a], 256);
     }
     *abort_flag = 0;
@@ -677,9 +683,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
+  } else if (warp == 1 || warp >= 6) {
+    // ------------------------------------------------------------ MMA issuers (leader), one per chunk
     if (leader && lane == 0) {
+      const int sc = warp == 1 ? 0 : warp - 5;  // output chunk of this thread
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -691,7 +698,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * BN + sc * NCHUNK;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           int to = 0;
@@ -701,17 +708,12 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_pair_kernel(const __grid_const
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
+          // descriptors of k-step k are the k = 0 ones plus 32 bytes (2 in the address field) per step
+          const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + stage * Cfg::B_BYTES) + sc * Cfg::BROWS * 128);
+          const uint32_t first = kb != 0 ? 1u : 0u;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t adesc = sdesc_kmajor_sw128(a_addr + k * 32);
-#pragma unroll
-            for (int s = 0; s < NSPLIT; ++s) {
-              const uint64_t bdesc = sdesc_kmajor_sw128(b_addr + s * Cfg::BROWS * 128 + k * 32);
-              umma2_bf16(d_tmem + s * NCHUNK, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
-            }
-          }
+          for (int k = 0; k < 4; ++k) umma2_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, Cfg::IDESC, k ? 1u : first);
           umma2_commit_mc(&empty_bar[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
