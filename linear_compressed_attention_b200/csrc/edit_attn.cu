@@ -206,6 +206,7 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.tiles_w = (W + pl.TW - 1) / pl.TW;
     pl.gn_chunk = 32;  // tokens per GroupNorm partial (many blocks: the pass is latency-bound otherwise)
     pl.gn_P = static_cast<int>((pl.HW + pl.gn_chunk - 1) / pl.gn_chunk);
+    if (pl.gn_P < 2) pl.gn_P = 2;  // the fused GroupNorm runs at least two blocks
     // [S_h | z_h] has d + 1 columns; the apply GEMM is built for N = 48, 80, 144.
     pl.NP = (pl.d + 1 <= 48) ? 48 : (pl.d + 1 <= 80) ? 80 : 144;
     pl.KP = (pl.d + 63) / 64 * 64;
@@ -649,6 +650,51 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
   return EDIT_OK;
 }
 
+// Cooperative launch of the fused GroupNorm (bf16): as many blocks as are
+// co-resident (at most gn_P, the partial buffer's capacity), 512 threads.
+// The grid barrier counter is word 16 of the status block, which every call
+// zeroes before its first launch.
+int launch_gn_fused(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+  // two blocks per SM at most: more blocks only add partials to combine
+  int nblk = 2 * num_sms();
+  if (nblk > pl.gn_P) nblk = pl.gn_P;
+  if (nblk > GN_FUSED_MAXB) nblk = GN_FUSED_MAXB;
+  const size_t smem = (512 * 4 + static_cast<size_t>(pl.Cr) * 4) * sizeof(float);
+  static bool attr_set = false;  // one device model per process
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gn_fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) !=
+        cudaSuccess)
+      return EDIT_ERR_CUDA;
+    attr_set = true;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gn_fused_bf16_kernel, 512, smem) != cudaSuccess ||
+      per_sm * num_sms() < nblk)
+    return EDIT_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(nblk, 1, 1);
+  cfg.blockDim = dim3(512, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, gn_fused_bf16_kernel, reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), pl.B,
+                         static_cast<long>(pl.HW), pl.Cr, pl.G, w->gn_eps,
+                         static_cast<const __nv_bfloat16*>(w->gn_gamma), static_cast<const __nv_bfloat16*>(w->gn_beta),
+                         w->leaky_slope, reinterpret_cast<float*>(ws + pl.gnpart),
+                         reinterpret_cast<unsigned int*>(ws + pl.status + 64), reinterpret_cast<float*>(ws + pl.gnstats),
+                         reinterpret_cast<float*>(ws + pl.gnss), reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb),
+                         reinterpret_cast<int*>(ws + pl.status)) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  return last_launch();
+}
+
 // Steps 4-7: Q = ReLU([X | G] [Wq | Wq W1]^T + Wq b1 + bq) into the workspace.
 template <typename T>
 int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
@@ -699,6 +745,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
   stage_mark(4, st);
   // 5. U = Conv3x3(X) (+ GroupNorm partials)
   float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
+  bool gn_fused = false;
   if (pl.bf16) {
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -741,14 +788,13 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
       EDIT_TRY(gemm_conv(p, Cr, st));
       stage_mark(5, st);
     }
-    if ((Cr / pl.G) >= 8) {
-      const int nvec = Cr / 8;
-      const int kt = 256 / nvec > 0 ? 256 / nvec : 1;
-      const int threads = kt * nvec;
-      launch_pdl(gn_stats_bf16_kernel, dim3(dim3(pl.gn_P, pl.B)), dim3(threads), threads * 4 * sizeof(float), st, 
-          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_chunk,
-          pl.gn_P, gnpart);
-    } else {
+    if ((Cr / pl.G) >= 8 && Cr / 8 <= 512) {
+      // 6. G = LeakyReLU(GN(U)) in one cooperative grid: statistics, grid barrier, apply
+      const int r = launch_gn_fused(pl, w, ws, st);
+      if (r != EDIT_OK && r != EDIT_ERR_UNSUPPORTED) return r;
+      gn_fused = r == EDIT_OK;
+    }
+    if (!gn_fused) {
       launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, 
           reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
     }
@@ -778,25 +824,27 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     EDIT_TRY(last_launch());
   }
   // 6. G = LeakyReLU(GN(U))
-  launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
-                                              static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
-                                              reinterpret_cast<float*>(ws + pl.gnstats),
-                                              reinterpret_cast<float*>(ws + pl.gnss));
-  EDIT_TRY(last_launch());
-  if (pl.bf16) {
-    const int nvec = Cr / 8;
-    const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
-    const int threads = per_block * nvec;
-    launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(threads), 0, st, 
-        reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-        w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
-  } else {
-    const long total = tok * Cr;
-    launch_pdl(gn_apply_leaky_kernel<float>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
-        reinterpret_cast<const float*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-        w->leaky_slope, reinterpret_cast<float*>(ws + pl.Gb), total);
+  if (!gn_fused) {
+    launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
+                                                static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
+                                                reinterpret_cast<float*>(ws + pl.gnstats),
+                                                reinterpret_cast<float*>(ws + pl.gnss));
+    EDIT_TRY(last_launch());
+    if (pl.bf16) {
+      const int nvec = Cr / 8;
+      const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
+      const int threads = per_block * nvec;
+      launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(threads), 0, st, 
+          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
+          w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
+    } else {
+      const long total = tok * Cr;
+      launch_pdl(gn_apply_leaky_kernel<float>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
+          reinterpret_cast<const float*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
+          w->leaky_slope, reinterpret_cast<float*>(ws + pl.Gb), total);
+    }
+    EDIT_TRY(last_launch());
   }
-  EDIT_TRY(last_launch());
   stage_mark(6, st);
   // 7. Q
   if (pl.bf16) {

@@ -147,28 +147,50 @@ __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int g
   }
 }
 
-// bf16 GroupNorm partial sums with 16-byte loads: thread (kt, v) reads the 8
-// channels 8v..8v+7 of tokens t0 + kt, t0 + kt + KT, ... of its chunk; with at
-// least 8 channels per group those 8 channels touch at most two groups, so
-// each thread keeps two (sum, sum of squares) pairs. The block then sums the
-// per-thread pairs of each group in a fixed order (vector, then kt) in fp64.
-// U [B][HW][Cr]; part[b][chunk][g][2]; blockDim = KT * (Cr / 8) threads.
-__global__ void gn_stats_bf16_kernel(const __nv_bfloat16* __restrict__ U, int HW, int Cr, int groups,
-                                     int chunk_tokens, int chunks, float* __restrict__ part) {
+// GroupNorm + LeakyReLU in one cooperative grid (bf16, channels per group >= 8,
+// Cr % 8 == 0). Each block owns a contiguous token range of every image:
+//  1. per-thread sums of 8-channel vectors (at most two groups per vector),
+//     fixed-order block reduction -> part[b][block][group][2];
+//  2. grid barrier: one arrival per block on a zeroed counter, then a bounded
+//     spin (EDIT_ERR_TIMEOUT after 2 s; the launch is cooperative, so every
+//     block is resident);
+//  3. per image: every block combines all blocks' partials in the same fixed
+//     order (one warp per group, fp64), forms the per-channel affine form
+//     scale = gamma * rstd, shift = beta - mean * scale, and applies
+//     G = LeakyReLU(scale * U + shift) to its tokens (U is re-read from L2).
+// Block 0 also writes stats [b][group] = (mean, rstd) and ss [b][c] = (scale,
+// shift). Dynamic shared memory: blockDim * 4 + Cr * 4 floats. At most
+// GN_FUSED_MAXB blocks (part is [B][groups][2][nblk]).
+constexpr int GN_FUSED_MAXB = 320;
+
+__global__ void __launch_bounds__(512) gn_fused_bf16_kernel(const __nv_bfloat16* __restrict__ U, int B, long HW,
+                                                            int Cr, int groups, float eps,
+                                                            const __nv_bfloat16* __restrict__ gamma,
+                                                            const __nv_bfloat16* __restrict__ beta, float slope,
+                                                            float* __restrict__ part, unsigned int* arrive,
+                                                            float* __restrict__ stats, float* __restrict__ ss,
+                                                            __nv_bfloat16* __restrict__ G, int* status) {
   pdl_wait();
-  extern __shared__ float gs_red[];  // [KT * nvec][4]
-  const int b = blockIdx.y, chunk = blockIdx.x;
-  const int nvec = Cr / 8, KT = blockDim.x / nvec;
-  const int cpg = Cr / groups;
-  const int t = threadIdx.x;
-  if (t < KT * nvec) {
-    const int v = t % nvec, kt = t / nvec;
-    const int c0 = v * 8, g0 = c0 / cpg;
-    const int t0 = chunk * chunk_tokens;
-    const int t1 = min(HW, t0 + chunk_tokens);
+  extern __shared__ float gf_sm[];
+  float* red = gf_sm;                      // [blockDim][4]
+  float* aff = gf_sm + blockDim.x * 4;     // [Cr][2] scale, shift of the current image
+  float* gb = aff + Cr * 2;                // [Cr][2] gamma, beta
+  __shared__ int gf_abort;
+  const int nblk = gridDim.x, blk = blockIdx.x;
+  const int nvec = Cr / 8, kt_n = blockDim.x / nvec;
+  const int t = threadIdx.x, v = t % nvec, kt = t / nvec;
+  const bool active = kt < kt_n;
+  const int cpg = Cr / groups, c0 = v * 8, g0 = c0 / cpg;
+  const long chunk = (HW + nblk - 1) / nblk;
+  const long t0 = blk * chunk, t1 = t0 + chunk < HW ? t0 + chunk : HW;
+  for (int c = t; c < Cr; c += blockDim.x) {  // the affine weights, fetched while the statistics run
+    gb[c * 2] = __bfloat162float(gamma[c]);
+    gb[c * 2 + 1] = __bfloat162float(beta[c]);
+  }
+  // ---- 1. partial sums of this block's tokens, per image
+  for (int b = 0; b < B; ++b) {
     float a0 = 0.f, q0 = 0.f, a1 = 0.f, q1 = 0.f;
-    for (int tok = t0 + kt; tok < t1; tok += KT) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(U + (static_cast<long>(b) * HW + tok) * Cr + c0);
+    auto accum = [&](const uint4& raw) {
       const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -181,26 +203,137 @@ __global__ void gn_stats_bf16_kernel(const __nv_bfloat16* __restrict__ U, int HW
           q1 = fmaf(x, x, q1);
         }
       }
+    };
+    if (active) {
+      const __nv_bfloat16* ub = U + static_cast<long>(b) * HW * Cr + c0;
+      long tok = t0 + kt;
+      for (; tok + 3 * kt_n < t1; tok += 4 * kt_n) {  // four independent loads in flight
+        uint4 r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = *reinterpret_cast<const uint4*>(ub + (tok + j * kt_n) * Cr);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) accum(r[j]);
+      }
+      for (; tok < t1; tok += kt_n) accum(*reinterpret_cast<const uint4*>(ub + tok * Cr));
     }
-    gs_red[t * 4 + 0] = a0;
-    gs_red[t * 4 + 1] = q0;
-    gs_red[t * 4 + 2] = a1;
-    gs_red[t * 4 + 3] = q1;
+    red[t * 4 + 0] = a0;
+    red[t * 4 + 1] = q0;
+    red[t * 4 + 2] = a1;
+    red[t * 4 + 3] = q1;
+    __syncthreads();
+    for (int g = t; g < groups; g += blockDim.x) {
+      double s1 = 0.0, s2 = 0.0;
+      const int vlo = (g * cpg) / 8, vhi = ((g + 1) * cpg - 1) / 8;
+      for (int vv = vlo; vv <= vhi; ++vv) {
+        const int slot = ((vv * 8) / cpg == g) ? 0 : 2;
+        for (int k = 0; k < kt_n; ++k) {
+          s1 += red[(k * nvec + vv) * 4 + slot];
+          s2 += red[(k * nvec + vv) * 4 + slot + 1];
+        }
+      }
+      float* o = part + (static_cast<long>(b) * groups + g) * 2 * nblk + blk;  // [b][g][sum | sumsq][block]
+      o[0] = static_cast<float>(s1);
+      o[nblk] = static_cast<float>(s2);
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
-    double s1 = 0.0, s2 = 0.0;
-    const int vlo = (g * cpg) / 8, vhi = ((g + 1) * cpg - 1) / 8;
-    for (int v = vlo; v <= vhi; ++v) {
-      const int slot = ((v * 8) / cpg == g) ? 0 : 2;
-      for (int kt = 0; kt < KT; ++kt) {
-        s1 += gs_red[(kt * nvec + v) * 4 + slot];
-        s2 += gs_red[(kt * nvec + v) * 4 + slot + 1];
+  // ---- 2. grid barrier
+  if (t == 0) {
+    gf_abort = 0;
+    __threadfence();
+    atomicAdd(arrive, 1u);
+    const uint64_t w0 = globaltimer_ns();
+    while (*reinterpret_cast<volatile unsigned int*>(arrive) < static_cast<unsigned int>(nblk)) {
+      if (globaltimer_ns() - w0 > EDIT_WAIT_TIMEOUT_NS) {
+        record_status(status, EDIT_ERR_TIMEOUT);
+        gf_abort = 1;
+        break;
       }
     }
-    float* o = part + ((static_cast<long>(b) * chunks + chunk) * groups + g) * 2;
-    o[0] = static_cast<float>(s1);
-    o[1] = static_cast<float>(s2);
+    __threadfence();
+  }
+  __syncthreads();
+  if (gf_abort) return;
+  // ---- 3. per image: combine, affine form, apply
+  const int warp = t >> 5, lane = t & 31, nwarps = blockDim.x >> 5;
+  const long cnt = HW * cpg;
+  for (int b = 0; b < B; ++b) {
+    for (int g = warp; g < groups; g += nwarps) {
+      // lane l sums blocks l, l + 32, ... in that order (all loads issued first), then a fixed butterfly
+      const float* ps = part + (static_cast<long>(b) * groups + g) * 2 * nblk;
+      float r1[GN_FUSED_MAXB / 32], r2[GN_FUSED_MAXB / 32];
+#pragma unroll
+      for (int j = 0; j < GN_FUSED_MAXB / 32; ++j) {
+        const int kk = lane + 32 * j;
+        r1[j] = kk < nblk ? ps[kk] : 0.f;
+        r2[j] = kk < nblk ? ps[nblk + kk] : 0.f;
+      }
+      double s1 = 0.0, s2 = 0.0;
+#pragma unroll
+      for (int j = 0; j < GN_FUSED_MAXB / 32; ++j) {
+        s1 += r1[j];
+        s2 += r2[j];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      }
+      const double mean = s1 / static_cast<double>(cnt);
+      double var = s2 / static_cast<double>(cnt) - mean * mean;
+      if (var < 0.0) var = 0.0;
+      const double rstd = 1.0 / sqrt(var + static_cast<double>(eps));
+      for (int c = g * cpg + lane; c < (g + 1) * cpg; c += 32) {
+        const double sc = static_cast<double>(gb[c * 2]) * rstd;
+        const double sh = static_cast<double>(gb[c * 2 + 1]) - mean * sc;
+        aff[c * 2] = static_cast<float>(sc);
+        aff[c * 2 + 1] = static_cast<float>(sh);
+        if (blk == 0) {
+          ss[(static_cast<long>(b) * Cr + c) * 2] = static_cast<float>(sc);
+          ss[(static_cast<long>(b) * Cr + c) * 2 + 1] = static_cast<float>(sh);
+        }
+      }
+      if (blk == 0 && lane == 0) {
+        stats[(b * groups + g) * 2] = static_cast<float>(mean);
+        stats[(b * groups + g) * 2 + 1] = static_cast<float>(rstd);
+      }
+    }
+    __syncthreads();
+    if (active) {
+      float sc[8], sh[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sc[j] = aff[(c0 + j) * 2];
+        sh[j] = aff[(c0 + j) * 2 + 1];
+      }
+      auto apply = [&](const uint4& raw) {
+        const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
+        float o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float y = fmaf(__bfloat162float(u[j]), sc[j], sh[j]);
+          o[j] = y >= 0.f ? y : y * slope;
+        }
+        uint4 out;
+        out.x = pack_bf16x2(o[0], o[1]);
+        out.y = pack_bf16x2(o[2], o[3]);
+        out.z = pack_bf16x2(o[4], o[5]);
+        out.w = pack_bf16x2(o[6], o[7]);
+        return out;
+      };
+      const long base = static_cast<long>(b) * HW * Cr + c0;
+      long tok = t0 + kt;
+      for (; tok + 3 * kt_n < t1; tok += 4 * kt_n) {  // four independent loads in flight
+        uint4 r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = *reinterpret_cast<const uint4*>(U + base + (tok + j * kt_n) * Cr);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(G + base + (tok + j * kt_n) * Cr) = apply(r[j]);
+      }
+      for (; tok < t1; tok += kt_n)
+        *reinterpret_cast<uint4*>(G + base + tok * Cr) = apply(*reinterpret_cast<const uint4*>(U + base + tok * Cr));
+    }
+    __syncthreads();
   }
 }
 
