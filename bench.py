@@ -39,7 +39,7 @@ DOMINANT = "conv3x3"   # largest FLOP share of the layer (40%)
 # the dominant kernel, from the ncu capture summarised in
 # profiles/conv3x3_px4096.md; reported only while the kernel's sources are the
 # ones that capture measured (hash of tc_conv.cuh + tc_gemm.cuh + common.cuh).
-TRAFFIC = {"src_sha": "f3b2f953d4bfebb8", "bytes_per_launch": 159513344 + 25180160}
+TRAFFIC = {"src_sha": "1bc7576c1d516be7", "bytes_per_launch": 160815104 + 25376256}
 
 
 def kernel_src_sha():
