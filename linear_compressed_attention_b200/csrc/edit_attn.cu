@@ -580,7 +580,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
             !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
           return EDIT_ERR_CUDA;
       }
-      launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.Ho, pl.B * (2 * pl.C / 64))), dim3(256), 0, st, 
+      launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, 
           mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
           static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
           static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));

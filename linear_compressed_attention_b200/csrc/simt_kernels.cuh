@@ -597,9 +597,11 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   const int Wo = (W + 1) / 2;
-  const int j0 = blockIdx.x * JT, i = blockIdx.y;
+  // grid (column tiles, image x channel blocks, output rows): rows vary slowest and
+  // run bottom-up, so the rows the K|V GEMM wrote last (still in L2) are read first
+  const int j0 = blockIdx.x * JT, i = gridDim.z - 1 - blockIdx.z;
   const int nblk = 2 * C / CB;
-  const int b = blockIdx.z / nblk, cb = blockIdx.z - b * nblk;
+  const int b = blockIdx.y / nblk, cb = blockIdx.y - b * nblk;
   const int gc0 = cb * CB;
   const bool isk = gc0 < C;
   const int ch0 = isk ? gc0 : gc0 - C;
