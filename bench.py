@@ -6,8 +6,9 @@ A step is one full layer forward (every kernel of the path) over one image
 of the workload. `value` is tokens/s over all ranks (each rank runs its own
 image: weak scaling, no collective on the data path), timed on the device
 with CUDA events on the launching stream, L2 flushed between steps. `e2e`
-is the same metric with the input copied from pinned host memory and the
-output copied back inside the timed region. `--impl reference` times the
+is the same metric with each step's input copied from pinned host memory and
+its output copied back inside the timed region; copies in, layer and copies
+out run on three streams so consecutive steps overlap. `--impl reference` times the
 fp64 CPU oracle on bounded crops of the same workload.
 """
 from __future__ import annotations
@@ -296,22 +297,46 @@ def run_ours(args, cfg):
     tokens = world * B * N * args.steps
     value = tokens / (total_ms / 1e3)
 
-    # e2e: pinned host input -> device -> layer -> pinned host output
+    # e2e: pinned host input -> device -> layer -> pinned host output, every
+    # step. Three streams pipeline consecutive steps: the copy in of step k+1
+    # and the copy out of step k-1 run while the layer computes step k
+    # (double-buffered device input/output and host output; events order each
+    # buffer's reuse).
     xh = torch.from_numpy(d["x"]).to(layer.tdtype).pin_memory()
-    oh = torch.empty(xh.shape, dtype=layer.tdtype).pin_memory()
+    ohs = [torch.empty(xh.shape, dtype=layer.tdtype).pin_memory() for _ in range(2)]
+    xs, outs = [x, torch.empty_like(x)], [out, torch.empty_like(out)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        x.copy_(xh, non_blocking=True)
-        layer.forward(x, out)
-        oh.copy_(out, non_blocking=True)
+
+    def e2e_run(nsteps, e0=None, e1=None):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        if e0 is not None:
+            e0.record(s_in)
+        for k in range(nsteps):
+            j = k % 2
+            if k >= 2:
+                s_in.wait_event(ev_cmp[j])        # the layer of step k-2 has read xs[j]
+            with torch.cuda.stream(s_in):
+                xs[j].copy_(xh, non_blocking=True)
+            ev_in[j].record(s_in)
+            s_cmp.wait_event(ev_in[j])
+            if k >= 2:
+                s_cmp.wait_event(ev_out[j])       # the copy out of step k-2 has read outs[j]
+            layer.forward(xs[j], outs[j], stream=s_cmp)
+            ev_cmp[j].record(s_cmp)
+            s_out.wait_event(ev_cmp[j])
+            with torch.cuda.stream(s_out):
+                ohs[j].copy_(outs[j], non_blocking=True)
+            ev_out[j].record(s_out)
+        if e1 is not None:
+            e1.record(s_out)                      # after the last copy out, which follows everything
+
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(xh, non_blocking=True)
-        layer.forward(x, out)
-        oh.copy_(out, non_blocking=True)
-    e1.record(stream)
+    e2e_run(e2e_steps, e0, e1)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
     t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
