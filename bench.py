@@ -217,6 +217,83 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def side_measurements(dev, peaks, steps=50, warmup=5):
+    """The metric's other sizes (4K and 16K tokens) and the MM-EDiT hybrid at
+    1024 px (4096 image + 333 prompt tokens): median step time with L2 flushed
+    between steps, tokens/s and the fraction of each layer's roofline. The
+    MM line adds its stage times (prompt projections, the two softmax passes)."""
+    import torch
+
+    from linear_compressed_attention_b200 import binding as bd
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, nstages=0):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        evs, stage = [], []
+        for s in range(steps):
+            flush.zero_()
+            if nstages and s == steps - 1:
+                st = [torch.cuda.Event(enable_timing=True) for _ in range(nstages)]
+                for e in st:
+                    e.record(stream)
+                bd.edit_attn_set_stage_events([e.cuda_event for e in st])
+                stage = st
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if nstages and s == steps - 1:
+                bd.edit_attn_set_stage_events(None)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        ms = statistics.median(a.elapsed_time(b) for a, b in (evs[:-1] if nstages else evs))
+        return ms, stage
+
+    res = {}
+    for name in ("px1024", "px2048"):
+        cfg = dict(WORKLOADS[name])
+        d = make_inputs(**cfg)
+        layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"], device=dev)
+        x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
+        out = torch.empty_like(x)
+        ms, _ = timed(lambda: layer.forward(x, out))
+        assert layer.status() == 0
+        n = cfg["B"] * cfg["H"] * cfg["W"]
+        roof = max(layer_flops(cfg)["total"] / (peaks["bf16_tflops"] * 1e12), min_bytes(cfg) / (peaks["hbm_gbs"] * 1e9))
+        res[str(n)] = {"workload": name, "tokens_per_s": n / (ms / 1e3), "ms_per_step": ms,
+                       "layer_roofline_frac": roof * 1e3 / ms}
+        del layer, x, out
+    cfg = dict(WORKLOADS["mm1024"])
+    d = make_inputs(**cfg)
+    nt = cfg["n_txt"]
+    layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"], n_txt=nt, mm=True,
+                             device=dev)
+    xi = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
+    xt = torch.from_numpy(d["x_txt"]).to(dev, layer.tdtype)
+    oi, ot = torch.empty_like(xi), torch.empty_like(xt)
+    ms, st = timed(lambda: layer.forward_mm(xi, xt, oi, ot), bd.STAGE_EVENTS_MM)
+    assert layer.status() == 0
+    ni, C, h = cfg["H"] * cfg["W"], cfg["C"], cfg["heads"]
+    m = ((cfg["H"] + 1) // 2) * ((cfg["W"] + 1) // 2)
+    sdpa_flops = 4.0 * C * (ni * nt + nt * m + nt * nt)       # QK^T and PV of the three softmax blocks
+    mm_flops = layer_flops(cfg)["total"] + 2.0 * nt * C * 3 * C + sdpa_flops
+    roof = max(mm_flops / (peaks["bf16_tflops"] * 1e12), min_bytes(cfg) / (peaks["hbm_gbs"] * 1e9))
+    stage_ms = [st[i].elapsed_time(st[i + 1]) for i in range(len(st) - 1)] if st else []
+    res["mm_edit"] = {"workload": "mm1024: MM-EDiT, 64x64 image grid (4096 tokens, M=1024) + 333 prompt tokens, "
+                                  "C=1536, 24 heads x 64, bf16",
+                      "tokens_per_s": (ni + nt) / (ms / 1e3), "ms_per_step": ms, "layer_roofline_frac": roof * 1e3 / ms,
+                      "sdpa_gflop": sdpa_flops / 1e9,
+                      "stages_ms": {"edit_part": sum(stage_ms[:8]) if len(stage_ms) > 7 else None,
+                                    "prompt_projections": stage_ms[8] if len(stage_ms) > 8 else None,
+                                    "image_row_softmax": stage_ms[9] if len(stage_ms) > 9 else None,
+                                    "prompt_row_softmax": stage_ms[10] if len(stage_ms) > 10 else None}}
+    return res
+
+
 def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
@@ -374,6 +451,8 @@ def run_ours(args, cfg):
                     "d2h_bytes_per_step": nbytes},
             "gpu_launches": launches,
         }
+        if args.workload == "px4096":
+            line["other_sizes"] = side_measurements(dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)

@@ -24,6 +24,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "sdpa_mma.cuh"
 #include "simt_kernels.cuh"
 #include "tc_conv.cuh"
 #include "tc_gemm.cuh"
@@ -946,6 +947,10 @@ int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t*
 
 template <typename T, int D>
 int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
+  if (sizeof(T) == 2) {  // bf16: tensor-core flash-style kernel, 64 query rows per block
+    launch_pdl(sdpa_mma_kernel<D>, dim3(dim3(ceil_div(p.Nq, 64), p.heads, B)), dim3(128), 0, st, p);
+    return last_launch();
+  }
   const size_t smem = (128 * D + 128 * (D + 1)) * sizeof(float);
   auto kern = sdpa_blend_kernel<T, D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -6,6 +6,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "sdpa_mma.cuh"  // SdpaParams
 
 namespace edit {
 namespace {  // internal linkage: each translation unit that uses these keeps its own copy
@@ -881,23 +882,6 @@ __global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restri
 // with each softmax over its own key set (k2 absent when n2 == 0). One thread
 // per (query, head); keys staged through shared memory; online softmax with
 // exp2f. q: [B][Nq][ldq]; k*, v*: [B][n*][ld*] (head h at columns h*d).
-struct SdpaParams {
-  const void* q;
-  long ldq;
-  const void* k1;
-  const void* v1;
-  long ld1;
-  int n1;
-  const void* k2;
-  const void* v2;
-  long ld2;
-  int n2;
-  void* out;
-  long ldo;
-  int Nq, heads, d;
-  float w0, w1, w2;
-  int blend_in;
-};
 
 // Accumulates w * softmax(q K^T) V over one key set into res (registers).
 // q rows live in shared memory (qs, stride D + 1), one row per thread.
