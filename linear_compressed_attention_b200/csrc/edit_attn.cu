@@ -150,6 +150,7 @@ struct Plan {
   int es;  // bytes per element of activations/weights
   int TH, TW, tiles_h, tiles_w;
   int gn_P;       // GroupNorm partials per image
+  int conv_pair_tiles = 0, conv_ksplit = 1;  // per-tap conv: pair tiles, k-parts per tile
   int gn_chunk;   // bf16: tokens per GroupNorm partial
   int kv_chunks;  // KV-state partials per (image, head)
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
@@ -205,6 +206,18 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.TH = 128 / pl.TW;
     pl.tiles_h = (H + pl.TH - 1) / pl.TH;
     pl.tiles_w = (W + pl.TW - 1) / pl.TW;
+    // per-tap conv (W < 128): when its pair tiles would fill at most half of the
+    // CTA pairs, split every tile's 9C / 64 k-blocks over idle pairs
+    pl.conv_pair_tiles = (B * pl.tiles_h * pl.tiles_w + 1) / 2;
+    pl.conv_ksplit = 1;
+    if (pl.TW < 128) {
+      const int pairs = num_sms_hint() / 2, nkb = 9 * C / 64;
+      if (2 * pl.conv_pair_tiles <= pairs) {
+        int k = pairs / pl.conv_pair_tiles;
+        if (k > nkb / 9) k = nkb / 9;  // at least 9 k-blocks (one channel block of every tap) per part
+        pl.conv_ksplit = k > 1 ? k : 1;
+      }
+    }
     pl.gn_chunk = 32;  // tokens per GroupNorm partial (many blocks: the pass is latency-bound otherwise)
     pl.gn_P = static_cast<int>((pl.HW + pl.gn_chunk - 1) / pl.gn_chunk);
     if (pl.gn_P < 2) pl.gn_P = 2;  // the fused GroupNorm runs at least two blocks
@@ -262,6 +275,8 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
   // fp32 halves of the conv tiles split in the last wave (tap-reuse conv only)
   pl.fixpart = (pl.bf16 && pl.TW == 128) ? take(static_cast<size_t>(kConvMaxSplit) * 4 * 128 * pl.Cr * 4) : 0;
+  if (pl.bf16 && pl.TW < 128 && pl.conv_ksplit > 1)  // per-tap conv split over k: one fp32 partial per item
+    pl.fixpart = take(static_cast<size_t>(pl.conv_pair_tiles) * pl.conv_ksplit * 2 * 128 * pl.Cr * 4);
   pl.total = off;
   return EDIT_OK;
 }
@@ -456,7 +471,7 @@ int gemm_linear(const TcGemmParams& p, int bn, cudaStream_t st) {
 
 // 3x3 conv on CTA pairs: 256 tokens x Cr pair tiles.
 int gemm_conv(TcGemmParams& p, int cr, cudaStream_t st) {
-  p.num_tiles = (p.num_m_tiles + 1) / 2;
+  p.num_tiles = (p.num_m_tiles + 1) / 2 * (p.ksplit > 1 ? p.ksplit : 1);
   switch (cr) {
     case 64: return launch_pair<64, 1, 9, EPI_CONV>(p, st);
     case 128: return launch_pair<128, 1, 7, EPI_CONV>(p, st);
@@ -786,8 +801,17 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
         EDIT_TRY(last_launch());
       }
     } else {
+      p.ksplit = pl.conv_ksplit;
+      p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
       EDIT_TRY(gemm_conv(p, Cr, st));
       stage_mark(5, st);
+      if (pl.conv_ksplit > 1) {
+        const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
+        launch_pdl(conv_splitk_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit,
+                   pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
+                   static_cast<const __nv_bfloat16*>(w->cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+        EDIT_TRY(last_launch());
+      }
     }
     if ((Cr / pl.G) >= 8 && Cr / 8 <= 512) {
       // 6. G = LeakyReLU(GN(U)) in one cooperative grid: statistics, grid barrier, apply

@@ -744,6 +744,44 @@ __global__ void conv_fixup_kernel(const float* __restrict__ part, int split_firs
   }
 }
 
+// Split-K per-tap conv: U = bias + sum of the ksplit k-part partials of each
+// pair tile, summed in part order (deterministic), bf16 out. part is
+// [(tile * ksplit + part) * 2 + rank][128][Cr] fp32; row r of CTA tile m_tile
+// is pixel (h0 + r / TW, w0 + r % TW) of a TH x TW tile (TH * TW = 128).
+__global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksplit, int pair_tiles, int tiles_w,
+                                         int tiles_h, int TH, int TW, int H, int W, int Cr,
+                                         const __nv_bfloat16* __restrict__ bias, int num_m_tiles,
+                                         __nv_bfloat16* __restrict__ U) {
+  pdl_wait();
+  const int cv = Cr / 4;
+  const long total = static_cast<long>(pair_tiles) * 2 * 128 * cv;
+  for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(e % cv) * 4;
+    const long rr = e / cv;  // (tile, rank, row)
+    const int row = static_cast<int>(rr & 127), rank = static_cast<int>((rr >> 7) & 1);
+    const int pt = static_cast<int>(rr >> 8);
+    const int m_tile = 2 * pt + rank;
+    if (m_tile >= num_m_tiles) continue;
+    const int per_img = tiles_h * tiles_w;
+    const int img = m_tile / per_img, u = m_tile - img * per_img;
+    const int hh = (u / tiles_w) * TH + row / TW, ww = (u % tiles_w) * TW + row % TW;
+    if (hh >= H || ww >= W) continue;
+    float4 a = make_float4(__bfloat162float(bias[c]), __bfloat162float(bias[c + 1]), __bfloat162float(bias[c + 2]),
+                           __bfloat162float(bias[c + 3]));
+    for (int k = 0; k < ksplit; ++k) {
+      const float4 q = *reinterpret_cast<const float4*>(
+          part + (((static_cast<long>(pt) * ksplit + k) * 2 + rank) * 128 + row) * Cr + c);
+      a.x += q.x;
+      a.y += q.y;
+      a.z += q.z;
+      a.w += q.w;
+    }
+    __nv_bfloat16* dst = U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
 // ================================================================ KV state
 // Partial [S_h | z_h] over a chunk of compressed tokens:
 // part[b][h][chunk][a][c], a < d, c <= d, with column d = sum_j K_ja.

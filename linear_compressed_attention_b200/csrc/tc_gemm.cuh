@@ -66,6 +66,10 @@ struct TcGemmParams {
   // fix_part [split tile][half][rank][128][N] (summed with the bias afterwards)
   int split_first, split_count;
   float* fix_part;
+  // per-tap conv (pair kernel, EPI_CONV): ksplit > 1 splits every tile's
+  // k-blocks into ksplit parts; item it = tile it / ksplit, part it % ksplit,
+  // whose fp32 partial goes to fix_part [item][rank][128][N]
+  int ksplit;
   float* kv_part;       // EPI_KVSTATE: [img][heads][num_chunks][d][d+1]
   // epilogue
   void* out;        // bf16, row (img*R + r) at out + row*ldo (+ column offset)
@@ -142,6 +146,12 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const TcGemmParams& p, int
   TileCoord t;
   t.kb0 = 0;
   t.nkb = p.num_kb;
+  if (EPI == EPI_CONV && p.ksplit > 1) {
+    const int part = pt % p.ksplit;
+    pt /= p.ksplit;
+    t.kb0 = static_cast<int>(static_cast<long>(part) * p.num_kb / p.ksplit);
+    t.nkb = static_cast<int>(static_cast<long>(part + 1) * p.num_kb / p.ksplit) - t.kb0;
+  }
   const int mp = pt / p.num_n_tiles;
   t.n_tile = pt - mp * p.num_n_tiles;
   t.m_tile = 2 * mp + rank;
@@ -668,8 +678,8 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
         for (int kb = 0; kb < tc.nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status)) break;
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
-          load_stage<BN, NSPLIT, EPI, true>(p, tc, kb, sA + stage * Cfg::A_BYTES, sB + stage * Cfg::B_BYTES,
-                                            &full_bar[stage], rank);
+          load_stage<BN, NSPLIT, EPI, true>(p, tc, tc.kb0 + kb, sA + stage * Cfg::A_BYTES,
+                                            sB + stage * Cfg::B_BYTES, &full_bar[stage], rank);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -699,8 +709,9 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN + sc * NCHUNK;
+        const int nkb = decode_pair_tile<EPI>(p, pt, 0).nkb;
         bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           int to = 0;
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status, &to)) {
             if (to) record_wait_site(p.status, 3, pt, kb, stage, phase);
@@ -746,7 +757,21 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
       tc_fence_after();
       const TileCoord tc = decode_pair_tile<EPI>(p, pt, rank);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_tile_staged<BN, EPI>(p, tc, t_row, q, lane, stg, sbuf);
+      if (EPI == EPI_CONV && p.ksplit > 1) {  // fp32 partial of this k-part, row q * 32 + lane
+        float* prow = p.fix_part + ((static_cast<long>(pt) * 2 + rank) * 128 + q * 32 + lane) * p.N;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          float v[64];
+          tmem_ld64(t_row + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + 4 * j < BN)
+              *reinterpret_cast<float4*>(prow + c0 + 4 * j) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      } else {
+        epilogue_tile_staged<BN, EPI>(p, tc, t_row, q, lane, stg, sbuf);
+      }
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader0 + acc * 8);
       ++ntile_done;
