@@ -792,4 +792,277 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
   }
 }
 
+
+// ----------------------------------------------------------------------------
+// Linear projections on CTA pairs with 256 x 384 pair tiles (the Linear layers
+// of section "Spatial Compressor" and the query Linear of eq. Q^EDiT).
+//
+// A 384-column tile halves the weight bytes each CTA ingests per MMA cycle
+// against 256 columns (40 KB per k-block for 768 MMA cycles instead of 32 KB
+// for 512), which is what bounds the 256-column kernel. A tile is three
+// 128-column MMA chunks, each issued by its own thread (warps 1, 6, 7 of the
+// leader). TMEM (512 columns) is a ring of four 128-column slots: chunk
+// g = 3 * (local tile index) + c lives in slot g % 4, so the drain of one
+// tile's chunks overlaps the next tile's main loop.
+//
+// Weight rows: CTA rank r loads the 192 contiguous rows n0 + 192 r ... of the
+// tile as one TMA box; chunk c multiplies rows 64 c .. 64 c + 63 of both CTAs'
+// boxes, so accumulator column j of chunk c is output column n0 + 64 c + j
+// (j < 64) or n0 + 192 + 64 c + (j - 64) (j >= 64).
+template <int STAGES, int STGBUF>
+struct RingCfg {
+  static constexpr int BN = 384, NCH = 3, NCHUNK = 128, BROWS = 192, SLOTS = 4;
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = BROWS * 64 * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+  static constexpr int STG_BYTES = 4 * STGBUF * 4096;    // 4 epilogue warps x STGBUF x (32 rows x 128 B)
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * SLOTS) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert((BROWS / NCH) * 128 % 1024 == 0, "chunk offset keeps the 1024-byte swizzle atom");
+  static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
+};
+constexpr int kRingThreads = 256;
+
+// Bias, optional ReLU, bf16 staging and one TMA store for 32 rows x 64 output
+// columns [n, n + 64) (one weight source: n_split is a multiple of 64). The
+// bias vectors are 16-byte aligned (checked by the host), so each thread
+// reads the 64 values as 16 (fp32) or 8 (bf16) uniform vector loads.
+template <int STGBUF>
+__device__ __forceinline__ void ring_store64(const TcGemmParams& p, const TileCoord& tc, float (&v)[64], int n,
+                                             int q, int lane, uint8_t* stg, int& sbuf) {
+  if (n < p.N) {
+    const int src = n / p.n_split;
+    const void* bias = src < 3 ? p.bias[src] : nullptr;
+    if (bias) {
+      const int j0 = n - src * p.n_split;
+      if (p.bias_f32) {
+        const float4* b4 = reinterpret_cast<const float4*>(static_cast<const float*>(bias) + j0);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 t = __ldg(b4 + i);
+          v[4 * i] += t.x;
+          v[4 * i + 1] += t.y;
+          v[4 * i + 2] += t.z;
+          v[4 * i + 3] += t.w;
+        }
+      } else {
+        const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(bias) + j0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 t = __ldg(b8 + i);
+          const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // bf16 pair -> two fp32 (low half first)
+            v[8 * i + 2 * k] += __uint_as_float(w[k] << 16);
+            v[8 * i + 2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
+          }
+        }
+      }
+    }
+  }
+  if (p.relu) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+  }
+  if (lane == 0) bulk_wait_read<STGBUF - 1>();  // the store that last read this buffer is done
+  __syncwarp();
+  uint8_t* buf = stg + sbuf * 4096;
+  uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 128);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint4 o;
+    o.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+    o.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+    o.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+    o.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+    rowp[j ^ (lane & 7)] = o;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && tc.m_tile < p.num_m_tiles && tc.r0 + q * 32 < p.R && n < p.N) {
+    tma_store_2d(&p.out_map, buf, n, tc.img * p.R + tc.r0 + q * 32);
+    bulk_commit();
+  }
+  if (++sbuf == STGBUF) sbuf = 0;
+}
+
+template <int STAGES, int STGBUF>
+__global__ void __launch_bounds__(kRingThreads, 1) tc_linear_ring_kernel(const __grid_constant__ TcGemmParams p) {
+  using Cfg = RingCfg<STAGES, STGBUF>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* stg_base = sB + STAGES * Cfg::B_BYTES;  // 1024-byte aligned
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + Cfg::SLOTS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + Cfg::SLOTS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], Cfg::NCH);  // one commit per chunk issuer
+    }
+    for (int a = 0; a < Cfg::SLOTS; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.a0);
+    tma_prefetch_desc(&p.b0);
+  }
+  if (warp == 1) tmem_alloc2(tmem_slot, 512);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs of this grid are ready past this point
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t full0 = mapa_shared(smem_u32(&full_bar[0]), 0);  // the leader's barriers
+      const int last_src = (p.N - 1) / p.n_split;
+      for (int pt = pair; pt < p.num_tiles && !*abort_flag; pt += npairs) {
+        const TileCoord tc = decode_pair_tile<EPI_LINEAR>(p, pt, rank);
+        const int nb = tc.n_tile * Cfg::BN + rank * Cfg::BROWS;  // first weight row of this CTA
+        int src = nb / p.n_split;
+        if (src > last_src) src = last_src;  // rows past N: out of the map, zero-filled
+        const CUtensorMap* bmap = src == 0 ? &p.b0 : (src == 1 ? &p.b1 : &p.b2);
+        const int yb = nb - src * p.n_split;
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          int to = 0;
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status, &to)) {
+            if (to) record_wait_site(p.status, 10 + warp, pt, kb, stage, phase ^ 1);
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
+          const uint32_t bar = full0 + stage * 8;
+          if (kb < p.kb_split) {
+            tma2_load_3d(&p.a0, bar, sA + stage * Cfg::A_BYTES, kb * 64, tc.r0, tc.img);
+            tma2_load_2d(bmap, bar, sB + stage * Cfg::B_BYTES, kb * 64, yb);
+          } else {
+            tma2_load_3d(&p.a1, bar, sA + stage * Cfg::A_BYTES, (kb - p.kb_split) * 64, tc.r0, tc.img);
+            tma2_load_2d(&p.bk, bar, sB + stage * Cfg::B_BYTES, (kb - p.kb_split) * 64, nb);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {  // let loads already issued land before the CTA can exit
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp >= 6) {
+    // ------------------------------------------------------------ MMA issuers (leader), one per chunk
+    if (leader && lane == 0) {
+      const int c = warp == 1 ? 0 : warp - 5;
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int pt = pair; pt < p.num_tiles && !*abort_flag; pt += npairs, ++it) {
+        const int g = Cfg::NCH * it + c;
+        const int slot = g & 3;
+        const uint32_t use = static_cast<uint32_t>(g >> 2) & 1u;
+        int to = 0;
+        if (!mbar_wait(&tempty_bar[slot], use ^ 1u, abort_flag, p.status, &to)) {
+          if (to) record_wait_site(p.status, 2, pt, c, slot, use ^ 1u);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + slot * Cfg::NCHUNK;
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          int to = 0;
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status, &to)) {
+            if (to) record_wait_site(p.status, 3, pt, kb, stage, phase);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // descriptors of k-step k are the k = 0 ones plus 32 bytes (2 in the address field) per step
+          const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+          const uint64_t bdesc =
+              sdesc_kmajor_sw128(smem_u32(sB + stage * Cfg::B_BYTES) + c * (Cfg::BROWS / Cfg::NCH) * 128);
+          const uint32_t first = kb != 0 ? 1u : 0u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) umma2_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, Cfg::IDESC, k ? 1u : first);
+          umma2_commit_mc(&empty_bar[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&tfull_bar[slot], 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs), warps 2..5
+    const int q = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    uint8_t* stg = stg_base + q * STGBUF * 4096;
+    int sbuf = 0;
+    int it = 0;
+    bool ok = true;
+    for (int pt = pair; pt < p.num_tiles && ok; pt += npairs, ++it) {
+      const TileCoord tc = decode_pair_tile<EPI_LINEAR>(p, pt, rank);
+      const int n0 = tc.n_tile * Cfg::BN;
+#pragma unroll 1
+      for (int c = 0; c < Cfg::NCH; ++c) {
+        const int g = Cfg::NCH * it + c;
+        const int slot = g & 3;
+        const uint32_t use = static_cast<uint32_t>(g >> 2) & 1u;
+        int to = 0;
+        if (!warp_wait(&tfull_bar[slot], use, abort_flag, p.status, &to)) {
+          if (lane == 0 && to) record_wait_site(p.status, 20 + rank * 10 + q, pt, c, slot, use);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + slot * Cfg::NCHUNK + (static_cast<uint32_t>(q * 32) << 16);
+        float v0[64], v1[64];
+        tmem_ld64(t_row, v0);
+        tmem_ld64(t_row + 64, v1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed_cluster(tempty_leader0 + slot * 8);  // slot free for chunk g + 4
+        ring_store64<STGBUF>(p, tc, v0, n0 + 64 * c, q, lane, stg, sbuf);
+        ring_store64<STGBUF>(p, tc, v1, n0 + Cfg::BROWS + 64 * c, q, lane, stg, sbuf);
+      }
+    }
+    if (lane == 0) bulk_wait_read<0>();  // staged stores have read shared memory before it is released
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, 512);
+  }
+}
+
 }  // namespace edit
