@@ -101,11 +101,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete. Returns false when the
-// block was aborted (by this waiter's timeout or by another role's).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int* timed_out = nullptr) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait, out of line so that every wait site stays a few
+// instructions (single-thread issue loops are sensitive to code size).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                            int* timed_out) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -117,6 +116,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// Wait for the phase with the given parity to complete. Returns false when the
+// block was aborted (by this waiter's timeout or by another role's).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status, int* timed_out = nullptr) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, status, timed_out);
 }
 
 // ----------------------------------------------------------------- TMA

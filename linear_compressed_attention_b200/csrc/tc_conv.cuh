@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(conv_threads(NSPLIT), 1) tc_conv_pair_kernel(c
         }
       }
       tc_fence_before();
-      mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      mbar_arrive_relaxed_cluster(tempty_leader0 + acc * 8);  // TMEM reads done (wait::ld)
       if (++acc == ACC) {
         acc = 0;
         acc_phase ^= 1;

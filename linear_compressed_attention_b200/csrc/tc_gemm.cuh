@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
         epilogue_tile_staged<BN, EPI>(p, tc, t_row, q, lane, stg, sbuf);
       }
       tc_fence_before();
-      mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      mbar_arrive_relaxed_cluster(tempty_leader0 + acc * 8);  // TMEM reads done (wait::ld)
       ++ntile_done;
       if (++acc == ACC) {
         acc = 0;
@@ -816,50 +816,53 @@ struct RingCfg {
   static constexpr int B_BYTES = BROWS * 64 * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
   static constexpr int STG_BYTES = 4 * STGBUF * 4096;    // 4 epilogue warps x STGBUF x (32 rows x 128 B)
+  static constexpr int BIAS_BYTES = 4 * BN * 4;          // per epilogue warp: the tile's bias in fp32
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * SLOTS) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + BIAS_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert((BROWS / NCH) * 128 % 1024 == 0, "chunk offset keeps the 1024-byte swizzle atom");
   static constexpr uint32_t IDESC = idesc_bf16_f32(256, NCHUNK);
 };
 constexpr int kRingThreads = 256;
 
-// Bias, optional ReLU, bf16 staging and one TMA store for 32 rows x 64 output
-// columns [n, n + 64) (one weight source: n_split is a multiple of 64). The
-// bias vectors are 16-byte aligned (checked by the host), so each thread
-// reads the 64 values as 16 (fp32) or 8 (bf16) uniform vector loads.
-template <int STGBUF>
-__device__ __forceinline__ void ring_store64(const TcGemmParams& p, const TileCoord& tc, float (&v)[64], int n,
-                                             int q, int lane, uint8_t* stg, int& sbuf) {
-  if (n < p.N) {
-    const int src = n / p.n_split;
-    const void* bias = src < 3 ? p.bias[src] : nullptr;
-    if (bias) {
-      const int j0 = n - src * p.n_split;
-      if (p.bias_f32) {
-        const float4* b4 = reinterpret_cast<const float4*>(static_cast<const float*>(bias) + j0);
+// Bias of output columns [n0, n0 + 384) in fp32, 12 per lane (columns
+// 4 (32 i + lane) .. + 3, i < 3); zero past N or without a bias. One weight
+// source per 4 columns (n_split is a multiple of 64); the bias vectors are
+// 16-byte aligned (checked by the host).
+__device__ __forceinline__ void ring_bias_fetch(const TcGemmParams& p, int n0, int lane, float4 (&b)[3]) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 t = __ldg(b4 + i);
-          v[4 * i] += t.x;
-          v[4 * i + 1] += t.y;
-          v[4 * i + 2] += t.z;
-          v[4 * i + 3] += t.w;
-        }
-      } else {
-        const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(bias) + j0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 t = __ldg(b8 + i);
-          const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {  // bf16 pair -> two fp32 (low half first)
-            v[8 * i + 2 * k] += __uint_as_float(w[k] << 16);
-            v[8 * i + 2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
-          }
+  for (int i = 0; i < 3; ++i) {
+    const int n = n0 + 4 * (32 * i + lane);
+    b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n < p.N) {
+      const int src = n / p.n_split;
+      const void* bias = src < 3 ? p.bias[src] : nullptr;
+      if (bias) {
+        const int j0 = n - src * p.n_split;
+        if (p.bias_f32) {
+          b[i] = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(bias) + j0));
+        } else {
+          const uint2 t = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(bias) + j0));
+          b[i] = make_float4(__uint_as_float(t.x << 16), __uint_as_float(t.x & 0xffff0000u),
+                             __uint_as_float(t.y << 16), __uint_as_float(t.y & 0xffff0000u));
         }
       }
     }
+  }
+}
+
+// Bias (from the warp's shared copy, 64 values at bsm), optional ReLU, bf16
+// staging and one TMA store for 32 rows x 64 output columns [n, n + 64).
+template <int STGBUF>
+__device__ __forceinline__ void ring_store64(const TcGemmParams& p, const TileCoord& tc, float (&v)[64], int n,
+                                             const float* bsm, int q, int lane, uint8_t* stg, int& sbuf) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float4 t = reinterpret_cast<const float4*>(bsm)[i];
+    v[4 * i] += t.x;
+    v[4 * i + 1] += t.y;
+    v[4 * i + 2] += t.z;
+    v[4 * i + 3] += t.w;
   }
   if (p.relu) {
 #pragma unroll
@@ -895,7 +898,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) tc_linear_ring_kernel(const _
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
   uint8_t* stg_base = sB + STAGES * Cfg::B_BYTES;  // 1024-byte aligned
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
+  float* bias_base = reinterpret_cast<float*>(stg_base + Cfg::STG_BYTES);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES + Cfg::BIAS_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;
   uint64_t* tempty_bar = tfull_bar + Cfg::SLOTS;
@@ -1024,12 +1028,15 @@ __global__ void __launch_bounds__(kRingThreads, 1) tc_linear_ring_kernel(const _
     const int q = warp & 3;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     uint8_t* stg = stg_base + q * STGBUF * 4096;
+    float* bsm = bias_base + q * Cfg::BN;
     int sbuf = 0;
     int it = 0;
     bool ok = true;
     for (int pt = pair; pt < p.num_tiles && ok; pt += npairs, ++it) {
       const TileCoord tc = decode_pair_tile<EPI_LINEAR>(p, pt, rank);
       const int n0 = tc.n_tile * Cfg::BN;
+      float4 bias4[3];  // fetched before the wait for the tile's first chunk, which hides the latency
+      ring_bias_fetch(p, n0, lane, bias4);
 #pragma unroll 1
       for (int c = 0; c < Cfg::NCH; ++c) {
         const int g = Cfg::NCH * it + c;
@@ -1042,6 +1049,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) tc_linear_ring_kernel(const _
           break;
         }
         tc_fence_after();
+        if (c == 0) {  // the previous tile's reads of bsm are complete (program order + the wait's warp sync)
+#pragma unroll
+          for (int i = 0; i < 3; ++i) reinterpret_cast<float4*>(bsm)[32 * i + lane] = bias4[i];
+          __syncwarp();
+        }
         const uint32_t t_row = tmem_base + slot * Cfg::NCHUNK + (static_cast<uint32_t>(q * 32) << 16);
         float v0[64], v1[64];
         tmem_ld64(t_row, v0);
@@ -1049,8 +1061,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) tc_linear_ring_kernel(const _
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_relaxed_cluster(tempty_leader0 + slot * 8);  // slot free for chunk g + 4
-        ring_store64<STGBUF>(p, tc, v0, n0 + 64 * c, q, lane, stg, sbuf);
-        ring_store64<STGBUF>(p, tc, v1, n0 + Cfg::BROWS + 64 * c, q, lane, stg, sbuf);
+        ring_store64<STGBUF>(p, tc, v0, n0 + 64 * c, bsm + 64 * c, q, lane, stg, sbuf);
+        ring_store64<STGBUF>(p, tc, v1, n0 + Cfg::BROWS + 64 * c, bsm + Cfg::BROWS + 64 * c, q, lane, stg, sbuf);
       }
     }
     if (lane == 0) bulk_wait_read<0>();  // staged stores have read shared memory before it is released
