@@ -40,7 +40,7 @@ DOMINANT = "conv3x3"   # largest FLOP share of the layer (40%)
 # the dominant kernel, from the ncu capture summarised in
 # profiles/conv3x3_px4096.md; reported only while the kernel's sources are the
 # ones that capture measured (hash of tc_conv.cuh + tc_gemm.cuh + common.cuh).
-TRAFFIC = {"src_sha": "1bc7576c1d516be7", "bytes_per_launch": 160815104 + 25376256}
+TRAFFIC = {"src_sha": "d3f6defd9a529003", "bytes_per_launch": 160921088 + 25559296}
 
 
 def kernel_src_sha():
@@ -451,7 +451,7 @@ def run_ours(args, cfg):
                     "d2h_bytes_per_step": nbytes},
             "gpu_launches": launches,
         }
-        if args.workload == "px4096":
+        if args.workload == "px4096" and not args.no_side:
             line["other_sizes"] = side_measurements(dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
@@ -469,6 +469,7 @@ def main():
     ap.add_argument("--workload", default="px4096", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true", help="skip the 4K/16K-token and MM-EDiT side measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
