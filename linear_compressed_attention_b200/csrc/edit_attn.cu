@@ -155,11 +155,12 @@ struct Plan {
   int kv_chunks;  // KV-state partials per (image, head)
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
+  int sdpa_split = 0;  // MM-EDiT prompt rows (bf16): ranges of the image keys per query tile, 0 = no split
   int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      fixpart, total;
+      fixpart, sdpapart, total;
 };
 
 int next_pow2(int v) {
@@ -273,6 +274,18 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
   pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
   pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
+  // MM-EDiT prompt rows walk all M image keys per query: when their query tiles
+  // fill less than two waves, split the image keys into ranges of about
+  // max(256, NT) keys (one more item takes the prompt keys) and merge after.
+  pl.sdpapart = 0;
+  if (pl.bf16 && NT > 0) {
+    const long ctas = static_cast<long>(B) * heads * ((NT + 63) / 64);
+    const int span = NT > 256 ? NT : 256;
+    if (ctas < 2L * num_sms_hint() && pl.M > span) {
+      pl.sdpa_split = (pl.M + span - 1) / span;
+      pl.sdpapart = take(static_cast<size_t>(B) * heads * NT * (pl.sdpa_split + 1) * (pl.d + 2) * 4);
+    }
+  }
   // fp32 halves of the conv tiles split in the last wave (tap-reuse conv only)
   pl.fixpart = (pl.bf16 && pl.TW == 128) ? take(static_cast<size_t>(kConvMaxSplit) * 4 * 128 * pl.Cr * 4) : 0;
   if (pl.bf16 && pl.TW < 128 && pl.conv_ksplit > 1)  // per-tap conv split over k: one fp32 partial per item
@@ -1024,7 +1037,12 @@ int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t*
 template <typename T, int D>
 int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
   if (sizeof(T) == 2) {  // bf16: tensor-core flash-style kernel, 64 query rows per block
-    launch_pdl(sdpa_mma_kernel<D>, dim3(dim3(ceil_div(p.Nq, 64), p.heads, B)), dim3(128), 0, st, p);
+    const int nitem = p.part ? p.nchunk1 + (p.n2 > 0 ? 1 : 0) : 1;
+    launch_pdl(sdpa_mma_kernel<D>, dim3(dim3(ceil_div(p.Nq, 64) * nitem, p.heads, B)), dim3(128), 0, st, p);
+    if (!p.part) return last_launch();
+    EDIT_TRY(last_launch());
+    launch_pdl(sdpa_combine_kernel, dim3(grid_for(static_cast<long>(B) * p.heads * p.Nq * 32, 256)), dim3(256), 0, st,
+               p);
     return last_launch();
   }
   const size_t smem = (128 * D + 128 * (D + 1)) * sizeof(float);
@@ -1100,6 +1118,11 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   t.d = pl.d;
   t.w1 = static_cast<float>(eta);
   t.w2 = static_cast<float>(1.0 - eta);
+  if (pl.sdpa_split > 0) {
+    t.nchunk1 = pl.sdpa_split;
+    t.nimg = pl.B;
+    t.part = reinterpret_cast<float*>(ws + pl.sdpapart);
+  }
   EDIT_TRY(sdpa<T>(t, pl.B, st));
   stage_mark(11, st);
   return EDIT_OK;

@@ -39,6 +39,13 @@ struct SdpaParams {
   int Nq, heads, d;
   float w0, w1, w2;
   int blend_in;
+  // Key-split mode (part != nullptr): the first key set is cut into nchunk1
+  // ranges and every block handles one (64-query tile, key range) item; the
+  // second set, if any, is one more item. Each item writes its unnormalised
+  // accumulator, running max (log2 units) and sum per query row to
+  // part [img][head][Nq][items][d + 2]; sdpa_combine_kernel merges them.
+  int nchunk1, nimg;
+  float* part;
 };
 
 namespace {
@@ -73,7 +80,9 @@ __global__ void __launch_bounds__(128) sdpa_mma_kernel(SdpaParams p) {
   __shared__ __align__(16) __nv_bfloat16 ks[KT * RS];
   __shared__ __align__(16) __nv_bfloat16 vt[DP * VS];
   const int h = blockIdx.y, b = blockIdx.z;
-  const int row0 = blockIdx.x * 64;
+  const int nitem = p.part ? p.nchunk1 + (p.n2 > 0 ? 1 : 0) : 1;
+  const int qt = blockIdx.x / nitem, item = blockIdx.x - qt * nitem;
+  const int row0 = qt * 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 
   // ---- this block's 64 query rows (rows >= Nq and columns >= D read as 0)
@@ -102,9 +111,11 @@ __global__ void __launch_bounds__(128) sdpa_mma_kernel(SdpaParams p) {
   float res[NO][4];
 #pragma unroll
   for (int o = 0; o < NO; ++o) res[o][0] = res[o][1] = res[o][2] = res[o][3] = 0.f;
+  float pm[2] = {0.f, 0.f}, pl[2] = {0.f, 0.f};  // key-split mode: the item's running max and sum per row
 
   // one key set: res += w * softmax(q K^T / sqrt(d)) V for rows g and g + 8 of this warp
-  auto one_set = [&](const __nv_bfloat16* kb, const __nv_bfloat16* vb, long ld, int nk, float w) {
+  // (raw: res = the unnormalised accumulator, max and sum kept in pm / pl)
+  auto one_set = [&](const __nv_bfloat16* kb, const __nv_bfloat16* vb, long ld, int nk, float w, bool raw) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float acc[NO][4];
 #pragma unroll
@@ -193,6 +204,17 @@ __global__ void __launch_bounds__(128) sdpa_mma_kernel(SdpaParams p) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (raw) {
+      pm[0] = m0;
+      pm[1] = m1;
+      pl[0] = l0;
+      pl[1] = l1;
+#pragma unroll
+      for (int o = 0; o < NO; ++o)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) res[o][e] = acc[o][e];
+      return;
+    }
     const float s0 = l0 > 0.f ? w / l0 : 0.f, s1 = l1 > 0.f ? w / l1 : 0.f;
 #pragma unroll
     for (int o = 0; o < NO; ++o) {
@@ -203,13 +225,36 @@ __global__ void __launch_bounds__(128) sdpa_mma_kernel(SdpaParams p) {
     }
   };
 
-  one_set(reinterpret_cast<const __nv_bfloat16*>(p.k1) + static_cast<long>(b) * p.n1 * p.ld1 + h * D,
-          reinterpret_cast<const __nv_bfloat16*>(p.v1) + static_cast<long>(b) * p.n1 * p.ld1 + h * D, p.ld1, p.n1,
-          p.w1);
-  if (p.n2 > 0)
-    one_set(reinterpret_cast<const __nv_bfloat16*>(p.k2) + static_cast<long>(b) * p.n2 * p.ld2 + h * D,
-            reinterpret_cast<const __nv_bfloat16*>(p.v2) + static_cast<long>(b) * p.n2 * p.ld2 + h * D, p.ld2, p.n2,
-            p.w2);
+  const __nv_bfloat16* k1 = reinterpret_cast<const __nv_bfloat16*>(p.k1) + static_cast<long>(b) * p.n1 * p.ld1 + h * D;
+  const __nv_bfloat16* v1 = reinterpret_cast<const __nv_bfloat16*>(p.v1) + static_cast<long>(b) * p.n1 * p.ld1 + h * D;
+  const __nv_bfloat16* k2 = reinterpret_cast<const __nv_bfloat16*>(p.k2) + static_cast<long>(b) * p.n2 * p.ld2 + h * D;
+  const __nv_bfloat16* v2 = reinterpret_cast<const __nv_bfloat16*>(p.v2) + static_cast<long>(b) * p.n2 * p.ld2 + h * D;
+  if (p.part) {
+    // one item: a range of the first key set, or the whole second set
+    if (item < p.nchunk1) {
+      const int j0 = static_cast<int>(static_cast<long>(item) * p.n1 / p.nchunk1);
+      const int j1 = static_cast<int>(static_cast<long>(item + 1) * p.n1 / p.nchunk1);
+      one_set(k1 + static_cast<long>(j0) * p.ld1, v1 + static_cast<long>(j0) * p.ld1, p.ld1, j1 - j0, 1.f, true);
+    } else {
+      one_set(k2, v2, p.ld2, p.n2, 1.f, true);
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = row0 + warp * 16 + g + 8 * half;
+      if (r >= p.Nq) continue;
+      float* pp = p.part + ((static_cast<long>(b * p.heads + h) * p.Nq + r) * nitem + item) * (D + 2);
+#pragma unroll
+      for (int o = 0; o < NO; ++o)
+        *reinterpret_cast<float2*>(pp + 8 * o + 2 * t) = make_float2(res[o][2 * half], res[o][2 * half + 1]);
+      if (t == 0) {
+        pp[D] = pm[half];
+        pp[D + 1] = pl[half];
+      }
+    }
+    return;
+  }
+  one_set(k1, v1, p.ld1, p.n1, p.w1, false);
+  if (p.n2 > 0) one_set(k2, v2, p.ld2, p.n2, p.w2, false);
 
   // ---- store (blending in w0 * out): rows g and g + 8, columns 8 o + 2 t, 2 t + 1
   __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long>(b) * p.Nq * p.ldo + h * D;
@@ -228,6 +273,37 @@ __global__ void __launch_bounds__(128) sdpa_mma_kernel(SdpaParams p) {
       }
       *dst = pack_bf16x2(v0, v1);
     }
+  }
+}
+
+// Merge of the key-split items, one warp per (image, head, query row), fixed
+// order: the first set's ranges by the usual max / rescale / sum rule, then
+// out = [w0 out +] w1 softmax_1 V_1 + w2 softmax_2 V_2.
+__global__ void __launch_bounds__(256) sdpa_combine_kernel(SdpaParams p) {
+  pdl_wait();
+  const int D = p.d, nitem = p.nchunk1 + (p.n2 > 0 ? 1 : 0);
+  const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;  // (img * heads + h) * Nq + r
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long>(p.nimg) * p.heads * p.Nq) return;
+  const int r = static_cast<int>(row % p.Nq);
+  const long bh = row / p.Nq;
+  const int h = static_cast<int>(bh % p.heads), b = static_cast<int>(bh / p.heads);
+  const float* pp = p.part + row * nitem * (D + 2);
+  float M = -INFINITY;
+  for (int c = 0; c < p.nchunk1; ++c) M = fmaxf(M, pp[c * (D + 2) + D]);
+  float L = 0.f;
+  for (int c = 0; c < p.nchunk1; ++c) L += pp[c * (D + 2) + D + 1] * exp2f(pp[c * (D + 2) + D] - M);
+  const float s1 = p.w1 / L;
+  const float* p2 = pp + p.nchunk1 * (D + 2);
+  const float s2 = p.n2 > 0 ? p.w2 / p2[D + 1] : 0.f;
+  __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D;
+  for (int col = lane; col < D; col += 32) {
+    float a = 0.f;
+    for (int c = 0; c < p.nchunk1; ++c) a += pp[c * (D + 2) + col] * exp2f(pp[c * (D + 2) + D] - M);
+    float v = a * s1;
+    if (p.n2 > 0) v += p2[col] * s2;
+    if (p.blend_in) v = fmaf(p.w0, __bfloat162float(og[col]), v);
+    og[col] = __float2bfloat16_rn(v);
   }
 }
 

@@ -169,6 +169,8 @@ MM_SMALL = [
     dict(dtype="bf16", B=2, H=6, W=7, C=128, c_red=64, gn_groups=8, heads=2, n_txt=5),     # d = 64
     dict(dtype="bf16", B=1, H=9, W=9, C=1152, c_red=288, gn_groups=32, heads=16, n_txt=70),  # d = 72
     dict(dtype="bf16", B=1, H=4, W=4, C=128, c_red=64, gn_groups=8, heads=4, n_txt=1),     # d = 32, one prompt token
+    dict(dtype="bf16", B=2, H=40, W=30, C=1152, c_red=288, gn_groups=32, heads=16, n_txt=100),  # prompt rows key-split (2 ranges)
+    dict(dtype="bf16", B=1, H=48, W=48, C=128, c_red=64, gn_groups=8, heads=4, n_txt=20),  # d = 32, key-split (3 ranges)
     dict(dtype="f32", B=2, H=5, W=3, C=64, c_red=16, gn_groups=4, heads=2, n_txt=7),       # d = 32
 ]
 
