@@ -11,8 +11,11 @@ all channels scaled by 8); then the weights cf3_w, cf1_w, q_w, k_w, v_w,
 kdw_w, vdw_w, each N(0, 1/fan_in) with fan_in = 9C, Cr, C, C, C, 9, 9; for
 MM-EDiT workloads then x_txt [B, N_T, C] and the prompt weights tq_w, tk_w,
 tv_w (fan_in C). Biases are 0, GroupNorm gamma = 1 and beta = 0, unless
-``nonzero_affine`` asks for random ones (drawn last, so the stream above is
-unchanged). bf16 workloads round every array once to bf16
+``nonzero_affine`` asks for random ones (drawn after the weights, so the
+stream above is unchanged). ``variant_weights`` adds, drawn after all of
+that, the key's own ConvFusion weights kcf3_w, kcf1_w (fan_in 9C, Cr) and the
+output projection o_w (fan_in C), then (with ``nonzero_affine``) their
+biases and GroupNorm affine. bf16 workloads round every array once to bf16
 (round-to-nearest-even) and hand out float32 arrays holding exactly those
 values.
 """
@@ -54,7 +57,7 @@ def _normal(rng, shape, var):
 
 
 def make_inputs(B, H, W, C, c_red, gn_groups, heads, seed, dtype="bf16",
-                outliers=False, n_txt=None, nonzero_affine=False, **_ignored):
+                outliers=False, n_txt=None, nonzero_affine=False, variant_weights=False, **_ignored):
     """Draw one workload. Returns a dict with x (and x_txt) plus every weight
     under the C header's names and the declared constants; arrays are float32
     (bf16-exact for bf16 workloads). Shapes: x [B, H*W, C]; cf3_w [Cr, 3, 3, C];
@@ -98,6 +101,21 @@ def make_inputs(B, H, W, C, c_red, gn_groups, heads, seed, dtype="bf16",
         if n_txt is not None:
             for name in ("tq_b", "tk_b", "tv_b"):
                 d[name] = _normal(rng, (C,), 0.01)
+    if variant_weights:
+        d["kcf3_w"] = _normal(rng, (c_red, 3, 3, C), 1.0 / (9 * C))
+        d["kcf1_w"] = _normal(rng, (C, c_red), 1.0 / c_red)
+        d["o_w"] = _normal(rng, (C, C), 1.0 / C)
+        d["kcf3_b"] = zeros(c_red)
+        d["kgn_gamma"] = np.ones((c_red,), dtype=np.float32)
+        d["kgn_beta"] = zeros(c_red)
+        d["kcf1_b"] = zeros(C)
+        d["o_b"] = zeros(C)
+        if nonzero_affine:
+            d["kcf3_b"] = _normal(rng, (c_red,), 0.01)
+            d["kgn_gamma"] = (1.0 + _normal(rng, (c_red,), 0.01)).astype(np.float32)
+            d["kgn_beta"] = _normal(rng, (c_red,), 0.01)
+            d["kcf1_b"] = _normal(rng, (C,), 0.01)
+            d["o_b"] = _normal(rng, (C,), 0.01)
     if dtype == "bf16":
         d = {k: round_bf16(v) for k, v in d.items()}
     d.update(dict(c_red=c_red, gn_groups=gn_groups, **DECLARED))

@@ -208,6 +208,20 @@ def mix_ratio(N_I, N_T):
 # EDiT layer
 # --------------------------------------------------------------------------
 
+def convfusion_residual(X, cf3_w, cf3_b, groups, gamma, beta, gn_eps, slope, cf1_w, cf1_b):
+    """R = X + Conv1x1(LeakyReLU(GN(Conv3x3(X)))), the argument of the Linear
+    in ConvFusion, eq. (Q^EDiT). X: [B, H, W, C] grid. Returns
+    (R [B, H, W, C], U, gn_mean, gn_var, Lk) with U = Conv3x3(X) and
+    Lk = LeakyReLU(GN(U))."""
+    U = conv3x3_same(X, cf3_w, cf3_b)
+    gn_mean, gn_var = group_norm_stats(U, groups)
+    G = group_norm(U, groups, gamma, beta, gn_eps)
+    Lk = leaky_relu(G, slope)
+    # the 1x1 conv restoring the channels is a per-pixel Linear Cr -> C
+    R = _f64(X) + linear(Lk, cf1_w, cf1_b)
+    return R, U, gn_mean, gn_var, Lk
+
+
 def edit_branches(x, H, W, w, heads):
     """The three branches of one EDiT layer, step by step.
 
@@ -225,12 +239,9 @@ def edit_branches(x, H, W, w, heads):
     B, N, C = np.shape(x)
     X = grid_view(x, H, W)
     # ConvFusion, eq. (Q^EDiT)
-    U = conv3x3_same(X, w["cf3_w"], w["cf3_b"])
-    gn_mean, gn_var = group_norm_stats(U, w["gn_groups"])
-    G = group_norm(U, w["gn_groups"], w["gn_gamma"], w["gn_beta"], w["gn_eps"])
-    Lk = leaky_relu(G, w["leaky_slope"])
-    # the 1x1 conv restoring the channels is a per-pixel Linear Cr -> C
-    R = X + linear(Lk, w["cf1_w"], w["cf1_b"])
+    R, U, gn_mean, gn_var, Lk = convfusion_residual(
+        X, w["cf3_w"], w["cf3_b"], w["gn_groups"], w["gn_gamma"], w["gn_beta"], w["gn_eps"],
+        w["leaky_slope"], w["cf1_w"], w["cf1_b"])
     Q = relu(linear(R, w["q_w"], w["q_b"]))
     # Spatial Compressor, eq. (phi_SC): Linear first, then the depthwise conv;
     # separate K and V weights [R1]
@@ -292,3 +303,71 @@ def mmedit_forward(x_img, x_txt, H, W, w, heads, return_intermediates=False):
                    "eta": eta})
         return out_img, out_txt, br
     return out_img, out_txt
+
+
+# --------------------------------------------------------------------------
+# Ablation variants of the query/key/value processing, optional output
+# projection
+# --------------------------------------------------------------------------
+
+PROC_NONE, PROC_CF, PROC_SC = "none", "cf", "sc"
+# (q, k, v) processing combinations with equal key and value counts: the
+# ablation table "Query/Key/Value processing" (消融实验) lists (CF, SC, SC),
+# (CF, CF, -), (-, SC, SC) and (CF, -, -); the query choice is independent of
+# the key/value choice, so both queries go with every key/value pair.
+KV_PAIRS = ((PROC_SC, PROC_SC), (PROC_CF, PROC_NONE), (PROC_NONE, PROC_NONE))
+
+
+def edit_variant_forward(x, H, W, w, heads, q_proc=PROC_CF, k_proc=PROC_SC, v_proc=PROC_SC, out_proj=False,
+                         return_intermediates=False):
+    """One EDiT layer with the query, key and value processing chosen as in the
+    ablation table of the EDiT notes page (section 消融实验, "Query/Key/Value
+    processing"), followed by an optional output projection.
+
+    Readings [R20] (the table names only the processing, not the formula):
+      query  cf:   Q = ReLU(Linear_Q(X + Conv1x1(LeakyReLU(GN(Conv3x3(X))))))
+             none: Q = ReLU(Linear_Q(X))      (the ReLU feature map stays)
+      key    sc:   K = ReLU(DW_K(Linear_K(X)))                       M tokens
+             cf:   K = ReLU(Linear_K(X + Conv1x1_K(LeakyReLU(GN_K(Conv3x3_K(X))))))
+                   with the key's own ConvFusion weights (kcf3_w, kcf3_b,
+                   kgn_gamma, kgn_beta, kcf1_w, kcf1_b)             N tokens
+             none: K = ReLU(Linear_K(X))                             N tokens
+      value  sc:   V = DW_V(Linear_V(X));  none: V = Linear_V(X)
+    then y = eq. (y_i) over the M (or N) key/value tokens and, with
+    out_proj, out = y o_w^T + o_b (the attention block's output Linear;
+    the page's layer has none [R8], so it is an option here [R21]).
+    (cf, sc, sc) without out_proj is edit_forward.
+    """
+    if q_proc not in (PROC_CF, PROC_NONE) or (k_proc, v_proc) not in KV_PAIRS:
+        raise ValueError(f"unsupported processing ({q_proc}, {k_proc}, {v_proc})")
+    B, N, C = np.shape(x)
+    X = grid_view(x, H, W)
+    it = {}
+    if q_proc == PROC_CF:
+        R = convfusion_residual(X, w["cf3_w"], w["cf3_b"], w["gn_groups"], w["gn_gamma"], w["gn_beta"],
+                                w["gn_eps"], w["leaky_slope"], w["cf1_w"], w["cf1_b"])[0]
+        Q = relu(linear(R, w["q_w"], w["q_b"]))
+    else:
+        Q = relu(linear(X, w["q_w"], w["q_b"]))
+    Kp = linear(X, w["k_w"], w["k_b"])
+    Vp = linear(X, w["v_w"], w["v_b"])
+    if k_proc == PROC_SC:
+        K = relu(dwconv3x3_s2(Kp, w["kdw_w"], w["kdw_b"]))
+        V = dwconv3x3_s2(Vp, w["vdw_w"], w["vdw_b"])
+    else:
+        if k_proc == PROC_CF:
+            RK = convfusion_residual(X, w["kcf3_w"], w["kcf3_b"], w["gn_groups"], w["kgn_gamma"], w["kgn_beta"],
+                                     w["gn_eps"], w["leaky_slope"], w["kcf1_w"], w["kcf1_b"])[0]
+            K = relu(linear(RK, w["k_w"], w["k_b"]))
+        else:
+            K = relu(Kp)
+        V = Vp
+    Q = Q.reshape(B, N, C)
+    K = K.reshape(B, -1, C)
+    V = V.reshape(B, -1, C)
+    y, S, z = linear_attention(Q, K, V, heads, w["attn_eps"])
+    out = linear(y, w["o_w"], w["o_b"]) if out_proj else y
+    if return_intermediates:
+        it.update({"Q": Q, "K": K, "V": V, "S": S, "z": z, "y": y})
+        return out, it
+    return out

@@ -414,3 +414,123 @@ def test_planted_mistake_is_caught(monkeypatch, mutant):
     monkeypatch.setattr(O, name, make(orig))
     oi, op = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, cfg["heads"])
     assert max(rel(oi, ri), rel(op, rp)) > 1e-3, mutant
+
+
+# ------------------------------------------- ablation variants, output Linear
+
+VARIANTS = [(q, k, v) for q in (O.PROC_CF, O.PROC_NONE) for (k, v) in O.KV_PAIRS]
+
+
+def _torch_variant_layer(d, cfg, qp, kp, vp, proj):
+    """The variant layers composed from PyTorch CPU float64 library routines
+    (conv2d, group_norm, leaky_relu, linear, relu, depthwise conv2d), with the
+    explicit quadratic form for the attention step."""
+    B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+    t = {k: torch.tensor(np.asarray(v, np.float64)) for k, v in d.items() if isinstance(v, np.ndarray)}
+    X = t["x"].reshape(B, H, W, C).permute(0, 3, 1, 2)
+
+    def convfusion_feature(pre, lin_w, lin_b):
+        U = F.conv2d(X, t[pre + "cf3_w"].permute(0, 3, 1, 2), t[pre + "cf3_b"], padding=1)
+        G = F.group_norm(U, d["gn_groups"], t[pre + "gn_gamma"], t[pre + "gn_beta"], eps=d["gn_eps"])
+        R = X + F.conv2d(F.leaky_relu(G, d["leaky_slope"]), t[pre + "cf1_w"][:, :, None, None], t[pre + "cf1_b"])
+        return F.relu(F.linear(R.permute(0, 2, 3, 1).reshape(B, H * W, C), lin_w, lin_b))
+
+    Q = convfusion_feature("", t["q_w"], t["q_b"]) if qp == "cf" else F.relu(F.linear(t["x"], t["q_w"], t["q_b"]))
+    if kp == "sc":
+        Kp = F.linear(t["x"], t["k_w"], t["k_b"]).reshape(B, H, W, C).permute(0, 3, 1, 2)
+        Vp = F.linear(t["x"], t["v_w"], t["v_b"]).reshape(B, H, W, C).permute(0, 3, 1, 2)
+        K = F.relu(F.conv2d(Kp, t["kdw_w"][:, None], t["kdw_b"], stride=2, padding=1, groups=C))
+        V = F.conv2d(Vp, t["vdw_w"][:, None], t["vdw_b"], stride=2, padding=1, groups=C)
+        K = K.permute(0, 2, 3, 1).reshape(B, -1, C)
+        V = V.permute(0, 2, 3, 1).reshape(B, -1, C)
+    else:
+        K = convfusion_feature("k", t["k_w"], t["k_b"]) if kp == "cf" else F.relu(F.linear(t["x"], t["k_w"], t["k_b"]))
+        V = F.linear(t["x"], t["v_w"], t["v_b"])
+    dh = C // heads
+    q = Q.reshape(B, -1, heads, dh).transpose(1, 2)
+    k = K.reshape(B, -1, heads, dh).transpose(1, 2)
+    v = V.reshape(B, -1, heads, dh).transpose(1, 2)
+    A = q @ k.transpose(-1, -2)
+    y = ((A @ v) / (A.sum(-1, keepdim=True) + d["attn_eps"])).transpose(1, 2).reshape(B, -1, C)
+    out = F.linear(y, t["o_w"], t["o_b"]) if proj else y
+    return out.numpy(), K.numpy()
+
+
+@pytest.mark.parametrize("proj", [False, True])
+@pytest.mark.parametrize("qkv", VARIANTS, ids=lambda v: "-".join(v))
+def test_variant_vs_torch_composition(qkv, proj):
+    cfg = small_cfg(H=5, W=6, variant_weights=True)
+    d = make_inputs(**cfg)
+    out, it = O.edit_variant_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"], *qkv, out_proj=proj,
+                                     return_intermediates=True)
+    ref, K_t = _torch_variant_layer(d, cfg, *qkv, proj)
+    n_kv = O.compressed_count(5, 6) if qkv[1] == "sc" else 30
+    assert it["K"].shape == (cfg["B"], n_kv, cfg["C"]) and it["V"].shape == it["K"].shape
+    assert rel(it["K"], K_t) < 1e-12
+    assert rel(out, ref) < 1e-11
+
+
+def test_variant_default_is_edit_layer():
+    cfg = small_cfg(variant_weights=True)
+    d = make_inputs(**cfg)
+    y = O.edit_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"])
+    assert np.array_equal(O.edit_variant_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"]), y)
+
+
+def test_variant_uncompressed_vs_brute_force():
+    """(-, -, -) keys/values: K = ReLU(x Wk^T + bk), V = x Wv^T + bv over all N
+    tokens, attention in the explicit O(N^2) loop form."""
+    cfg = small_cfg(B=1, H=3, W=2, C=4, c_red=2, gn_groups=1, heads=2, variant_weights=True)
+    d = make_inputs(**cfg)
+    out = O.edit_variant_forward(d["x"], 3, 2, d, 2, "none", "none", "none")
+    x = np.asarray(d["x"][0], float)
+    kw, kb, vw, vb, qw, qb = (np.asarray(d[n], float) for n in ("k_w", "k_b", "v_w", "v_b", "q_w", "q_b"))
+    lin = lambda w, b: np.array([[b[o] + sum(x[n, i] * w[o, i] for i in range(4)) for o in range(4)]
+                                 for n in range(6)])  # noqa: E731
+    Q, K, V = np.maximum(lin(qw, qb), 0), np.maximum(lin(kw, kb), 0), lin(vw, vb)
+    for h in range(2):
+        sl = slice(2 * h, 2 * h + 2)
+        ref = _brute_linear_attention(Q[:, sl], K[:, sl], V[:, sl], d["attn_eps"])
+        assert rel(out[0, :, sl], ref) < 1e-12
+
+
+def test_variant_special_cases():
+    cfg = small_cfg(variant_weights=True)
+    d = make_inputs(**cfg)
+    H, W, h = cfg["H"], cfg["W"], cfg["heads"]
+    # identity output Linear with zero bias leaves y unchanged
+    e = dict(d, o_w=np.eye(cfg["C"]), o_b=np.zeros(cfg["C"]))
+    assert np.array_equal(O.edit_variant_forward(d["x"], H, W, e, h, out_proj=True),
+                          O.edit_variant_forward(d["x"], H, W, e, h))
+    # a zero 1x1 conv makes the ConvFusion query the plain ReLU(Linear) query
+    e = dict(d, cf1_w=np.zeros_like(d["cf1_w"]), cf1_b=np.zeros_like(d["cf1_b"]))
+    a = O.edit_variant_forward(d["x"], H, W, e, h, "cf", "none", "none")
+    b = O.edit_variant_forward(d["x"], H, W, e, h, "none", "none", "none")
+    assert rel(a, b) < 1e-13
+    # key ConvFusion with the query's weights and Linear gives K == Q
+    e = dict(d, kcf3_w=d["cf3_w"], kcf3_b=d["cf3_b"], kgn_gamma=d["gn_gamma"], kgn_beta=d["gn_beta"],
+             kcf1_w=d["cf1_w"], kcf1_b=d["cf1_b"], k_w=d["q_w"], k_b=d["q_b"])
+    _, it = O.edit_variant_forward(d["x"], H, W, e, h, "cf", "cf", "none", return_intermediates=True)
+    assert np.array_equal(it["K"], it["Q"])
+    with pytest.raises(ValueError):
+        O.edit_variant_forward(d["x"], H, W, d, h, "cf", "sc", "none")
+
+
+VARIANT_MUTANTS = {
+    "convfusion_without_1x1": ("convfusion_residual", ("cf", "cf", "none"),
+                               lambda orig: (lambda X, *a: (np.asarray(X, float),) + orig(X, *a)[1:])),
+    "relu_dropped": ("relu", ("none", "none", "none"), lambda orig: (lambda x: np.asarray(x, float))),
+    "linear_transposed": ("linear", ("none", "none", "none"),
+                          lambda orig: (lambda x, w, b: np.asarray(x, float) @ np.asarray(w, float) + b)),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(VARIANT_MUTANTS))
+def test_variant_planted_mistake_is_caught(monkeypatch, mutant):
+    name, qkv, make = VARIANT_MUTANTS[mutant]
+    cfg = small_cfg(H=4, W=5, variant_weights=True)
+    d = make_inputs(**cfg)
+    ref = _torch_variant_layer(d, cfg, *qkv, True)[0]
+    assert rel(O.edit_variant_forward(d["x"], 4, 5, d, cfg["heads"], *qkv, out_proj=True), ref) < 1e-11
+    monkeypatch.setattr(O, name, make(getattr(O, name)))
+    assert rel(O.edit_variant_forward(d["x"], 4, 5, d, cfg["heads"], *qkv, out_proj=True), ref) > 1e-3, mutant
