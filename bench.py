@@ -69,6 +69,22 @@ def layer_flops(cfg):
     return f
 
 
+def variant_flops(cfg, qkv, proj):
+    """Algorithmic FLOPs of one layer with the query / key / value processing
+    qkv ('cf' | 'sc' | 'none' each) and an optional output Linear."""
+    B, N, C, Cr = cfg["B"], cfg["H"] * cfg["W"], cfg["C"], cfg["c_red"]
+    q, k, _ = qkv
+    m = ((cfg["H"] + 1) // 2) * ((cfg["W"] + 1) // 2) if k == "sc" else N
+    d = C // cfg["heads"]
+    conv_fusion = 2.0 * B * N * Cr * 9 * C + 2.0 * B * N * C * Cr
+    f = 2.0 * B * N * C * C + 4.0 * B * N * C * C                      # Linear_Q, Linear_K, Linear_V
+    f += conv_fusion * ((q == "cf") + (k == "cf"))
+    f += 2.0 * 9 * B * m * 2 * C if k == "sc" else 0.0                  # depthwise stride-2 conv
+    f += 2.0 * B * m * C * (d + 1) + 2.0 * B * N * C * (d + 1)          # KV state, apply
+    f += 2.0 * B * N * C * C if proj else 0.0
+    return f
+
+
 def min_bytes(cfg, es=2):
     B, N, C = cfg["B"], cfg["H"] * cfg["W"], cfg["C"]
     Cr = cfg["c_red"]
@@ -218,10 +234,12 @@ def run_reference(args, cfg):
 
 
 def side_measurements(dev, peaks, steps=50, warmup=5):
-    """The metric's other sizes (4K and 16K tokens) and the MM-EDiT hybrid at
-    1024 px (4096 image + 333 prompt tokens): median step time with L2 flushed
-    between steps, tokens/s and the fraction of each layer's roofline. The
-    MM line adds its stage times (prompt projections, the two softmax passes)."""
+    """The metric's other sizes (4K and 16K tokens, and the 262K-token 8192 px
+    layer), the ablation table's query/key/value processing variants (and the
+    output Linear) at 65K tokens, and the MM-EDiT hybrid at 1024 px (4096 image
+    + 333 prompt tokens): median step time with L2 flushed between steps,
+    tokens/s and the fraction of each layer's roofline. The MM line adds its
+    stage times (prompt projections, the two softmax passes)."""
     import torch
 
     from linear_compressed_attention_b200 import binding as bd
@@ -254,7 +272,7 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
         return ms, stage
 
     res = {}
-    for name in ("px1024", "px2048"):
+    for name in ("px1024", "px2048", "px8192"):
         cfg = dict(WORKLOADS[name])
         d = make_inputs(**cfg)
         layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"], device=dev)
@@ -267,6 +285,28 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
         res[str(n)] = {"workload": name, "tokens_per_s": n / (ms / 1e3), "ms_per_step": ms,
                        "layer_roofline_frac": roof * 1e3 / ms}
         del layer, x, out
+    # the ablation table's query/key/value processing rows and the output Linear,
+    # on the 65,536-token workload
+    cfg = dict(WORKLOADS["px4096"], variant_weights=True)
+    d = make_inputs(**cfg)
+    n = cfg["B"] * cfg["H"] * cfg["W"]
+    var = {}
+    for qkv, proj in ((("cf", "sc", "sc"), True), (("cf", "cf", "none"), False), (("none", "sc", "sc"), False),
+                      (("cf", "none", "none"), False)):
+        layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"], device=dev,
+                                 variant=qkv, out_proj=proj)
+        x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
+        out = torch.empty_like(x)
+        ms, _ = timed(lambda: layer.forward(x, out))
+        assert layer.status() == 0
+        extra = (2 * cfg["C"] * cfg["C"] * 2) if proj else 0
+        roof = max(variant_flops(cfg, qkv, proj) / (peaks["bf16_tflops"] * 1e12),
+                   (min_bytes(cfg) + extra) / (peaks["hbm_gbs"] * 1e9))
+        var["-".join(qkv) + ("+out_linear" if proj else "")] = {
+            "tokens_per_s": n / (ms / 1e3), "ms_per_step": ms, "gflop": variant_flops(cfg, qkv, proj) / 1e9,
+            "layer_roofline_frac": roof * 1e3 / ms}
+        del layer, x, out
+    res["variants_px4096"] = var
     cfg = dict(WORKLOADS["mm1024"])
     d = make_inputs(**cfg)
     nt = cfg["n_txt"]
@@ -469,7 +509,7 @@ def main():
     ap.add_argument("--workload", default="px4096", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-side", action="store_true", help="skip the 4K/16K-token and MM-EDiT side measurements")
+    ap.add_argument("--no-side", action="store_true", help="skip the side measurements (other sizes, variants, MM-EDiT)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

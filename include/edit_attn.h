@@ -112,6 +112,57 @@ EDIT_API size_t edit_attn_workspace_bytes(int B, int H, int W, int C, int heads,
 EDIT_API int edit_attn_forward(const void *x, int B, int H, int W, int C, int heads, const edit_attn_weights *w,
                       void *out, void *stream);
 
+/* Ablation variants of the query / key / value processing and an optional
+ * output Linear. The ablation table of the notes page (section 消融实验,
+ * "Query/Key/Value processing") compares the EDiT layer (CF, SC, SC) with
+ * (CF, CF, -), (-, SC, SC) and (CF, -, -), where CF is ConvFusion, SC the
+ * Spatial Compressor and - no processing beyond the Linear. Readings of the
+ * table used here (it names the processing, not the formulas):
+ *   q_proc  EDIT_PROC_CF:   Q = ReLU(Linear_Q(X + Conv1x1(LeakyReLU(GN(Conv3x3(X))))))
+ *           EDIT_PROC_NONE: Q = ReLU(Linear_Q(X))
+ *   k_proc  EDIT_PROC_SC:   K = ReLU(DW_K(Linear_K(X)))              (M keys)
+ *           EDIT_PROC_CF:   K = ReLU(Linear_K(X + Conv1x1_K(LeakyReLU(GN_K(Conv3x3_K(X))))))
+ *                           with the key's own ConvFusion weights below (N keys)
+ *           EDIT_PROC_NONE: K = ReLU(Linear_K(X))                    (N keys)
+ *   v_proc  EDIT_PROC_SC:   V = DW_V(Linear_V(X)); EDIT_PROC_NONE: V = Linear_V(X)
+ * Keys and values must have equal counts, so (k_proc, v_proc) is one of
+ * (SC, SC), (CF, NONE), (NONE, NONE); any other combination returns
+ * EDIT_ERR_UNSUPPORTED. The attention step is eq. (y_i) over the M or N
+ * key/value tokens. With o_w non-NULL the layer ends with the attention
+ * block's output Linear, out = y o_w^T + o_b (o_w [C][C] torch layout, o_b
+ * [C]); the page's layer has none, so it is optional.
+ * kcf3_w [c_red][3][3][C], kcf3_b, kgn_gamma, kgn_beta [c_red], kcf1_w
+ * [C][c_red], kcf1_b [C] are read only when k_proc is EDIT_PROC_CF; they use
+ * the c_red, gn_groups, gn_eps and leaky_slope of the edit_attn_weights.
+ * Weights a variant does not read may be NULL in both structs (for example
+ * all ConvFusion weights, c_red and gn_groups when neither q_proc nor k_proc
+ * is EDIT_PROC_CF; the depthwise weights without the compressor). */
+enum { EDIT_PROC_NONE = 0, EDIT_PROC_CF = 1, EDIT_PROC_SC = 2 };
+
+typedef struct {
+  int q_proc;
+  int k_proc;
+  int v_proc;
+  const void *kcf3_w, *kcf3_b;
+  const void *kgn_gamma, *kgn_beta;
+  const void *kcf1_w, *kcf1_b;
+  const void *o_w, *o_b;
+} edit_attn_variant;
+
+/* Workspace bytes of edit_attn_variant_forward (0 on a shape, dtype or
+ * processing error, or a NULL variant). Host-only. */
+EDIT_API size_t edit_attn_variant_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
+                                                  const edit_attn_variant *v);
+
+/* One layer with the processing chosen in `v` (conventions as
+ * edit_attn_forward; the workspace is w->workspace and must hold
+ * edit_attn_variant_workspace_bytes). {CF, SC, SC} with o_w == NULL computes
+ * exactly what edit_attn_forward computes. Stage events (the hook below) are
+ * the EDiT layer's 0-8, plus 9 after the output Linear when there is one. */
+EDIT_API int edit_attn_variant_forward(const void *x, int B, int H, int W, int C, int heads,
+                                       const edit_attn_weights *w, const edit_attn_variant *v, void *out,
+                                       void *stream);
+
 /* Weights of the MM-EDiT hybrid: the EDiT image-stream weights (`img`, its
  * dtype field is the dtype of everything) plus the prompt-token projections
  * tq_w, tk_w, tv_w [C][C] (torch Linear layout) and their biases [C]. The
@@ -167,6 +218,12 @@ typedef struct {
 
 EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
                                edit_ws_layout *layout);
+
+/* The same for an edit_attn_variant_forward workspace (v NULL: the EDiT
+ * layer). Without the compressor, KT and VTx hold all N tokens in one padded
+ * row (Mp = Wop = N rounded up to a multiple of 8). */
+EDIT_API int edit_attn_variant_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
+                                                const edit_attn_variant *v, edit_ws_layout *layout);
 
 /* Measurement hooks (no counterpart on the page; used by the benchmark).
  *

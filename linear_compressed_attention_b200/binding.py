@@ -21,8 +21,11 @@ WEIGHT_NAMES = ("cf3_w", "cf3_b", "gn_gamma", "gn_beta", "cf1_w", "cf1_b", "q_w"
 TEXT_NAMES = ("tq_w", "tq_b", "tk_w", "tk_b", "tv_w", "tv_b")
 EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_bytes", "mmedit_hybrid_forward",
            "edit_attn_read_status", "edit_status_string", "edit_attn_workspace_layout",
-           "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc")
+           "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc",
+           "edit_attn_variant_workspace_bytes", "edit_attn_variant_forward", "edit_attn_variant_workspace_layout")
 STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
+PROC = {"none": 0, "cf": 1, "sc": 2}
+VARIANT_NAMES = ("kcf3_w", "kcf3_b", "kgn_gamma", "kgn_beta", "kcf1_w", "kcf1_b", "o_w", "o_b")
 
 
 class EditAttnWeights(ctypes.Structure):
@@ -35,6 +38,11 @@ class EditAttnWeights(ctypes.Structure):
 class MMEditWeights(ctypes.Structure):
     _fields_ = [("img", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in TEXT_NAMES] + \
                [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class EditAttnVariant(ctypes.Structure):
+    _fields_ = [("q_proc", ctypes.c_int), ("k_proc", ctypes.c_int), ("v_proc", ctypes.c_int)] + \
+               [(n, ctypes.c_void_p) for n in VARIANT_NAMES]
 
 
 class WsLayout(ctypes.Structure):
@@ -76,6 +84,13 @@ def lib():
     L.edit_attn_kernel_launches.restype = ctypes.c_uint64
     L.edit_linear_attention_noalloc.argtypes = [p, p, p, i, i, i, i, i, i, ctypes.c_float, p, p]
     L.edit_linear_attention_noalloc.restype = i
+    V = ctypes.POINTER(EditAttnVariant)
+    L.edit_attn_variant_workspace_bytes.argtypes = [i, i, i, i, i, W, V]
+    L.edit_attn_variant_workspace_bytes.restype = sz
+    L.edit_attn_variant_forward.argtypes = [p, i, i, i, i, i, W, V, p, p]
+    L.edit_attn_variant_forward.restype = i
+    L.edit_attn_variant_workspace_layout.argtypes = [i, i, i, i, i, W, V, ctypes.POINTER(WsLayout)]
+    L.edit_attn_variant_workspace_layout.restype = i
     _lib = L
     return L
 
@@ -184,6 +199,37 @@ def edit_attn_kernel_launches() -> int:
     return int(lib().edit_attn_kernel_launches())
 
 
+def make_variant_struct(q_proc="cf", k_proc="sc", v_proc="sc", w: dict | None = None) -> EditAttnVariant:
+    """Processing names 'cf' / 'sc' / 'none'; `w` holds the key ConvFusion
+    weights and/or the output Linear (o_w, o_b) as device tensors, or None."""
+    v = EditAttnVariant()
+    v.q_proc, v.k_proc, v.v_proc = PROC[q_proc], PROC[k_proc], PROC[v_proc]
+    for n in VARIANT_NAMES:
+        t = (w or {}).get(n)
+        setattr(v, n, None if t is None else t.data_ptr())
+    return v
+
+
+def edit_attn_variant_workspace_bytes(B, H, W, C, heads, weights: EditAttnWeights, variant: EditAttnVariant) -> int:
+    return int(lib().edit_attn_variant_workspace_bytes(B, H, W, C, heads, ctypes.byref(weights),
+                                                       ctypes.byref(variant)))
+
+
+def edit_attn_variant_forward(x, B, H, W, C, heads, weights: EditAttnWeights, variant: EditAttnVariant, out,
+                              stream=None) -> int:
+    return int(lib().edit_attn_variant_forward(_ptr(x), B, H, W, C, heads, ctypes.byref(weights),
+                                               ctypes.byref(variant), _ptr(out), _stream(stream)))
+
+
+def edit_attn_variant_workspace_layout(B, H, W, C, heads, weights: EditAttnWeights, variant) -> dict:
+    lay = WsLayout()
+    vp = None if variant is None else ctypes.byref(variant)
+    rc = lib().edit_attn_variant_workspace_layout(B, H, W, C, heads, ctypes.byref(weights), vp, ctypes.byref(lay))
+    if rc != 0:
+        raise EditError(rc)
+    return {n: int(getattr(lay, n)) for n, _ in WsLayout._fields_}
+
+
 def edit_linear_attention_noalloc(q, k, v, B, N, M, C, heads, dtype_code, attn_eps, out, stream=None) -> int:
     """Linear attention step with the library's static scratch (no workspace);
     q, out [B, N, C], k, v [B, M, C] device tensors. Returns the status code."""
@@ -200,35 +246,57 @@ class EditAttention:
     """
 
     def __init__(self, arrays: dict, B: int, H: int, W: int, C: int, heads: int, dtype: str = "bf16",
-                 n_txt: int = 0, mm: bool | None = None, device="cuda"):
+                 n_txt: int = 0, mm: bool | None = None, device="cuda", variant: tuple | None = None,
+                 out_proj: bool = False):
+        """``variant`` = (q_proc, k_proc, v_proc) names ('cf', 'sc', 'none') and/or
+        ``out_proj`` select edit_attn_variant_forward; weights a variant does
+        not read are not copied to the device (NULL in the structs)."""
         import torch
         self.torch = torch
         self.B, self.H, self.W, self.C, self.heads, self.n_txt = B, H, W, C, heads, int(n_txt or 0)
         self.mm = bool(self.n_txt) if mm is None else bool(mm)
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         self.code = EDIT_BF16 if dtype == "bf16" else EDIT_F32
+        self.is_variant = variant is not None or out_proj
+        q, k, v = variant or ("cf", "sc", "sc")
         names = WEIGHT_NAMES + (TEXT_NAMES if self.mm else ())
+        if self.is_variant:
+            skip = set()
+            if q != "cf":
+                skip |= {"cf3_w", "cf3_b", "gn_gamma", "gn_beta", "cf1_w", "cf1_b"}
+            if k != "sc":
+                skip |= {"kdw_w", "kdw_b", "vdw_w", "vdw_b"}
+            names = tuple(n for n in names if n not in skip)
+            names += (("kcf3_w", "kcf3_b", "kgn_gamma", "kgn_beta", "kcf1_w", "kcf1_b") if k == "cf" else ())
+            names += (("o_w", "o_b") if out_proj else ())
         self.w = {n: torch.from_numpy(np.ascontiguousarray(arrays[n])).to(device=device, dtype=self.tdtype)
                   for n in names}
         self.consts = dict(c_red=arrays["c_red"], gn_groups=arrays["gn_groups"], gn_eps=arrays["gn_eps"],
                            leaky_slope=arrays["leaky_slope"], attn_eps=arrays["attn_eps"])
         s = make_weights_struct(self.w, self.code, **self.consts)
+        self.variant = make_variant_struct(q, k, v, self.w) if self.is_variant else None
         if self.mm:
             m = make_mm_struct(s, self.w)
             nbytes = mmedit_workspace_bytes(B, H, W, self.n_txt, C, heads, m)
+        elif self.is_variant:
+            nbytes = edit_attn_variant_workspace_bytes(B, H, W, C, heads, s, self.variant)
         else:
             nbytes = edit_attn_workspace_bytes(B, H, W, C, heads, s)
         if nbytes == 0:
-            raise ValueError("shape/dtype rejected by edit_attn_workspace_bytes")
+            raise ValueError("shape/dtype rejected by the workspace query")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.struct = make_weights_struct(self.w, self.code, workspace=self.workspace, **self.consts)
         self.mm_struct = make_mm_struct(self.struct, self.w, self.workspace) if self.mm else None
-        self.layout = edit_attn_workspace_layout(B, H, W, C, heads, self.struct)
+        self.layout = edit_attn_variant_workspace_layout(B, H, W, C, heads, self.struct, self.variant)
 
     def forward(self, x, out=None, stream=None):
         if out is None:
             out = self.torch.empty_like(x)
-        rc = edit_attn_forward(x, self.B, self.H, self.W, self.C, self.heads, self.struct, out, stream)
+        if self.is_variant:
+            rc = edit_attn_variant_forward(x, self.B, self.H, self.W, self.C, self.heads, self.struct, self.variant,
+                                           out, stream)
+        else:
+            rc = edit_attn_forward(x, self.B, self.H, self.W, self.C, self.heads, self.struct, out, stream)
         if rc != 0:
             raise EditError(rc)
         return out

@@ -51,6 +51,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+#define EDIT_TRY_CHECK(expr)          \
+  do {                                \
+    const int rc_ = (expr);           \
+    if (rc_ != EDIT_OK) return rc_;   \
+  } while (0)
+
 enum Swz { SWZ_NONE = 0, SWZ_64 = 64, SWZ_128 = 128 };
 
 bool encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
@@ -158,9 +164,14 @@ struct Plan {
   int sdpa_split = 0;  // MM-EDiT prompt rows (bf16): ranges of the image keys per query tile, 0 = no split
   int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
+  // query / key / value processing (edit_attn_variant; the EDiT layer is CF, SC, SC)
+  int q_proc = EDIT_PROC_CF, k_proc = EDIT_PROC_SC, v_proc = EDIT_PROC_SC;
+  bool compress = true;  // keys/values through the Spatial Compressor (M = ceil(H/2) ceil(W/2)), else M = N
+  bool any_cf = true;    // some ConvFusion runs (c_red, gn_groups and their weights are used)
+  bool oproj = false;    // output Linear after the attention
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      fixpart, sdpapart, total;
+      fixpart, sdpapart, Y, total;
 };
 
 int next_pow2(int v) {
@@ -173,24 +184,39 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Host-only shape/dtype checks and the workspace layout. Returns EDIT_OK or
 // an error code; fills `pl` on success.
-int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_weights* w, Plan& pl) {
+int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_weights* w, Plan& pl,
+              const edit_attn_variant* var = nullptr) {
   if (!w) return EDIT_ERR_NULL;
   if (w->dtype != EDIT_F32 && w->dtype != EDIT_BF16) return EDIT_ERR_DTYPE;
+  pl = Plan();
+  if (var) {
+    pl.q_proc = var->q_proc;
+    pl.k_proc = var->k_proc;
+    pl.v_proc = var->v_proc;
+    const bool q_ok = pl.q_proc == EDIT_PROC_CF || pl.q_proc == EDIT_PROC_NONE;
+    const bool kv_ok = (pl.k_proc == EDIT_PROC_SC && pl.v_proc == EDIT_PROC_SC) ||
+                       (pl.k_proc == EDIT_PROC_CF && pl.v_proc == EDIT_PROC_NONE) ||
+                       (pl.k_proc == EDIT_PROC_NONE && pl.v_proc == EDIT_PROC_NONE);
+    if (!q_ok || !kv_ok) return EDIT_ERR_UNSUPPORTED;
+    pl.compress = pl.k_proc == EDIT_PROC_SC;
+    pl.any_cf = pl.q_proc == EDIT_PROC_CF || pl.k_proc == EDIT_PROC_CF;
+    pl.oproj = var->o_w != nullptr;
+  }
   if (B < 1 || H < 1 || W < 1 || C < 1 || heads < 1 || NT < 0) return EDIT_ERR_SHAPE;
-  if (C % heads != 0 || w->c_red < 1 || w->gn_groups < 1 || w->c_red % w->gn_groups != 0) return EDIT_ERR_SHAPE;
+  if (C % heads != 0) return EDIT_ERR_SHAPE;
+  if (pl.any_cf && (w->c_red < 1 || w->gn_groups < 1 || w->c_red % w->gn_groups != 0)) return EDIT_ERR_SHAPE;
   if (static_cast<long>(H) * W > (1L << 28) || static_cast<long>(B) * H * W > (1L << 30) || C > 65536)
     return EDIT_ERR_SHAPE;
-  pl = Plan();
   pl.B = B;
   pl.H = H;
   pl.W = W;
   pl.C = C;
   pl.heads = heads;
-  pl.Cr = w->c_red;
-  pl.G = w->gn_groups;
+  pl.Cr = pl.any_cf ? w->c_red : 0;
+  pl.G = pl.any_cf ? w->gn_groups : 1;
   pl.d = C / heads;
-  pl.Ho = (H + 1) / 2;
-  pl.Wo = (W + 1) / 2;
+  pl.Ho = pl.compress ? (H + 1) / 2 : H;
+  pl.Wo = pl.compress ? (W + 1) / 2 : W;
   pl.M = pl.Ho * pl.Wo;
   pl.HW = static_cast<long>(H) * W;
   pl.NT = NT;
@@ -200,7 +226,9 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     // Tensor-core path constraints: 64-wide k-blocks over C, Linear tiles that
     // divide C, conv tile N = Cr (instantiated sizes), 16-byte head offsets.
     if (C % 128 != 0) return EDIT_ERR_UNSUPPORTED;
-    if (!(pl.Cr == 64 || pl.Cr == 128 || pl.Cr == 256 || pl.Cr == 288 || pl.Cr == 384)) return EDIT_ERR_UNSUPPORTED;
+    if (pl.any_cf && !(pl.Cr == 64 || pl.Cr == 128 || pl.Cr == 256 || pl.Cr == 288 || pl.Cr == 384))
+      return EDIT_ERR_UNSUPPORTED;
+    if (!pl.compress && static_cast<long>(B) * (2 * C / 64) > 65535) return EDIT_ERR_UNSUPPORTED;
     if (pl.d % 8 != 0 || pl.d + 1 > 144) return EDIT_ERR_UNSUPPORTED;
     pl.bn_lin = (C % 256 == 0) ? 256 : (C % 192 == 0) ? 192 : 128;
     pl.TW = next_pow2(W) < 128 ? next_pow2(W) : 128;
@@ -222,18 +250,20 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.gn_chunk = 32;  // tokens per GroupNorm partial (many blocks: the pass is latency-bound otherwise)
     pl.gn_P = static_cast<int>((pl.HW + pl.gn_chunk - 1) / pl.gn_chunk);
     if (pl.gn_P < 2) pl.gn_P = 2;  // the fused GroupNorm runs at least two blocks
+    if (!pl.any_cf) pl.gn_P = 0;
     // [S_h | z_h] has d + 1 columns; the apply GEMM is built for N = 48, 80, 144.
     pl.NP = (pl.d + 1 <= 48) ? 48 : (pl.d + 1 <= 80) ? 80 : 144;
     pl.KP = (pl.d + 63) / 64 * 64;
   } else {
-    pl.gn_P = static_cast<int>(pl.HW < 64 ? pl.HW : 64);
+    pl.gn_P = pl.any_cf ? static_cast<int>(pl.HW < 64 ? pl.HW : 64) : 0;
   }
   if (NT > 0 && !(pl.d == 32 || pl.d == 64 || pl.d == 72)) return EDIT_ERR_UNSUPPORTED;
   if (pl.bf16) {
     // Tensor-core KV state: tokens on a grid padded to 32 columns, split into
     // chunks of kv_kb 64-token blocks so that B * heads * chunks fills the GPU.
-    pl.Wop = (pl.Wo + 31) / 32 * 32;
-    pl.Mp = pl.Ho * pl.Wop;
+    // (without the compressor: the N tokens in one row padded to a multiple of 8)
+    pl.Wop = pl.compress ? (pl.Wo + 31) / 32 * 32 : static_cast<int>((pl.HW + 7) / 8 * 8);
+    pl.Mp = pl.compress ? pl.Ho * pl.Wop : pl.Wop;
     const int total_kb = (pl.Mp + 63) / 64;
     const int want = (2 * num_sms_hint() + B * heads - 1) / (B * heads);  // chunks per (image, head)
     pl.kv_kb = (total_kb + want - 1) / (want > 0 ? want : 1);
@@ -259,7 +289,7 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.gnpart = take(static_cast<size_t>(B) * pl.gn_P * pl.G * 2 * 4);
   pl.gnstats = take(static_cast<size_t>(B) * pl.G * 2 * 4);
   pl.gnss = take(static_cast<size_t>(B) * pl.Cr * 2 * 4);
-  pl.W1t = take(static_cast<size_t>(pl.Cr) * C * es);
+  pl.W1t = take(static_cast<size_t>(pl.Cr) * C * es);  // (Cr = 0 when no ConvFusion runs)
   pl.Wqw1 = take(static_cast<size_t>(C) * pl.Cr * es);
   pl.bfold = take(static_cast<size_t>(C) * 4);
   pl.Q = take(tok * C * es);
@@ -290,16 +320,39 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.fixpart = (pl.bf16 && pl.TW == 128) ? take(static_cast<size_t>(kConvMaxSplit) * 4 * 128 * pl.Cr * 4) : 0;
   if (pl.bf16 && pl.TW < 128 && pl.conv_ksplit > 1)  // per-tap conv split over k: one fp32 partial per item
     pl.fixpart = take(static_cast<size_t>(pl.conv_pair_tiles) * pl.conv_ksplit * 2 * 128 * pl.Cr * 4);
+  pl.Y = pl.oproj ? take(tok * C * es) : 0;  // attention output before the output Linear
   pl.total = off;
   return EDIT_OK;
 }
 
-int check_weights(const edit_attn_weights* w) {
-  const void* ptrs[] = {w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b, w->q_w, w->q_b,
-                        w->k_w,   w->k_b,   w->v_w,      w->v_b,     w->kdw_w, w->kdw_b, w->vdw_w, w->vdw_b};
-  for (const void* p : ptrs) {
-    if (!p) return EDIT_ERR_NULL;
-    if (!aligned(p, 16)) return EDIT_ERR_ALIGN;
+int check_ptrs(const void* const* ptrs, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) return EDIT_ERR_NULL;
+    if (!aligned(ptrs[i], 16)) return EDIT_ERR_ALIGN;
+  }
+  return EDIT_OK;
+}
+
+// The weights the plan's processing reads must be present and 16-byte aligned;
+// the others are not touched and may be NULL.
+int check_weights(const edit_attn_weights* w, const Plan& pl, const edit_attn_variant* var = nullptr) {
+  const void* lin[] = {w->q_w, w->q_b, w->k_w, w->k_b, w->v_w, w->v_b};
+  EDIT_TRY_CHECK(check_ptrs(lin, 6));
+  if (pl.q_proc == EDIT_PROC_CF) {
+    const void* cf[] = {w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b};
+    EDIT_TRY_CHECK(check_ptrs(cf, 6));
+  }
+  if (pl.compress) {
+    const void* sc[] = {w->kdw_w, w->kdw_b, w->vdw_w, w->vdw_b};
+    EDIT_TRY_CHECK(check_ptrs(sc, 4));
+  }
+  if (var && pl.k_proc == EDIT_PROC_CF) {
+    const void* kcf[] = {var->kcf3_w, var->kcf3_b, var->kgn_gamma, var->kgn_beta, var->kcf1_w, var->kcf1_b};
+    EDIT_TRY_CHECK(check_ptrs(kcf, 6));
+  }
+  if (var && pl.oproj) {
+    const void* o[] = {var->o_w, var->o_b};
+    EDIT_TRY_CHECK(check_ptrs(o, 2));
   }
   return EDIT_OK;
 }
@@ -565,14 +618,14 @@ int gemm_kvstate(const TcGemmParams& p, int np, cudaStream_t st) {
 
 int ceil_div(long a, long b) { return static_cast<int>((a + b - 1) / b); }
 
-// Plain Linear on the tensor cores: out[rows][nsrc*C] = A[rows][K] [W0; W1; W2]^T + bias.
+// Plain Linear on the tensor cores: out[rows][nsrc*C] = A[rows][K] [W0; W1; W2]^T + bias
+// (optionally ReLU'd), output rows ldo elements apart.
 int tc_linear(const void* a, long rows, int K, const void* const* wts, const void* const* biases, int nsrc, int C,
-              int bn, void* out, int* status, cudaStream_t st) {
+              void* out, long ldo, int relu, int* status, cudaStream_t st) {
   TcGemmParams p;
   std::memset(&p, 0, sizeof(p));
   if (!map_a(&p.a0, a, K, rows, 1, K, rows * K)) return EDIT_ERR_CUDA;
   p.a1 = p.a0;
-  (void)bn;
   const int lbn = linear_bn(rows, nsrc * C, C, biases, nsrc);
   CUtensorMap* bm[3] = {&p.b0, &p.b1, &p.b2};
   for (int s = 0; s < 3; ++s)
@@ -586,15 +639,16 @@ int tc_linear(const void* a, long rows, int K, const void* const* wts, const voi
   p.n_split = C;
   p.N = nsrc * C;
   p.out = out;
-  p.ldo = static_cast<long>(nsrc) * C;
+  p.ldo = ldo;
   if (!map_out2d(&p.out_map, out, p.N, rows, p.ldo)) return EDIT_ERR_CUDA;
   for (int s = 0; s < nsrc; ++s) p.bias[s] = biases[s];
+  p.relu = relu;
   p.status = status;
   return gemm_linear_pair(p, lbn, st);
 }
 
 int simt_linear(const void* a, long rows, int K, const void* const* wts, const void* const* biases, int nsrc,
-                int C, void* out, cudaStream_t st) {
+                int C, void* out, int ldo, int relu, cudaStream_t st) {
   SimtGemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.a0 = static_cast<const float*>(a);
@@ -607,7 +661,8 @@ int simt_linear(const void* a, long rows, int K, const void* const* wts, const v
   p.M = static_cast<int>(rows);
   p.N = nsrc * C;
   p.out = static_cast<float*>(out);
-  p.ldo = nsrc * C;
+  p.ldo = ldo;
+  p.relu = relu;
   launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(p.N, 64), ceil_div(p.M, 64))), dim3(256), 0, st, p);
   return last_launch();
 }
@@ -618,22 +673,58 @@ int simt_linear(const void* a, long rows, int K, const void* const* wts, const v
     if (rc_ != EDIT_OK) return rc_; \
   } while (0)
 
-// Steps 1-3: K, V and the per-head [S | z] (fp32) into the workspace.
+// One ConvFusion feature map: out = ReLU(Linear(X + Conv1x1(LeakyReLU(GN(Conv3x3(X)))))).
+struct CfWeights {
+  const void *cf3_w, *cf3_b, *gamma, *beta, *cf1_w, *cf1_b, *lin_w, *lin_b;
+};
 template <typename T>
-int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* out, long ldo,
+                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st);
+
+// Steps 1-3: K, V and the per-head [S | z] (fp32) into the workspace. With the
+// Spatial Compressor (the EDiT layer) K = ReLU(DW(Linear_K(X))), V = DW(Linear_V(X));
+// without it the keys and values keep all N tokens: K = ReLU(Linear_K(X)) or the
+// key's own ConvFusion feature map, V = Linear_V(X).
+template <typename T>
+int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit_attn_variant* var, uint8_t* ws,
+           cudaStream_t st) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
   const long tok = static_cast<long>(pl.B) * pl.HW;
   const void* wts[3] = {w->k_w, w->v_w, w->k_w};
   const void* bs[3] = {w->k_b, w->v_b, nullptr};
-  if (pl.bf16)
-    EDIT_TRY(tc_linear(x, tok, pl.C, wts, bs, 2, pl.C, pl.bn_lin, ws + pl.KVp, status, st));
-  else
-    EDIT_TRY(simt_linear(x, tok, pl.C, wts, bs, 2, pl.C, ws + pl.KVp, st));
+  if (pl.k_proc == EDIT_PROC_CF) {
+    // key = ConvFusion feature map with the key's weights (its GroupNorm uses
+    // grid-barrier word 32 of the status block), value = Linear_V(X), side by
+    // side in the token-major K'|V' rows (bf16) or into K and V (fp32)
+    const CfWeights kcf = {var->kcf3_w, var->kcf3_b, var->kgn_gamma, var->kgn_beta,
+                           var->kcf1_w, var->kcf1_b, w->k_w,         w->k_b};
+    const long ldk = pl.bf16 ? 2L * pl.C : pl.C;
+    EDIT_TRY(run_convfusion<T>(x, pl, kcf, w->gn_eps, w->leaky_slope, ws + (pl.bf16 ? pl.KVp : pl.K), ldk, 128,
+                               false, ws, st));
+    const void* vw[1] = {w->v_w};
+    const void* vb[1] = {w->v_b};
+    if (pl.bf16)
+      EDIT_TRY(tc_linear(x, tok, pl.C, vw, vb, 1, pl.C, ws + pl.KVp + pl.C * 2, 2L * pl.C, 0, status, st));
+    else
+      EDIT_TRY(simt_linear(x, tok, pl.C, vw, vb, 1, pl.C, ws + pl.V, pl.C, 0, st));
+  } else if (pl.bf16) {
+    EDIT_TRY(tc_linear(x, tok, pl.C, wts, bs, 2, pl.C, ws + pl.KVp, 2L * pl.C, 0, status, st));
+  } else if (pl.compress) {
+    EDIT_TRY(simt_linear(x, tok, pl.C, wts, bs, 2, pl.C, ws + pl.KVp, 2 * pl.C, 0, st));
+  } else {
+    EDIT_TRY(simt_linear(x, tok, pl.C, wts, bs, 1, pl.C, ws + pl.K, pl.C, 1, st));
+    EDIT_TRY(simt_linear(x, tok, pl.C, wts + 1, bs + 1, 1, pl.C, ws + pl.V, pl.C, 0, st));
+  }
   stage_mark(1, st);
   if (pl.bf16) {
     __nv_bfloat16* KT = reinterpret_cast<__nv_bfloat16*>(ws + pl.KT);
     __nv_bfloat16* VTx = reinterpret_cast<__nv_bfloat16*>(ws + pl.VTx);
-    {
+    if (!pl.compress) {
+      launch_pdl(kv_transpose_kernel, dim3(static_cast<unsigned>((pl.Mp + 63) / 64), pl.B * (2 * pl.C / 64)),
+                 dim3(256), 0, st, reinterpret_cast<const __nv_bfloat16*>(ws + pl.KVp), static_cast<long>(pl.HW),
+                 pl.C, pl.d, pl.heads, pl.NP, static_cast<long>(pl.Mp), KT, VTx);
+      EDIT_TRY(last_launch());
+    } else {
       DwTmaMaps mp;
       std::memset(&mp, 0, sizeof(mp));
       const long C2 = 2L * pl.C;
@@ -693,7 +784,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
     p.status = reinterpret_cast<int*>(ws + pl.status);
     EDIT_TRY(gemm_kvstate(p, pl.NP, st));
   } else {
-    {
+    if (pl.compress) {
       const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C);
       launch_pdl(dwconv_s2_kernel<T, 1>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
           reinterpret_cast<const T*>(ws + pl.KVp), pl.B, pl.H, pl.W, pl.C, static_cast<const T*>(w->kdw_w),
@@ -731,9 +822,11 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* w
 
 // Cooperative launch of the fused GroupNorm (bf16): as many blocks as are
 // co-resident (at most gn_P, the partial buffer's capacity), 512 threads.
-// The grid barrier counter is word 16 of the status block, which every call
-// zeroes before its first launch.
-int launch_gn_fused(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+// The grid barrier counter is the status-block word at byte barrier_off (16 for
+// the query's ConvFusion, 32 for the key's), which every call zeroes before its
+// first launch.
+int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slope, int barrier_off, uint8_t* ws,
+                    cudaStream_t st) {
   // two blocks per SM at most: more blocks only add partials to combine
   int nblk = 2 * num_sms();
   if (nblk > pl.gn_P) nblk = pl.gn_P;
@@ -764,30 +857,37 @@ int launch_gn_fused(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cud
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, gn_fused_bf16_kernel, reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), pl.B,
-                         static_cast<long>(pl.HW), pl.Cr, pl.G, w->gn_eps,
-                         static_cast<const __nv_bfloat16*>(w->gn_gamma), static_cast<const __nv_bfloat16*>(w->gn_beta),
-                         w->leaky_slope, reinterpret_cast<float*>(ws + pl.gnpart),
-                         reinterpret_cast<unsigned int*>(ws + pl.status + 64), reinterpret_cast<float*>(ws + pl.gnstats),
+                         static_cast<long>(pl.HW), pl.Cr, pl.G, gn_eps,
+                         static_cast<const __nv_bfloat16*>(cf.gamma), static_cast<const __nv_bfloat16*>(cf.beta),
+                         slope, reinterpret_cast<float*>(ws + pl.gnpart),
+                         reinterpret_cast<unsigned int*>(ws + pl.status + barrier_off), reinterpret_cast<float*>(ws + pl.gnstats),
                          reinterpret_cast<float*>(ws + pl.gnss), reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb),
                          reinterpret_cast<int*>(ws + pl.status)) != cudaSuccess)
     return EDIT_ERR_CUDA;
   return last_launch();
 }
 
-// Steps 4-7: Q = ReLU([X | G] [Wq | Wq W1]^T + Wq b1 + bq) into the workspace.
+// Steps 4-7 for one ConvFusion feature map (the query's in the EDiT layer):
+// out = ReLU([X | G] [Wl | Wl W1]^T + Wl b1 + bl), rows ldo elements apart,
+// with G = LeakyReLU(GN(Conv3x3(X))) and Wl, bl the Linear after the residual.
+// Stage events 4-7 are recorded when `marks` is set.
 template <typename T>
-int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* qout, long ldo,
+                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
+  auto mark = [&](int i) {
+    if (marks) stage_mark(i, st);
+  };
   const long tok = static_cast<long>(pl.B) * pl.HW;
   const int C = pl.C, Cr = pl.Cr;
   // 4. weight folding
   launch_pdl(transpose_kernel<T>, dim3(dim3(ceil_div(Cr, 32), ceil_div(C, 32))), dim3(dim3(32, 8)), 0, st, 
-      static_cast<const T*>(w->cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t));
+      static_cast<const T*>(cf.cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t));
   EDIT_TRY(last_launch());
   if (pl.bf16) {
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
-    if (!map_a(&p.a0, w->q_w, C, C, 1, C, static_cast<long>(C) * C)) return EDIT_ERR_CUDA;
+    if (!map_a(&p.a0, cf.lin_w, C, C, 1, C, static_cast<long>(C) * C)) return EDIT_ERR_CUDA;
     p.a1 = p.a0;
     if (!map_b(&p.b0, ws + pl.W1t, C, Cr, C, 32)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.bk = p.b0;
@@ -807,7 +907,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
-    p.a0 = static_cast<const float*>(w->q_w);
+    p.a0 = static_cast<const float*>(cf.lin_w);
     p.K0 = C;
     p.b[0] = reinterpret_cast<const float*>(ws + pl.W1t);
     p.n_split = Cr;
@@ -818,10 +918,10 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(C, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
-  launch_pdl(fold_bias_kernel<T>, dim3(ceil_div(C, 8)), dim3(256), 0, st, static_cast<const T*>(w->q_w), static_cast<const T*>(w->q_b),
-                                         static_cast<const T*>(w->cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
+  launch_pdl(fold_bias_kernel<T>, dim3(ceil_div(C, 8)), dim3(256), 0, st, static_cast<const T*>(cf.lin_w), static_cast<const T*>(cf.lin_b),
+                                         static_cast<const T*>(cf.cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
   EDIT_TRY(last_launch());
-  stage_mark(4, st);
+  mark(4);
   // 5. U = Conv3x3(X) (+ GroupNorm partials)
   float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
   bool gn_fused = false;
@@ -830,7 +930,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     std::memset(&p, 0, sizeof(p));
     if (!map_grid(&p.a0, x, pl.B, pl.H, pl.W, C, pl.TW, pl.TH)) return EDIT_ERR_CUDA;
     p.a1 = p.a0;
-    if (!map_b(&p.b0, w->cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr) / 2)) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, cf.cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr) / 2)) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.bk = p.b0;
     p.num_kb = 9 * C / 64;
     p.kb_split = p.num_kb;
@@ -848,37 +948,37 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.out = ws + pl.U;
     p.ldo = Cr;
     if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
-    p.bias[0] = w->cf3_b;
+    p.bias[0] = cf.cf3_b;
     p.status = status;
     if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
       if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
       p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
       bool split = false;
       EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
-      stage_mark(5, st);
+      mark(5);
       if (split) {
         const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
         launch_pdl(conv_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, 
             p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
-            static_cast<const __nv_bfloat16*>(w->cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+            static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
         EDIT_TRY(last_launch());
       }
     } else {
       p.ksplit = pl.conv_ksplit;
       p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
       EDIT_TRY(gemm_conv(p, Cr, st));
-      stage_mark(5, st);
+      mark(5);
       if (pl.conv_ksplit > 1) {
         const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
         launch_pdl(conv_splitk_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit,
                    pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
-                   static_cast<const __nv_bfloat16*>(w->cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+                   static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
         EDIT_TRY(last_launch());
       }
     }
     if ((Cr / pl.G) >= 8 && Cr / 8 <= 512) {
       // 6. G = LeakyReLU(GN(U)) in one cooperative grid: statistics, grid barrier, apply
-      const int r = launch_gn_fused(pl, w, ws, st);
+      const int r = launch_gn_fused(pl, cf, gn_eps, slope, barrier_off, ws, st);
       if (r != EDIT_OK && r != EDIT_ERR_UNSUPPORTED) return r;
       gn_fused = r == EDIT_OK;
     }
@@ -897,8 +997,8 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.H = pl.H;
     p.W = pl.W;
     p.Cin = C;
-    p.b[0] = static_cast<const float*>(w->cf3_w);
-    p.bias[0] = static_cast<const float*>(w->cf3_b);
+    p.b[0] = static_cast<const float*>(cf.cf3_w);
+    p.bias[0] = static_cast<const float*>(cf.cf3_b);
     p.n_split = Cr;
     p.M = static_cast<int>(tok);
     p.N = Cr;
@@ -906,15 +1006,15 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.ldo = Cr;
     launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(tok, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
-    stage_mark(5, st);
+    mark(5);
     launch_pdl(gn_partial_kernel<float>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, reinterpret_cast<const float*>(ws + pl.U),
                                                                   static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
     EDIT_TRY(last_launch());
   }
   // 6. G = LeakyReLU(GN(U))
   if (!gn_fused) {
-    launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), w->gn_eps,
-                                                static_cast<const T*>(w->gn_gamma), static_cast<const T*>(w->gn_beta),
+    launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), gn_eps,
+                                                static_cast<const T*>(cf.gamma), static_cast<const T*>(cf.beta),
                                                 reinterpret_cast<float*>(ws + pl.gnstats),
                                                 reinterpret_cast<float*>(ws + pl.gnss));
     EDIT_TRY(last_launch());
@@ -924,16 +1024,16 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
       const int threads = per_block * nvec;
       launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(threads), 0, st, 
           reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-          w->leaky_slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
+          slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
     } else {
       const long total = tok * Cr;
       launch_pdl(gn_apply_leaky_kernel<float>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
           reinterpret_cast<const float*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-          w->leaky_slope, reinterpret_cast<float*>(ws + pl.Gb), total);
+          slope, reinterpret_cast<float*>(ws + pl.Gb), total);
     }
     EDIT_TRY(last_launch());
   }
-  stage_mark(6, st);
+  mark(6);
   // 7. Q
   if (pl.bf16) {
     TcGemmParams p;
@@ -942,7 +1042,7 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     if (!map_a(&p.a1, ws + pl.Gb, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
     const void* qb = ws + pl.bfold;
     const int lbn = linear_bn(tok, C, 1 << 30, &qb, 1);
-    if (!map_b(&p.b0, w->q_w, C, C, C, linear_box(lbn))) return EDIT_ERR_CUDA;
+    if (!map_b(&p.b0, cf.lin_w, C, C, C, linear_box(lbn))) return EDIT_ERR_CUDA;
     if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, linear_box(lbn))) return EDIT_ERR_CUDA;
     p.b1 = p.b2 = p.b0;
     p.R = static_cast<int>(tok);
@@ -952,9 +1052,9 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.num_kb = C / 64 + ceil_div(Cr, 64);
     p.n_split = 1 << 30;  // one weight source; rows past C read as zeros
     p.N = C;
-    p.out = ws + pl.Q;
-    p.ldo = C;
-    if (!map_out2d(&p.out_map, ws + pl.Q, C, tok, C)) return EDIT_ERR_CUDA;
+    p.out = qout;
+    p.ldo = ldo;
+    if (!map_out2d(&p.out_map, qout, C, tok, ldo)) return EDIT_ERR_CUDA;
     p.bias[0] = ws + pl.bfold;
     p.bias_f32 = 1;
     p.relu = 1;
@@ -967,18 +1067,37 @@ int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t
     p.a1 = reinterpret_cast<const float*>(ws + pl.Gb);
     p.K0 = C;
     p.K1 = Cr;
-    p.b[0] = static_cast<const float*>(w->q_w);
+    p.b[0] = static_cast<const float*>(cf.lin_w);
     p.bk = reinterpret_cast<const float*>(ws + pl.Wqw1);
     p.n_split = C;
     p.M = static_cast<int>(tok);
     p.N = C;
-    p.out = reinterpret_cast<float*>(ws + pl.Q);
-    p.ldo = C;
+    p.out = static_cast<float*>(qout);
+    p.ldo = static_cast<int>(ldo);
     p.bias[0] = reinterpret_cast<const float*>(ws + pl.bfold);
     p.relu = 1;
     launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(C, 64), ceil_div(tok, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
+  mark(7);
+  return EDIT_OK;
+}
+
+// Steps 4-7: the query. ConvFusion (the EDiT layer) or, in the variant
+// without it, Q = ReLU(X Wq^T + bq).
+template <typename T>
+int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
+  if (pl.q_proc == EDIT_PROC_CF) {
+    const CfWeights qcf = {w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b, w->q_w, w->q_b};
+    return run_convfusion<T>(x, pl, qcf, w->gn_eps, w->leaky_slope, ws + pl.Q, pl.C, 64, true, ws, st);
+  }
+  const long tok = static_cast<long>(pl.B) * pl.HW;
+  const void* qw[1] = {w->q_w};
+  const void* qb[1] = {w->q_b};
+  if (pl.bf16)
+    EDIT_TRY(tc_linear(x, tok, pl.C, qw, qb, 1, pl.C, ws + pl.Q, pl.C, 1, reinterpret_cast<int*>(ws + pl.status), st));
+  else
+    EDIT_TRY(simt_linear(x, tok, pl.C, qw, qb, 1, pl.C, ws + pl.Q, pl.C, 1, st));
   stage_mark(7, st);
   return EDIT_OK;
 }
@@ -1023,14 +1142,27 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
   return last_launch();
 }
 
+// One layer: steps 1-8, then (variants with an output Linear) out = Y Wo^T + bo
+// from the attention output Y kept in the workspace (stage event 9).
 template <typename T>
-int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st) {
+int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st,
+             const edit_attn_variant* var = nullptr) {
   if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
   stage_mark(0, st);
-  EDIT_TRY(run_kv<T>(x, pl, w, ws, st));
+  EDIT_TRY(run_kv<T>(x, pl, w, var, ws, st));
   EDIT_TRY(run_query<T>(x, pl, w, ws, st));
-  EDIT_TRY(run_apply<T>(pl, w, ws, out, st));
+  EDIT_TRY(run_apply<T>(pl, w, ws, pl.oproj ? static_cast<void*>(ws + pl.Y) : out, st));
   stage_mark(8, st);
+  if (pl.oproj) {
+    const long tok = static_cast<long>(pl.B) * pl.HW;
+    const void* ow[1] = {var->o_w};
+    const void* ob[1] = {var->o_b};
+    if (pl.bf16)
+      EDIT_TRY(tc_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, reinterpret_cast<int*>(ws + pl.status), st));
+    else
+      EDIT_TRY(simt_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, st));
+    stage_mark(9, st);
+  }
   return EDIT_OK;
 }
 
@@ -1073,9 +1205,9 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   const void* wts[3] = {w->tq_w, w->tk_w, w->tv_w};
   const void* bs[3] = {w->tq_b, w->tk_b, w->tv_b};
   if (pl.bf16)
-    EDIT_TRY(tc_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, pl.bn_lin, ws + pl.QKVt, status, st));
+    EDIT_TRY(tc_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, 3L * pl.C, 0, status, st));
   else
-    EDIT_TRY(simt_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, st));
+    EDIT_TRY(simt_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, 3 * pl.C, 0, st));
   stage_mark(9, st);
   const double eta = static_cast<double>(pl.HW) / static_cast<double>(pl.HW + pl.NT);
   const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
@@ -1129,9 +1261,9 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
 }
 
 int common_checks(const void* x, const void* out, const edit_attn_weights* w, void* ws, size_t ws_bytes,
-                  const Plan& pl) {
+                  const Plan& pl, const edit_attn_variant* var = nullptr) {
   if (!x || !out || !ws) return EDIT_ERR_NULL;
-  EDIT_TRY(check_weights(w));
+  EDIT_TRY(check_weights(w, pl, var));
   if (!aligned(x, 16) || !aligned(out, 16)) return EDIT_ERR_ALIGN;
   if (!aligned(ws, 256)) return EDIT_ERR_ALIGN;
   if (ws_bytes < pl.total) return EDIT_ERR_WORKSPACE;
@@ -1156,6 +1288,24 @@ int edit_attn_forward(const void* x, int B, int H, int W, int C, int heads, cons
   uint8_t* ws = static_cast<uint8_t*>(w->workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st) : run_edit<float>(x, pl, w, ws, out, st);
+}
+
+size_t edit_attn_variant_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights* w,
+                                         const edit_attn_variant* var) {
+  if (!var) return 0;
+  Plan pl;
+  return make_plan(B, H, W, C, heads, 0, w, pl, var) == EDIT_OK ? pl.total : 0;
+}
+
+int edit_attn_variant_forward(const void* x, int B, int H, int W, int C, int heads, const edit_attn_weights* w,
+                              const edit_attn_variant* var, void* out, void* stream) {
+  if (!var) return EDIT_ERR_NULL;
+  Plan pl;
+  EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl, var));
+  EDIT_TRY(common_checks(x, out, w, w->workspace, w->workspace_bytes, pl, var));
+  uint8_t* ws = static_cast<uint8_t*>(w->workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st, var) : run_edit<float>(x, pl, w, ws, out, st, var);
 }
 
 size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights* w) {
@@ -1212,9 +1362,14 @@ const char* edit_status_string(int status) {
 
 int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights* w,
                                edit_ws_layout* layout) {
+  return edit_attn_variant_workspace_layout(B, H, W, C, heads, w, nullptr, layout);
+}
+
+int edit_attn_variant_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights* w,
+                                       const edit_attn_variant* var, edit_ws_layout* layout) {
   if (!layout) return EDIT_ERR_NULL;
   Plan pl;
-  EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl));
+  EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl, var));
   layout->status = static_cast<int64_t>(pl.status);
   layout->U = static_cast<int64_t>(pl.U);
   layout->G = static_cast<int64_t>(pl.Gb);

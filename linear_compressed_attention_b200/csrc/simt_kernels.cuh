@@ -711,6 +711,58 @@ __global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int
   }
 }
 
+// Keys and values without the Spatial Compressor (ablation variants whose
+// keys and values keep all N tokens): the token-major rows kvp [B][N][2C]
+// (first C channels the key, already the Linear output or ReLU'd, the rest
+// the value) become the channel-major operands of the tensor-core KV state,
+// KT [B*C][Mp] = ReLU(key) and rows 0..d-1 of each head block of VTx
+// [B*heads][NP][Mp] = value; tokens N..Mp-1 are written as zeros (Mp % 8 == 0,
+// C % 64 == 0). One block moves 64 tokens x 64 channels through shared
+// memory: 16-byte loads along the channels, 16-byte stores along the tokens
+// (lane pairs write the two halves of one 32-byte sector).
+__global__ void __launch_bounds__(256) kv_transpose_kernel(const __nv_bfloat16* __restrict__ kvp, long N, int C,
+                                                           int d, int heads, int NP, long Mp,
+                                                           __nv_bfloat16* __restrict__ KT,
+                                                           __nv_bfloat16* __restrict__ VTx) {
+  pdl_wait();
+  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // [token][channel], rows padded to 144 bytes
+  const long t0 = static_cast<long>(blockIdx.x) * 64;
+  const int nblk = 2 * C / 64;
+  const int b = blockIdx.y / nblk, gc0 = (blockIdx.y - b * nblk) * 64;
+  for (int e = threadIdx.x; e < 64 * 8; e += 256) {
+    const int tt = e >> 3, v = e & 7;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t0 + tt < N) val = *reinterpret_cast<const uint4*>(kvp + (static_cast<long>(b) * N + t0 + tt) * (2L * C) + gc0 + 8 * v);
+    *reinterpret_cast<uint4*>(&tile[tt][8 * v]) = val;
+  }
+  __syncthreads();
+  const bool isk = gc0 < C;
+  for (int e = threadIdx.x; e < 64 * 8; e += 256) {
+    const int c = (e >> 1) & 63, v = 2 * (e >> 7) + (e & 1);
+    const long n0 = t0 + 8 * v;
+    if (n0 >= Mp) continue;
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = __bfloat162float(tile[8 * v + j][c]);
+      o[j] = isk ? fmaxf(x, 0.f) : x;
+    }
+    uint4 pk;
+    pk.x = pack_bf16x2(o[0], o[1]);
+    pk.y = pack_bf16x2(o[2], o[3]);
+    pk.z = pack_bf16x2(o[4], o[5]);
+    pk.w = pack_bf16x2(o[6], o[7]);
+    __nv_bfloat16* dst;
+    if (isk) {
+      dst = KT + (static_cast<long>(b) * C + gc0 + c) * Mp + n0;
+    } else {
+      const int ch = gc0 - C + c, h = ch / d, r = ch - h * d;
+      dst = VTx + ((static_cast<long>(b) * heads + h) * NP + r) * Mp + n0;
+    }
+    *reinterpret_cast<uint4*>(dst) = pk;
+  }
+}
+
 // Sum of the two fp32 halves of each split conv tile plus the bias -> U (bf16),
 // 4 channels per thread (Cr % 4 == 0). Tile t of the pair grid: CTA `rank`
 // holds 128-pixel tile 2t + rank (one image-row segment of 128 pixels).

@@ -133,3 +133,59 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     assert rc == -9 and bd.status_string(rc) == "request exceeds the library's fixed scratch"
     assert L.edit_linear_attention_noalloc(None, p(0x2000), p(0x3000), 1, 8, 4, 64, 2, 0, ctypes.c_float(1e-6),
                                            p(0x4000), None) == -1
+
+
+def fake_variant(q="cf", k="sc", v="sc", proj=False, base=0x900000):
+    var = bd.make_variant_struct(q, k, v)
+    for j, n in enumerate(bd.VARIANT_NAMES):
+        if n.startswith("o_") and not proj:
+            continue
+        setattr(var, n, base + 0x1000 * (j + 1))
+    return var
+
+
+def vfwd(s, var, B=1, H=64, W=64, C=1152, heads=16):
+    return bd.lib().edit_attn_variant_forward(ctypes.c_void_p(0x200000), B, H, W, C, heads, ctypes.byref(s),
+                                              ctypes.byref(var), ctypes.c_void_p(0x400000), None)
+
+
+def test_variant_workspace_and_processing_checks():
+    s = fake_struct()
+    base = bd.edit_attn_workspace_bytes(1, 64, 64, 1152, 16, s)
+    assert bd.edit_attn_variant_workspace_bytes(1, 64, 64, 1152, 16, s, fake_variant()) == base
+    # uncompressed keys/values (M = N) and the output Linear's buffer need more
+    assert bd.edit_attn_variant_workspace_bytes(1, 64, 64, 1152, 16, s, fake_variant("cf", "none", "none")) > base
+    assert bd.edit_attn_variant_workspace_bytes(1, 64, 64, 1152, 16, s, fake_variant(proj=True)) > base
+    for bad in (("cf", "sc", "none"), ("sc", "sc", "sc"), ("cf", "none", "sc"), ("cf", "cf", "cf")):
+        assert bd.edit_attn_variant_workspace_bytes(1, 64, 64, 1152, 16, s, fake_variant(*bad)) == 0
+        assert vfwd(s, fake_variant(*bad)) == -8
+    lay = bd.edit_attn_variant_workspace_layout(1, 64, 64, 1152, 16, s, fake_variant("none", "none", "none"))
+    assert lay["Mp"] == 4096 and lay["Wop"] == 4096
+    lay = bd.edit_attn_variant_workspace_layout(1, 5, 3, 1152, 16, s, fake_variant("none", "none", "none"))
+    assert lay["Mp"] == 16
+
+
+def test_variant_rejects_missing_weights_it_reads_only():
+    # no ConvFusion anywhere: its weights, c_red and gn_groups are not read
+    s = fake_struct(c_red=0, groups=0)
+    for n in ("cf3_w", "cf3_b", "gn_gamma", "gn_beta", "cf1_w", "cf1_b", "kdw_w", "kdw_b", "vdw_w", "vdw_b"):
+        setattr(s, n, None)
+    var = fake_variant("none", "none", "none")
+    assert bd.edit_attn_variant_workspace_bytes(1, 64, 64, 1152, 16, s, var) > 0
+    s.workspace_bytes = 1024
+    assert vfwd(s, var) == -5                       # validation passes up to the workspace size
+    assert vfwd(s, fake_variant("cf", "none", "none")) == -2   # ConvFusion needs c_red / gn_groups
+    s = fake_struct()
+    var = fake_variant("cf", "cf", "none")
+    var.kcf1_b = None
+    assert vfwd(s, var) == -1
+    var = fake_variant(proj=True)
+    var.o_b = None
+    assert vfwd(s, var) == -1
+    var = fake_variant(proj=True)
+    var.o_w = 0x900008
+    assert vfwd(s, var) == -3
+    s.kdw_w = None
+    assert vfwd(s, fake_variant()) == -1            # the compressor reads the depthwise weights
+    assert bd.lib().edit_attn_variant_forward(ctypes.c_void_p(0x200000), 1, 8, 8, 128, 2, ctypes.byref(s), None,
+                                              ctypes.c_void_p(0x400000), None) == -1
