@@ -34,6 +34,12 @@
  *            allocates, frees or synchronises (except edit_attn_read_status).
  *            Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *            default stream). Outputs must not alias inputs or the workspace.
+ *            Layers of at most 32768 tokens (B*H*W, bf16) run part of their
+ *            kernels on a second stream that the library creates for the
+ *            calling thread and device at its first such call (kept until
+ *            the process exits), forked from `stream` and joined back into it
+ *            within the call: everything still completes in `stream` order.
+ *            Make that first call before any stream capture.
  *   Workspace: caller-allocated device buffer of at least the size returned by
  *            the matching *_workspace_bytes query, 256-byte aligned. Distinct
  *            concurrent calls need distinct workspaces.

@@ -144,6 +144,10 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Planning is host-only (no CUDA call), so chunking uses the B200 SM count.
 int num_sms_hint() { return 148; }
 
+// Layers of at most this many tokens (B * H * W) run their K/V branch
+// concurrently with the query branch (see run_edit).
+constexpr long kForkMaxTokens = 32768;
+
 // Most conv pair tiles ever split in the last wave (at most half of the
 // co-resident pairs).
 constexpr int kConvMaxSplit = 40;
@@ -162,6 +166,7 @@ struct Plan {
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
   int sdpa_split = 0;  // MM-EDiT prompt rows (bf16): ranges of the image keys per query tile, 0 = no split
+  bool fork = false;   // K/V branch on the calling thread's side stream, concurrent with the query branch
   int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
   // query / key / value processing (edit_attn_variant; the EDiT layer is CF, SC, SC)
@@ -321,6 +326,8 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   if (pl.bf16 && pl.TW < 128 && pl.conv_ksplit > 1)  // per-tap conv split over k: one fp32 partial per item
     pl.fixpart = take(static_cast<size_t>(pl.conv_pair_tiles) * pl.conv_ksplit * 2 * 128 * pl.Cr * 4);
   pl.Y = pl.oproj ? take(tok * C * es) : 0;  // attention output before the output Linear
+  // the key ConvFusion shares the query's ConvFusion buffers, so it stays serial
+  pl.fork = pl.bf16 && pl.k_proc != EDIT_PROC_CF && static_cast<long>(B) * pl.HW <= kForkMaxTokens;
   pl.total = off;
   return EDIT_OK;
 }
@@ -369,6 +376,39 @@ thread_local uint64_t g_launches = 0;
 void stage_mark(int i, cudaStream_t st) {
   if (g_stage_events && i < g_stage_n && g_stage_events[i])
     cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), st);
+}
+
+// ------------------------------------------------------------ side stream
+// The K/V branch (steps 1-3) and the query branch (steps 4-7) of a layer share
+// no data. On small layers no kernel fills the GPU for long, so the K/V branch
+// runs on a second stream of the calling thread, forked from the caller's
+// stream after the status reset and joined back into it before the apply, and
+// the two branches' fixed latencies (launch, pipeline fill, last wave)
+// overlap. One non-blocking stream and two events per (thread, device),
+// created by the first such call and kept until the process exits.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+constexpr int kMaxDevices = 64;
+thread_local SideStream g_side[kMaxDevices];
+
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (ss.failed) return nullptr;
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      (void)cudaGetLastError();
+      ss.failed = true;  // run the branches in order on the caller's stream instead
+      return nullptr;
+    }
+  }
+  return &ss;
 }
 
 // ------------------------------------------------------------ launchers
@@ -1149,8 +1189,16 @@ int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t*
              const edit_attn_variant* var = nullptr) {
   if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
   stage_mark(0, st);
-  EDIT_TRY(run_kv<T>(x, pl, w, var, ws, st));
-  EDIT_TRY(run_query<T>(x, pl, w, ws, st));
+  // stage events time the branches one after the other, so they keep one stream
+  SideStream* ss = (pl.fork && !g_stage_events) ? side_stream() : nullptr;
+  if (ss && (cudaEventRecord(ss->fork, st) != cudaSuccess || cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess))
+    return EDIT_ERR_CUDA;
+  const int rkv = run_kv<T>(x, pl, w, var, ws, ss ? ss->s : st);
+  const int rq = (ss || rkv == EDIT_OK) ? run_query<T>(x, pl, w, ws, st) : EDIT_OK;
+  if (ss && (cudaEventRecord(ss->join, ss->s) != cudaSuccess || cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess))
+    return EDIT_ERR_CUDA;  // (joined even when a branch failed: nothing is left running unordered)
+  EDIT_TRY(rkv);
+  EDIT_TRY(rq);
   EDIT_TRY(run_apply<T>(pl, w, ws, pl.oproj ? static_cast<void*>(ws + pl.Y) : out, st));
   stage_mark(8, st);
   if (pl.oproj) {
