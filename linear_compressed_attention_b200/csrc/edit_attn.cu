@@ -269,10 +269,21 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     // (without the compressor: the N tokens in one row padded to a multiple of 8)
     pl.Wop = pl.compress ? (pl.Wo + 31) / 32 * 32 : static_cast<int>((pl.HW + 7) / 8 * 8);
     pl.Mp = pl.compress ? pl.Ho * pl.Wop : pl.Wop;
+    // The persistent kernel gives CTA i the tiles i, i + SMs, ...: pick the
+    // chunk length that minimises (tiles per CTA) x (k-blocks per tile + 2,
+    // the partial's store), i.e. no ragged extra wave of long tiles.
     const int total_kb = (pl.Mp + 63) / 64;
-    const int want = (2 * num_sms_hint() + B * heads - 1) / (B * heads);  // chunks per (image, head)
-    pl.kv_kb = (total_kb + want - 1) / (want > 0 ? want : 1);
-    if (pl.kv_kb < 4) pl.kv_kb = 4;
+    const long bh = static_cast<long>(B) * heads;
+    long best = -1;
+    for (int kb = 4; kb <= (total_kb > 4 ? total_kb : 4); ++kb) {
+      const long chunks = (total_kb + kb - 1) / kb;
+      const long waves = (bh * chunks + num_sms_hint() - 1) / num_sms_hint();
+      const long cost = waves * (kb + 2);
+      if (best < 0 || cost < best) {
+        best = cost;
+        pl.kv_kb = kb;
+      }
+    }
     pl.kv_chunks = (total_kb + pl.kv_kb - 1) / pl.kv_kb;
   } else {
     pl.kv_chunks = pl.M / 256;
@@ -388,7 +399,7 @@ void stage_mark(int i, cudaStream_t st) {
 // created by the first such call and kept until the process exits.
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, fold = nullptr, join = nullptr;
   bool failed = false;
 };
 constexpr int kMaxDevices = 64;
@@ -402,6 +413,7 @@ SideStream* side_stream() {
   if (!ss.s) {
     if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fold, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
       (void)cudaGetLastError();
       ss.failed = true;  // run the branches in order on the caller's stream instead
@@ -719,7 +731,8 @@ struct CfWeights {
 };
 template <typename T>
 int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* out, long ldo,
-                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st);
+                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st, bool fold = true,
+                   cudaEvent_t fold_ready = nullptr);
 
 // Steps 1-3: K, V and the per-head [S | z] (fp32) into the workspace. With the
 // Spatial Compressor (the EDiT layer) K = ReLU(DW(Linear_K(X))), V = DW(Linear_V(X));
@@ -727,7 +740,7 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
 // key's own ConvFusion feature map, V = Linear_V(X).
 template <typename T>
 int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit_attn_variant* var, uint8_t* ws,
-           cudaStream_t st) {
+           cudaStream_t st, cudaEvent_t after_linear = nullptr) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
   const long tok = static_cast<long>(pl.B) * pl.HW;
   const void* wts[3] = {w->k_w, w->v_w, w->k_w};
@@ -756,6 +769,7 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
     EDIT_TRY(simt_linear(x, tok, pl.C, wts + 1, bs + 1, 1, pl.C, ws + pl.V, pl.C, 0, st));
   }
   stage_mark(1, st);
+  if (after_linear && cudaEventRecord(after_linear, st) != cudaSuccess) return EDIT_ERR_CUDA;
   if (pl.bf16) {
     __nv_bfloat16* KT = reinterpret_cast<__nv_bfloat16*>(ws + pl.KT);
     __nv_bfloat16* VTx = reinterpret_cast<__nv_bfloat16*>(ws + pl.VTx);
@@ -791,15 +805,17 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
           return EDIT_ERR_CUDA;
       }
       launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, 
-          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
+          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.NP, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
           static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
           static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
       EDIT_TRY(last_launch());
     }
-    const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
-    launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP,
-               pl.Mp, reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT), pl.KP);
-    EDIT_TRY(last_launch());
+    if (!pl.compress) {  // (the depthwise conv writes these rows itself)
+      const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
+      launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d,
+                 pl.NP, pl.Mp);
+      EDIT_TRY(last_launch());
+    }
     stage_mark(2, st);
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -846,8 +862,9 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
     const int per_head = pl.d * (pl.d + 1);
     const long total = static_cast<long>(pl.B) * pl.heads * per_head;
     if (pl.bf16) {
-      launch_pdl(kv_state_combine_pack_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st,
-                 reinterpret_cast<const float*>(ws + pl.kvpart), pl.kv_chunks, pl.d, pl.NP, pl.KP, total,
+      const long total_t = static_cast<long>(pl.B) * pl.heads * pl.NP * pl.KP;
+      launch_pdl(kv_state_combine_pack_kernel, dim3(grid_for(total_t, 256)), dim3(256), 0, st,
+                 reinterpret_cast<const float*>(ws + pl.kvpart), pl.kv_chunks, pl.d, pl.NP, pl.KP, total_t,
                  reinterpret_cast<float*>(ws + pl.Sz), reinterpret_cast<__nv_bfloat16*>(ws + pl.SzT));
     } else {
       launch_pdl(kv_state_combine_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st,
@@ -907,22 +924,18 @@ int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slo
   return last_launch();
 }
 
-// Steps 4-7 for one ConvFusion feature map (the query's in the EDiT layer):
-// out = ReLU([X | G] [Wl | Wl W1]^T + Wl b1 + bl), rows ldo elements apart,
-// with G = LeakyReLU(GN(Conv3x3(X))) and Wl, bl the Linear after the residual.
-// Stage events 4-7 are recorded when `marks` is set.
+// Step 4 for one ConvFusion feature map: the weight folding
+// Wlw1 = Wl W1 and bl' = Wl b1 + bl (Wl, bl: the Linear after the residual).
+// It reads only weights, so it may run on another stream than the steps that
+// follow (the caller orders it before the query GEMM).
 template <typename T>
-int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* qout, long ldo,
-                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st) {
+int run_fold(const Plan& pl, const CfWeights& cf, uint8_t* ws, cudaStream_t st) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
-  auto mark = [&](int i) {
-    if (marks) stage_mark(i, st);
-  };
-  const long tok = static_cast<long>(pl.B) * pl.HW;
   const int C = pl.C, Cr = pl.Cr;
   // 4. weight folding
-  launch_pdl(transpose_kernel<T>, dim3(dim3(ceil_div(Cr, 32), ceil_div(C, 32))), dim3(dim3(32, 8)), 0, st, 
-      static_cast<const T*>(cf.cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t));
+  launch_pdl(fold_prep_kernel<T>, dim3(ceil_div(Cr, 32) * ceil_div(C, 32) + ceil_div(C, 8)), dim3(256), 0, st,
+             static_cast<const T*>(cf.cf1_w), C, Cr, reinterpret_cast<T*>(ws + pl.W1t), static_cast<const T*>(cf.lin_w),
+             static_cast<const T*>(cf.lin_b), static_cast<const T*>(cf.cf1_b), reinterpret_cast<float*>(ws + pl.bfold));
   EDIT_TRY(last_launch());
   if (pl.bf16) {
     TcGemmParams p;
@@ -958,9 +971,26 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
     launch_pdl(simt_gemm_f32, dim3(dim3(ceil_div(Cr, 64), ceil_div(C, 64))), dim3(256), 0, st, p);
     EDIT_TRY(last_launch());
   }
-  launch_pdl(fold_bias_kernel<T>, dim3(ceil_div(C, 8)), dim3(256), 0, st, static_cast<const T*>(cf.lin_w), static_cast<const T*>(cf.lin_b),
-                                         static_cast<const T*>(cf.cf1_b), C, reinterpret_cast<float*>(ws + pl.bfold));
-  EDIT_TRY(last_launch());
+
+  return EDIT_OK;
+}
+
+// Steps 4-7 for one ConvFusion feature map (the query's in the EDiT layer):
+// out = ReLU([X | G] [Wl | Wl W1]^T + Wl b1 + bl), rows ldo elements apart,
+// with G = LeakyReLU(GN(Conv3x3(X))) and Wl, bl the Linear after the residual.
+// Stage events 4-7 are recorded when `marks` is set. With `fold` false the
+// folded weights come from run_fold on another stream, which records
+// `fold_ready` after it: the query GEMM waits for that event.
+template <typename T>
+int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* qout, long ldo,
+                   int barrier_off, bool marks, uint8_t* ws, cudaStream_t st, bool fold, cudaEvent_t fold_ready) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  auto mark = [&](int i) {
+    if (marks) stage_mark(i, st);
+  };
+  const long tok = static_cast<long>(pl.B) * pl.HW;
+  const int C = pl.C, Cr = pl.Cr;
+  if (fold) EDIT_TRY(run_fold<T>(pl, cf, ws, st));
   mark(4);
   // 5. U = Conv3x3(X) (+ GroupNorm partials)
   float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
@@ -1075,6 +1105,7 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
   }
   mark(6);
   // 7. Q
+  if (fold_ready && cudaStreamWaitEvent(st, fold_ready, 0) != cudaSuccess) return EDIT_ERR_CUDA;
   if (pl.bf16) {
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -1125,12 +1156,16 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
 
 // Steps 4-7: the query. ConvFusion (the EDiT layer) or, in the variant
 // without it, Q = ReLU(X Wq^T + bq).
+CfWeights query_cf(const edit_attn_weights* w) {
+  return CfWeights{w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b, w->q_w, w->q_b};
+}
+
 template <typename T>
-int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st) {
-  if (pl.q_proc == EDIT_PROC_CF) {
-    const CfWeights qcf = {w->cf3_w, w->cf3_b, w->gn_gamma, w->gn_beta, w->cf1_w, w->cf1_b, w->q_w, w->q_b};
-    return run_convfusion<T>(x, pl, qcf, w->gn_eps, w->leaky_slope, ws + pl.Q, pl.C, 64, true, ws, st);
-  }
+int run_query(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, cudaStream_t st,
+              bool fold = true, cudaEvent_t fold_ready = nullptr) {
+  if (pl.q_proc == EDIT_PROC_CF)
+    return run_convfusion<T>(x, pl, query_cf(w), w->gn_eps, w->leaky_slope, ws + pl.Q, pl.C, 64, true, ws, st, fold,
+                             fold_ready);
   const long tok = static_cast<long>(pl.B) * pl.HW;
   const void* qw[1] = {w->q_w};
   const void* qb[1] = {w->q_b};
@@ -1189,15 +1224,39 @@ int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t*
              const edit_attn_variant* var = nullptr) {
   if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
   stage_mark(0, st);
-  // stage events time the branches one after the other, so they keep one stream
-  SideStream* ss = (pl.fork && !g_stage_events) ? side_stream() : nullptr;
-  if (ss && (cudaEventRecord(ss->fork, st) != cudaSuccess || cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess))
-    return EDIT_ERR_CUDA;
-  const int rkv = run_kv<T>(x, pl, w, var, ws, ss ? ss->s : st);
-  const int rq = (ss || rkv == EDIT_OK) ? run_query<T>(x, pl, w, ws, st) : EDIT_OK;
+  // Side stream (bf16; stage events time the steps one after the other, so
+  // they keep one stream): the query's weight folding, which reads only
+  // weights, and for small layers the whole K/V branch. Small layers fork at
+  // the start (side: folding, then K/V; main: conv, GroupNorm, query); larger
+  // ones fork after the K|V GEMM, so the folding fills SMs the memory-bound
+  // depthwise conv leaves idle instead of delaying the GEMM's CTAs. The key
+  // ConvFusion shares the folding buffers, so that variant stays serial.
+  const bool side_fold = pl.bf16 && pl.q_proc == EDIT_PROC_CF && pl.k_proc != EDIT_PROC_CF;
+  SideStream* ss = (!g_stage_events && (pl.fork || side_fold)) ? side_stream() : nullptr;
+  const bool fold_on_side = ss && side_fold;
+  int rkv = EDIT_OK, rq = EDIT_OK, rs = EDIT_OK;
+  if (ss && pl.fork) {
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess) return EDIT_ERR_CUDA;
+  } else if (ss) {
+    rkv = run_kv<T>(x, pl, w, var, ws, st, ss->fork);
+    if (rkv != EDIT_OK) return rkv;  // nothing was forked yet
+  }
+  if (ss) {
+    if (cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess) return EDIT_ERR_CUDA;
+    if (fold_on_side) {
+      rs = run_fold<T>(pl, query_cf(w), ws, ss->s);
+      if (cudaEventRecord(ss->fold, ss->s) != cudaSuccess && rs == EDIT_OK) rs = EDIT_ERR_CUDA;
+    }
+    if (pl.fork && rs == EDIT_OK) rs = run_kv<T>(x, pl, w, var, ws, ss->s);
+  } else {
+    rkv = run_kv<T>(x, pl, w, var, ws, st);
+  }
+  if (rkv == EDIT_OK && rs == EDIT_OK)
+    rq = run_query<T>(x, pl, w, ws, st, !fold_on_side, fold_on_side ? ss->fold : nullptr);
   if (ss && (cudaEventRecord(ss->join, ss->s) != cudaSuccess || cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess))
-    return EDIT_ERR_CUDA;  // (joined even when a branch failed: nothing is left running unordered)
+    return EDIT_ERR_CUDA;  // (joined even when a step failed: nothing is left running unordered)
   EDIT_TRY(rkv);
+  EDIT_TRY(rs);
   EDIT_TRY(rq);
   EDIT_TRY(run_apply<T>(pl, w, ws, pl.oproj ? static_cast<void*>(ws + pl.Y) : out, st));
   stage_mark(8, st);

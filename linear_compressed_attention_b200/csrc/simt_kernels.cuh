@@ -481,10 +481,9 @@ __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, 
 
 // bq' = Wq b1 + bq, one warp per output row (fp32).
 template <typename T>
-__global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__ bq, const T* __restrict__ b1,
-                                 int C, float* __restrict__ out) {
-  pdl_wait();
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+__device__ __forceinline__ void fold_bias_rows(const T* __restrict__ wq, const T* __restrict__ bq,
+                                               const T* __restrict__ b1, int C, float* __restrict__ out, int blk) {
+  const int row = blk * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= C) return;
   float s = 0.f;
@@ -502,6 +501,40 @@ __global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__
   }
   s = warp_sum(s);
   if (lane == 0) out[row] = s + to_f32(bq[row]);
+}
+
+template <typename T>
+__global__ void fold_bias_kernel(const T* __restrict__ wq, const T* __restrict__ bq, const T* __restrict__ b1,
+                                 int C, float* __restrict__ out) {
+  pdl_wait();
+  fold_bias_rows(wq, bq, b1, C, out, blockIdx.x);
+}
+
+// The two inputs of the weight folding in one launch of 256-thread blocks:
+// blocks [0, tiles_r * tiles_c) transpose W1 [C][Cr] -> W1t [Cr][C] in 32 x 32
+// tiles, the following ceil(C / 8) blocks form bq' = Wq b1 + bq (fp32).
+template <typename T>
+__global__ void __launch_bounds__(256) fold_prep_kernel(const T* __restrict__ w1, int C, int Cr, T* __restrict__ w1t,
+                                                        const T* __restrict__ wq, const T* __restrict__ bq,
+                                                        const T* __restrict__ b1, float* __restrict__ bout) {
+  pdl_wait();
+  __shared__ T tile[32][33];
+  const int tiles_c = (Cr + 31) / 32, ntr = tiles_c * ((C + 31) / 32);
+  if (static_cast<int>(blockIdx.x) >= ntr) {
+    fold_bias_rows(wq, bq, b1, C, bout, blockIdx.x - ntr);
+    return;
+  }
+  const int c0 = (blockIdx.x % tiles_c) * 32, r0 = (blockIdx.x / tiles_c) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + tx;
+    if (r < C && c < Cr) tile[i][tx] = w1[static_cast<long>(r) * Cr + c];
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + tx;
+    if (r < C && c < Cr) w1t[static_cast<long>(c) * C + r] = tile[tx][i];
+  }
 }
 
 // ====================================================== depthwise stride-2
@@ -584,7 +617,7 @@ struct DwTmaMaps {
 };
 
 __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constant__ DwTmaMaps m, int H, int W, int C,
-                                                            int d, int heads, int Wop,
+                                                            int d, int heads, int NP, int Wop,
                                                             const __nv_bfloat16* __restrict__ kw,
                                                             const __nv_bfloat16* __restrict__ kb,
                                                             const __nv_bfloat16* __restrict__ vw,
@@ -595,6 +628,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
   __shared__ __align__(128) __nv_bfloat16 in_s[3][PW][CB];
   __shared__ __align__(128) __nv_bfloat16 tok_s[JT][CB];    // [token][channel]
+  __shared__ __align__(128) __nv_bfloat16 pad_s[2][8 * JT];  // 8 VTx rows: ones row + 7 zero rows; 8 zero rows
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   const int Wo = (W + 1) / 2;
@@ -611,6 +645,10 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
+  // rows d..NP-1 of a head's VTx block (the ones row that yields z, then zeros);
+  // each row is one constant, so the 64-byte swizzle of the stores leaves it as is
+  for (int e = threadIdx.x; e < 2 * 8 * JT; e += blockDim.x)
+    pad_s[e / (8 * JT)][e % (8 * JT)] = __float2bfloat16_rn(e < JT ? 1.f : 0.f);
   __syncthreads();
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&m.in);
@@ -672,6 +710,8 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
         const int ch = ch0 + 8 * g;
         const int h = ch / d, rr = ch - h * d;
         tma_store_3d(&m.vtx, out_s + 8 * g * JT, t0, rr, b * heads + h);
+        if (rr + 8 == d)  // the head's last 8 value rows: this block also writes its padding rows
+          for (int pr = d; pr < NP; pr += 8) tma_store_3d(&m.vtx, pad_s[pr == d ? 0 : 1], t0, pr, b * heads + h);
       }
     }
     if (tokmajor && j0 < Wo) tma_store_4d(isk ? &m.ktok : &m.vtok, &tok_s[0][0], ch0, j0, i, b);
@@ -682,19 +722,10 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
 
 // Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
 // KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
-// (Mp % 8 == 0).
-__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp,
-                                    __nv_bfloat16* __restrict__ SzT, int KP) {
+// (Mp % 8 == 0). Used with the uncompressed keys/values; the depthwise conv
+// writes these rows itself.
+__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
   pdl_wait();
-  // also the zero padding of the apply operand SzT [BH][NP][KP]: rows c in
-  // (d, NP) and columns a in [d, KP) of rows c <= d (the combine fills the rest)
-  const long szn = static_cast<long>(BH) * NP * KP;
-  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < szn;
-       i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const int a = static_cast<int>(i % KP);
-    const int c = static_cast<int>((i / KP) % NP);
-    if (c > d || a >= d) SzT[i] = __float2bfloat16_rn(0.f);
-  }
   const int vpr = Mp / 8;                   // vectors per row
   const int rows = NP - d;
   const long total = static_cast<long>(BH) * rows * vpr;
@@ -919,23 +950,28 @@ __global__ void kv_state_combine_kernel(const float* __restrict__ part, int chun
 }
 
 // Same fixed-order combine, also writing [S_h | z_h] as the bf16 B operand of
-// the tensor-core apply: SzT[(b*heads + h)*NP + c][a] = Sz[b][h][a][c] for
-// c <= d, a < d. The zero padding of SzT (c in (d, NP), a in [d, KP)) is
-// written by vtx_pad_rows_kernel.
+// the tensor-core apply: one thread per element of SzT [BH][NP][KP] (total
+// elements); SzT[(b*heads + h)*NP + c][a] = Sz[b][h][a][c], summed over the
+// chunks in order (and stored to Sz fp32 [BH][d][d+1]), for c <= d, a < d;
+// every other element is zero padding.
 __global__ void kv_state_combine_pack_kernel(const float* __restrict__ part, int chunks, int d, int NP, int KP,
                                              long total, float* __restrict__ Sz, __nv_bfloat16* __restrict__ SzT) {
   pdl_wait();
   const int per_head = d * (d + 1);
   for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long bh = i / per_head;
-    const int e = static_cast<int>(i - bh * per_head);
-    const int a = e / (d + 1), c = e - a * (d + 1);
-    const float* q = part + bh * chunks * per_head + e;
+    const int a = static_cast<int>(i % KP);
+    const long r = i / KP;
+    const int c = static_cast<int>(r % NP);
+    const long bh = r / NP;
     float s = 0.f;
-    for (int k = 0; k < chunks; ++k) s += q[static_cast<long>(k) * per_head];
-    Sz[i] = s;
-    SzT[(bh * NP + c) * KP + a] = __float2bfloat16_rn(s);
+    if (c <= d && a < d) {
+      const int e = a * (d + 1) + c;
+      const float* q = part + bh * chunks * per_head + e;
+      for (int k = 0; k < chunks; ++k) s += q[static_cast<long>(k) * per_head];
+      Sz[bh * per_head + e] = s;
+    }
+    SzT[i] = __float2bfloat16_rn(s);
   }
 }
 
