@@ -399,7 +399,7 @@ void stage_mark(int i, cudaStream_t st) {
 // created by the first such call and kept until the process exits.
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, fold = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, fold = nullptr, kv = nullptr, join = nullptr;
   bool failed = false;
 };
 constexpr int kMaxDevices = 64;
@@ -414,6 +414,7 @@ SideStream* side_stream() {
     if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.fold, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.kv, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
       (void)cudaGetLastError();
       ss.failed = true;  // run the branches in order on the caller's stream instead
@@ -1217,62 +1218,6 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
   return last_launch();
 }
 
-// One layer: steps 1-8, then (variants with an output Linear) out = Y Wo^T + bo
-// from the attention output Y kept in the workspace (stage event 9).
-template <typename T>
-int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st,
-             const edit_attn_variant* var = nullptr) {
-  if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
-  stage_mark(0, st);
-  // Side stream (bf16; stage events time the steps one after the other, so
-  // they keep one stream): the query's weight folding, which reads only
-  // weights, and for small layers the whole K/V branch. Small layers fork at
-  // the start (side: folding, then K/V; main: conv, GroupNorm, query); larger
-  // ones fork after the K|V GEMM, so the folding fills SMs the memory-bound
-  // depthwise conv leaves idle instead of delaying the GEMM's CTAs. The key
-  // ConvFusion shares the folding buffers, so that variant stays serial.
-  const bool side_fold = pl.bf16 && pl.q_proc == EDIT_PROC_CF && pl.k_proc != EDIT_PROC_CF;
-  SideStream* ss = (!g_stage_events && (pl.fork || side_fold)) ? side_stream() : nullptr;
-  const bool fold_on_side = ss && side_fold;
-  int rkv = EDIT_OK, rq = EDIT_OK, rs = EDIT_OK;
-  if (ss && pl.fork) {
-    if (cudaEventRecord(ss->fork, st) != cudaSuccess) return EDIT_ERR_CUDA;
-  } else if (ss) {
-    rkv = run_kv<T>(x, pl, w, var, ws, st, ss->fork);
-    if (rkv != EDIT_OK) return rkv;  // nothing was forked yet
-  }
-  if (ss) {
-    if (cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess) return EDIT_ERR_CUDA;
-    if (fold_on_side) {
-      rs = run_fold<T>(pl, query_cf(w), ws, ss->s);
-      if (cudaEventRecord(ss->fold, ss->s) != cudaSuccess && rs == EDIT_OK) rs = EDIT_ERR_CUDA;
-    }
-    if (pl.fork && rs == EDIT_OK) rs = run_kv<T>(x, pl, w, var, ws, ss->s);
-  } else {
-    rkv = run_kv<T>(x, pl, w, var, ws, st);
-  }
-  if (rkv == EDIT_OK && rs == EDIT_OK)
-    rq = run_query<T>(x, pl, w, ws, st, !fold_on_side, fold_on_side ? ss->fold : nullptr);
-  if (ss && (cudaEventRecord(ss->join, ss->s) != cudaSuccess || cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess))
-    return EDIT_ERR_CUDA;  // (joined even when a step failed: nothing is left running unordered)
-  EDIT_TRY(rkv);
-  EDIT_TRY(rs);
-  EDIT_TRY(rq);
-  EDIT_TRY(run_apply<T>(pl, w, ws, pl.oproj ? static_cast<void*>(ws + pl.Y) : out, st));
-  stage_mark(8, st);
-  if (pl.oproj) {
-    const long tok = static_cast<long>(pl.B) * pl.HW;
-    const void* ow[1] = {var->o_w};
-    const void* ob[1] = {var->o_b};
-    if (pl.bf16)
-      EDIT_TRY(tc_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, reinterpret_cast<int*>(ws + pl.status), st));
-    else
-      EDIT_TRY(simt_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, st));
-    stage_mark(9, st);
-  }
-  return EDIT_OK;
-}
-
 template <typename T, int D>
 int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
   if (sizeof(T) == 2) {  // bf16: tensor-core flash-style kernel, 64 query rows per block
@@ -1302,11 +1247,9 @@ int sdpa(const SdpaParams& p, int B, cudaStream_t st) {
   return EDIT_ERR_UNSUPPORTED;
 }
 
+// MM-EDiT, prompt side: the prompt projections [Q_P | K_P | V_P] (stage 9).
 template <typename T>
-int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8_t* ws,
-           void* out_img, void* out_txt, cudaStream_t st) {
-  EDIT_TRY(run_edit<T>(x_img, pl, &w->img, ws, out_img, st));
-  if (pl.NT == 0) return EDIT_OK;  // eta = 1: the image rows are the EDiT layer
+int mm_project(const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8_t* ws, cudaStream_t st) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
   const long trow = static_cast<long>(pl.B) * pl.NT;
   const void* wts[3] = {w->tq_w, w->tk_w, w->tv_w};
@@ -1316,9 +1259,17 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   else
     EDIT_TRY(simt_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, 3 * pl.C, 0, st));
   stage_mark(9, st);
-  const double eta = static_cast<double>(pl.HW) / static_cast<double>(pl.HW + pl.NT);
+  return EDIT_OK;
+}
+
+double mm_eta(const Plan& pl) { return static_cast<double>(pl.HW) / static_cast<double>(pl.HW + pl.NT); }
+
+// Image rows: eta * y + (1 - eta) * A(Q_I, K_P, V_P), blended into out_img,
+// which holds y (stage 10).
+template <typename T>
+int mm_image_rows(const Plan& pl, uint8_t* ws, void* out_img, cudaStream_t st) {
+  const double eta = mm_eta(pl);
   const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
-  // image rows: eta * y + (1 - eta) * A(Q_I, K_P, V_P)
   SdpaParams a;
   std::memset(&a, 0, sizeof(a));
   a.q = ws + pl.Q;
@@ -1337,7 +1288,14 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   a.blend_in = 1;
   EDIT_TRY(sdpa<T>(a, pl.B, st));
   stage_mark(10, st);
-  // text rows: eta * A(Q_P, K_I, V_I) + (1 - eta) * A(Q_P, K_P, V_P)
+  return EDIT_OK;
+}
+
+// Prompt rows: eta * A(Q_P, K_I, V_I) + (1 - eta) * A(Q_P, K_P, V_P) (stage 11).
+template <typename T>
+int mm_prompt_rows(const Plan& pl, uint8_t* ws, void* out_txt, cudaStream_t st) {
+  const double eta = mm_eta(pl);
+  const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
   SdpaParams t;
   std::memset(&t, 0, sizeof(t));
   t.q = qkv;
@@ -1364,6 +1322,98 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   }
   EDIT_TRY(sdpa<T>(t, pl.B, st));
   stage_mark(11, st);
+  return EDIT_OK;
+}
+
+// MM-EDiT prompt-side work that run_edit may put on the side stream after the
+// K/V branch (it needs only K_I, V_I and the prompt tokens): the projections
+// and the prompt rows. `done` tells the caller whether it ran there.
+struct MmPrompt {
+  const void* x_txt;
+  const mmedit_weights* w;
+  void* out_txt;
+  bool done;
+};
+
+// One layer: steps 1-8, then (variants with an output Linear) out = Y Wo^T + bo
+// from the attention output Y kept in the workspace (stage event 9).
+template <typename T>
+int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st,
+             const edit_attn_variant* var = nullptr, MmPrompt* mm = nullptr) {
+  if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
+  stage_mark(0, st);
+  // Side stream (bf16; stage events time the steps one after the other, so
+  // they keep one stream): the query's weight folding, which reads only
+  // weights, and for small layers the whole K/V branch. Small layers fork at
+  // the start (side: folding, then K/V; main: conv, GroupNorm, query); larger
+  // ones fork after the K|V GEMM, so the folding fills SMs the memory-bound
+  // depthwise conv leaves idle instead of delaying the GEMM's CTAs. The key
+  // ConvFusion shares the folding buffers, so that variant stays serial.
+  const bool side_fold = pl.bf16 && pl.q_proc == EDIT_PROC_CF && pl.k_proc != EDIT_PROC_CF;
+  SideStream* ss = (!g_stage_events && (pl.fork || side_fold)) ? side_stream() : nullptr;
+  const bool fold_on_side = ss && side_fold;
+  int rkv = EDIT_OK, rq = EDIT_OK, rs = EDIT_OK;
+  if (ss && pl.fork) {
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess) return EDIT_ERR_CUDA;
+  } else if (ss) {
+    rkv = run_kv<T>(x, pl, w, var, ws, st, ss->fork);
+    if (rkv != EDIT_OK) return rkv;  // nothing was forked yet
+  }
+  if (ss) {
+    if (cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess) return EDIT_ERR_CUDA;
+    if (fold_on_side) {
+      rs = run_fold<T>(pl, query_cf(w), ws, ss->s);
+      if (cudaEventRecord(ss->fold, ss->s) != cudaSuccess && rs == EDIT_OK) rs = EDIT_ERR_CUDA;
+    }
+    if (pl.fork && rs == EDIT_OK) rs = run_kv<T>(x, pl, w, var, ws, ss->s);
+    if (cudaEventRecord(ss->kv, ss->s) != cudaSuccess && rs == EDIT_OK) rs = EDIT_ERR_CUDA;
+    // MM-EDiT: the prompt projections and prompt rows follow the K/V branch there
+    if (pl.fork && mm && pl.NT > 0 && rs == EDIT_OK) {
+      rs = mm_project<T>(mm->x_txt, pl, mm->w, ws, ss->s);
+      if (rs == EDIT_OK) rs = mm_prompt_rows<T>(pl, ws, mm->out_txt, ss->s);
+      mm->done = true;
+    }
+    if (cudaEventRecord(ss->join, ss->s) != cudaSuccess && rs == EDIT_OK) rs = EDIT_ERR_CUDA;
+  } else {
+    rkv = run_kv<T>(x, pl, w, var, ws, st);
+  }
+  if (rkv == EDIT_OK && rs == EDIT_OK)
+    rq = run_query<T>(x, pl, w, ws, st, !fold_on_side, fold_on_side ? ss->fold : nullptr);
+  int ra = EDIT_OK;
+  if (rkv == EDIT_OK && rs == EDIT_OK && rq == EDIT_OK) {
+    // (without the fork the side stream holds only the folding, already awaited)
+    if (ss && pl.fork && cudaStreamWaitEvent(st, ss->kv, 0) != cudaSuccess) ra = EDIT_ERR_CUDA;
+    if (ra == EDIT_OK) ra = run_apply<T>(pl, w, ws, pl.oproj ? static_cast<void*>(ws + pl.Y) : out, st);
+  }
+  if (ss && cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess)
+    return EDIT_ERR_CUDA;  // (joined even when a step failed: nothing is left running unordered)
+  EDIT_TRY(rkv);
+  EDIT_TRY(rs);
+  EDIT_TRY(rq);
+  EDIT_TRY(ra);
+  stage_mark(8, st);
+  if (pl.oproj) {
+    const long tok = static_cast<long>(pl.B) * pl.HW;
+    const void* ow[1] = {var->o_w};
+    const void* ob[1] = {var->o_b};
+    if (pl.bf16)
+      EDIT_TRY(tc_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, reinterpret_cast<int*>(ws + pl.status), st));
+    else
+      EDIT_TRY(simt_linear(ws + pl.Y, tok, pl.C, ow, ob, 1, pl.C, out, pl.C, 0, st));
+    stage_mark(9, st);
+  }
+  return EDIT_OK;
+}
+
+template <typename T>
+int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8_t* ws,
+           void* out_img, void* out_txt, cudaStream_t st) {
+  MmPrompt mm = {x_txt, w, out_txt, false};
+  EDIT_TRY(run_edit<T>(x_img, pl, &w->img, ws, out_img, st, nullptr, &mm));
+  if (pl.NT == 0) return EDIT_OK;  // eta = 1: the image rows are the EDiT layer
+  if (!mm.done) EDIT_TRY(mm_project<T>(x_txt, pl, w, ws, st));
+  EDIT_TRY(mm_image_rows<T>(pl, ws, out_img, st));
+  if (!mm.done) EDIT_TRY(mm_prompt_rows<T>(pl, ws, out_txt, st));
   return EDIT_OK;
 }
 
