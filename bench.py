@@ -297,7 +297,8 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
                                  variant=qkv, out_proj=proj)
         x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
         out = torch.empty_like(x)
-        ms, _ = timed(lambda: layer.forward(x, out))
+        uncompressed = qkv[1] != "sc"
+        ms, st = timed(lambda: layer.forward(x, out), bd.STAGE_EVENTS_EDIT if uncompressed else 0)
         assert layer.status() == 0
         extra = (2 * cfg["C"] * cfg["C"] * 2) if proj else 0
         roof = max(variant_flops(cfg, qkv, proj) / (peaks["bf16_tflops"] * 1e12),
@@ -305,6 +306,18 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
         var["-".join(qkv) + ("+out_linear" if proj else "")] = {
             "tokens_per_s": n / (ms / 1e3), "ms_per_step": ms, "gflop": variant_flops(cfg, qkv, proj) / 1e9,
             "layer_roofline_frac": roof * 1e3 / ms}
+        if uncompressed and st:
+            # kv_transpose_kernel (+ the VTx ones/zero rows), stage 2 of a staged step:
+            # reads K'|V' (N x 2C bf16), writes KT and the value rows of VTx (N x 2C)
+            # and the padding rows (heads x (NP - d) x N)
+            tr_ms = st[1].elapsed_time(st[2])
+            lay = layer.layout
+            tr_bytes = 2 * n * 2 * cfg["C"] * 2 + cfg["heads"] * (lay["NP"] - cfg["C"] // cfg["heads"]) * lay["Mp"] * 2
+            gbs = tr_bytes / (tr_ms / 1e3) / 1e9
+            var["-".join(qkv)]["kv_transpose"] = {
+                "ms": tr_ms, "bytes": tr_bytes, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+                "frac": gbs / peaks["hbm_gbs"], "bound": "hbm",
+                "note": "stage events of one step (no overlap with the neighbouring kernels)"}
         del layer, x, out
     res["variants_px4096"] = var
     cfg = dict(WORKLOADS["mm1024"])
@@ -348,14 +361,17 @@ def run_ours(args, cfg):
     dev = torch.device("cuda", local)
     B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
     N = H * W
-    d = make_inputs(**cfg)
-    layer = bd.EditAttention(d, B, H, W, C, heads, cfg["dtype"], device=dev)
+    qkv, proj = args.qkv, args.proj
+    is_variant = qkv != ("cf", "sc", "sc") or proj
+    d = make_inputs(**cfg, variant_weights=is_variant)
+    layer = bd.EditAttention(d, B, H, W, C, heads, cfg["dtype"], device=dev,
+                             variant=qkv if is_variant else None, out_proj=proj)
     x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
     out = torch.empty_like(x)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    nst = bd.STAGE_EVENTS_EDIT
+    nst = bd.STAGE_EVENTS_EDIT + (1 if proj else 0)
     def new_events():
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
         for e in evs:
@@ -404,8 +420,13 @@ def run_ours(args, cfg):
     assert layer.status() == 0, "device-side status after timing"
 
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    stage_ms = {name: [evs[i].elapsed_time(evs[i + 1]) for evs in per_step_events.values()]
-                for i, name in enumerate(STAGES)}
+    # without a ConvFusion query the folding, conv and GroupNorm events are not
+    # recorded: those stages merge into the query GEMM's
+    names = STAGES + (["out_linear"] if proj else [])
+    bounds = [0] + [i + 1 for i, n in enumerate(names)
+                    if not (qkv[0] == "none" and n in ("fold_weights", "conv3x3", "groupnorm"))]
+    stage_ms = {names[j - 1]: [evs[i].elapsed_time(evs[j]) for evs in per_step_events.values()]
+                for i, j in zip(bounds[:-1], bounds[1:])}
     total_ms = float(sum(step_ms))
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -466,11 +487,18 @@ def run_ours(args, cfg):
     if rank == 0:
         peaks = load_peaks()
         fl = layer_flops(cfg)
-        dom_ms = statistics.mean(stage_ms[DOMINANT])
-        achieved = fl["conv3x3"] / (dom_ms / 1e3) / 1e12
-        traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["src_sha"] == kernel_src_sha() else None
+        # dominant kernel: the 3x3 conv of the ConvFusion query, else the K|V GEMM
+        dominant, dom_kernel, dom_flops = (
+            (DOMINANT, "tc_conv_pair_kernel conv3x3 implicit GEMM", fl["conv3x3"]) if qkv[0] == "cf" else
+            ("kv_linear", "tc_linear_ring_kernel K|V Linear", fl["kv_linear"]))
+        dom_ms = statistics.mean(stage_ms[dominant])
+        achieved = dom_flops / (dom_ms / 1e3) / 1e12
+        traffic = (TRAFFIC["bytes_per_launch"] if TRAFFIC["src_sha"] == kernel_src_sha() and not is_variant
+                   and args.workload == "px4096" else None)
         ms_per_step = total_ms / args.steps
-        roof_t = max(fl["total"] / (peaks["bf16_tflops"] * 1e12), min_bytes(cfg) / (peaks["hbm_gbs"] * 1e9))
+        vflops = variant_flops(cfg, qkv, proj)
+        vbytes = min_bytes(cfg) + (2 * C * C * 2 if proj else 0)
+        roof_t = max(vflops / (peaks["bf16_tflops"] * 1e12), vbytes / (peaks["hbm_gbs"] * 1e9))
         line = {
             "metric": args.metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -478,7 +506,7 @@ def run_ours(args, cfg):
             "config": {"workload": args.workload_desc, "global_batch": world * B, "seq_len": N,
                        "parallelism": f"independent images, {world} rank(s)",
                        "l2": "flushed between steps (256 MB write, outside the timed events); input 151 MB > L2"},
-            "roofline": {"bound": "tensor", "kernel": "tc_gemm conv3x3 implicit GEMM", "achieved": achieved,
+            "roofline": {"bound": "tensor", "kernel": dom_kernel, "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                          "peak_source": f"{peaks['source']} bf16 burst", "launch_ms": dom_ms},
@@ -491,9 +519,9 @@ def run_ours(args, cfg):
                     "d2h_bytes_per_step": nbytes},
             "gpu_launches": launches,
         }
-        if args.workload == "px4096" and not args.no_side:
+        if args.workload == "px4096" and args.variant == "cf-sc-sc" and not args.no_side:
             line["other_sizes"] = side_measurements(dev, peaks)
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.variant == "cf-sc-sc":
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -510,6 +538,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the side measurements (other sizes, variants, MM-EDiT)")
+    ap.add_argument("--variant", default="cf-sc-sc",
+                    help="query-key-value processing of the timed layer, each cf | sc | none (ablation table), "
+                         "optionally +out_linear; default the EDiT layer cf-sc-sc")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -517,8 +548,14 @@ def main():
     if cfg.get("n_txt"):
         raise SystemExit("bench.py times the EDiT layer workloads; MM-EDiT is covered by the tests")
     args.metric = "EDiT attention-layer tokens/sec (bf16, B=1) at 4K/16K/64K tokens; % roofline"
+    args.proj = args.variant.endswith("+out_linear")
+    args.qkv = tuple(args.variant.replace("+out_linear", "").split("-"))
+    if len(args.qkv) != 3 or any(v not in ("cf", "sc", "none") for v in args.qkv):
+        raise SystemExit(f"--variant {args.variant}: expected q-k-v with each cf | sc | none")
     M = ((cfg["H"] + 1) // 2) * ((cfg["W"] + 1) // 2)
-    args.workload_desc = (f"{args.workload}: EDiT layer, B={cfg['B']}, {cfg['H']}x{cfg['W']} grid "
+    args.workload_desc = (f"{args.workload}: EDiT layer"
+                          + ("" if args.variant == "cf-sc-sc" else f" (Q/K/V processing {args.variant})")
+                          + f", B={cfg['B']}, {cfg['H']}x{cfg['W']} grid "
                           f"(N={cfg['H'] * cfg['W']}, M={M}), C={cfg['C']}, c_red={cfg['c_red']}, "
                           f"{cfg['heads']} heads x {cfg['C'] // cfg['heads']}, GN {cfg['gn_groups']} groups, "
                           f"{cfg['dtype']}" + (", 5% outlier tokens x8" if cfg["outliers"] else ""))

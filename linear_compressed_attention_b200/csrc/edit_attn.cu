@@ -806,12 +806,12 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
           return EDIT_ERR_CUDA;
       }
       launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, 
-          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.NP, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
+          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
           static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
           static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
       EDIT_TRY(last_launch());
     }
-    if (!pl.compress) {  // (the depthwise conv writes these rows itself)
+    {
       const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
       launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d,
                  pl.NP, pl.Mp);

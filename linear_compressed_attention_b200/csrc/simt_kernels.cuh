@@ -617,7 +617,7 @@ struct DwTmaMaps {
 };
 
 __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constant__ DwTmaMaps m, int H, int W, int C,
-                                                            int d, int heads, int NP, int Wop,
+                                                            int d, int heads, int Wop,
                                                             const __nv_bfloat16* __restrict__ kw,
                                                             const __nv_bfloat16* __restrict__ kb,
                                                             const __nv_bfloat16* __restrict__ vw,
@@ -628,7 +628,6 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
   __shared__ __align__(128) __nv_bfloat16 in_s[3][PW][CB];
   __shared__ __align__(128) __nv_bfloat16 tok_s[JT][CB];    // [token][channel]
-  __shared__ __align__(128) __nv_bfloat16 pad_s[2][8 * JT];  // 8 VTx rows: ones row + 7 zero rows; 8 zero rows
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   const int Wo = (W + 1) / 2;
@@ -645,10 +644,6 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
-  // rows d..NP-1 of a head's VTx block (the ones row that yields z, then zeros);
-  // each row is one constant, so the 64-byte swizzle of the stores leaves it as is
-  for (int e = threadIdx.x; e < 2 * 8 * JT; e += blockDim.x)
-    pad_s[e / (8 * JT)][e % (8 * JT)] = __float2bfloat16_rn(e < JT ? 1.f : 0.f);
   __syncthreads();
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&m.in);
@@ -710,8 +705,6 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
         const int ch = ch0 + 8 * g;
         const int h = ch / d, rr = ch - h * d;
         tma_store_3d(&m.vtx, out_s + 8 * g * JT, t0, rr, b * heads + h);
-        if (rr + 8 == d)  // the head's last 8 value rows: this block also writes its padding rows
-          for (int pr = d; pr < NP; pr += 8) tma_store_3d(&m.vtx, pad_s[pr == d ? 0 : 1], t0, pr, b * heads + h);
       }
     }
     if (tokmajor && j0 < Wo) tma_store_4d(isk ? &m.ktok : &m.vtok, &tok_s[0][0], ch0, j0, i, b);
@@ -722,8 +715,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
 
 // Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
 // KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
-// (Mp % 8 == 0). Used with the uncompressed keys/values; the depthwise conv
-// writes these rows itself.
+// (Mp % 8 == 0).
 __global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
   pdl_wait();
   const int vpr = Mp / 8;                   // vectors per row

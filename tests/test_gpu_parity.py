@@ -261,3 +261,40 @@ def test_workload_px8192_sampled_rows():
     err = max(float(np.max(np.abs(y[r] - ref[r]))) for r in rows) / scale
     print("px8192 sampled rows", err)
     assert err <= 2e-2
+
+
+@pytest.mark.parametrize("name", ["px1024", "px4096"])
+def test_streams_serial_and_graph_paths_agree(name):
+    """The same layer through its three launch paths gives bit-identical
+    outputs: the default (K/V branch and weight folding on the library's side
+    stream), the serial order taken while stage events are recorded, and a
+    CUDA-graph capture of the default path replayed."""
+    cfg = dict(WORKLOADS[name])
+    d = make_inputs(**cfg)
+    layer, x = gpu_layer(cfg, d)
+    y0 = layer.forward(x).clone()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(bd.STAGE_EVENTS_EDIT)]
+    for e in evs:
+        e.record()
+    bd.edit_attn_set_stage_events([e.cuda_event for e in evs])
+    try:
+        y1 = layer.forward(x).clone()
+    finally:
+        bd.edit_attn_set_stage_events(None)
+    torch.cuda.synchronize()
+    out = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward(x, out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert torch.equal(y0, y1) and torch.equal(y0, out)
