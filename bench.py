@@ -193,6 +193,30 @@ def cpu_baseline(cfg, budget_s=15.0):
 
 
 # ------------------------------------------------------------------ arms
+def reduce_max(value, world, device=None):
+    """Max of a per-rank float over all ranks: the whole job takes as long as
+    its slowest rank (identity on one rank)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_config(cfg, rank):
+    """The images rank `rank` processes: the workload's recipe with its seed
+    advanced by the rank, i.e. its own share of a global batch (weak scaling;
+    no data crosses ranks)."""
+    return dict(cfg, seed=cfg["seed"] + rank)
+
+
+def job_tokens_per_s(world, batch, tokens, steps, max_ms):
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return world * batch * tokens * steps / (max_ms / 1e3)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -363,7 +387,7 @@ def run_ours(args, cfg):
     N = H * W
     qkv, proj = args.qkv, args.proj
     is_variant = qkv != ("cf", "sc", "sc") or proj
-    d = make_inputs(**cfg, variant_weights=is_variant)
+    d = make_inputs(**rank_config(cfg, rank), variant_weights=is_variant)
     layer = bd.EditAttention(d, B, H, W, C, heads, cfg["dtype"], device=dev,
                              variant=qkv if is_variant else None, out_proj=proj)
     x = torch.from_numpy(d["x"]).to(dev, layer.tdtype)
@@ -427,13 +451,8 @@ def run_ours(args, cfg):
                     if not (qkv[0] == "none" and n in ("fold_weights", "conv3x3", "groupnorm"))]
     stage_ms = {names[j - 1]: [evs[i].elapsed_time(evs[j]) for evs in per_step_events.values()]
                 for i, j in zip(bounds[:-1], bounds[1:])}
-    total_ms = float(sum(step_ms))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    tokens = world * B * N * args.steps
-    value = tokens / (total_ms / 1e3)
+    total_ms = reduce_max(sum(step_ms), world, dev)
+    value = job_tokens_per_s(world, B, N, args.steps, total_ms)
 
     # e2e: pinned host input -> device -> layer -> pinned host output, every
     # step. Three streams pipeline consecutive steps: the copy in of step k+1
@@ -476,12 +495,8 @@ def run_ours(args, cfg):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_run(e2e_steps, e0, e1)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
-    e2e_value = world * B * N * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_tokens_per_s(world, B, N, e2e_steps, e2e_ms)
     nbytes = xh.numel() * xh.element_size()
 
     if rank == 0:
