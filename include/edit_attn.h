@@ -34,12 +34,16 @@
  *            allocates, frees or synchronises (except edit_attn_read_status).
  *            Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *            default stream). Outputs must not alias inputs or the workspace.
- *            Layers of at most 32768 tokens (B*H*W, bf16) run part of their
- *            kernels on a second stream that the library creates for the
- *            calling thread and device at its first such call (kept until
- *            the process exits), forked from `stream` and joined back into it
- *            within the call: everything still completes in `stream` order.
- *            Make that first call before any stream capture.
+ *            bf16 calls run part of their kernels on a second stream that
+ *            the library creates for the calling thread and device at its
+ *            first such call (kept until the process exits): the query's
+ *            weight folding, and for layers of at most 32768 tokens (B*H*W)
+ *            also the key/value branch and MM-EDiT's prompt-side attention.
+ *            It is forked from `stream` and joined back into it within the
+ *            call, so everything still completes in `stream` order and the
+ *            call can be captured in a CUDA graph; make the first call
+ *            before any stream capture. Stage events (below) and the
+ *            key-ConvFusion variant keep every kernel on `stream`.
  *   Workspace: caller-allocated device buffer of at least the size returned by
  *            the matching *_workspace_bytes query, 256-byte aligned. Distinct
  *            concurrent calls need distinct workspaces.
