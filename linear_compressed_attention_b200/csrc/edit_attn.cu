@@ -1056,8 +1056,8 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
     if (!gn_fused) {
       launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, 
           reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
+      EDIT_TRY(last_launch());
     }
-    EDIT_TRY(last_launch());
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
