@@ -189,3 +189,29 @@ def test_variant_rejects_missing_weights_it_reads_only():
     assert vfwd(s, fake_variant()) == -1            # the compressor reads the depthwise weights
     assert bd.lib().edit_attn_variant_forward(ctypes.c_void_p(0x200000), 1, 8, 8, 128, 2, ctypes.byref(s), None,
                                               ctypes.c_void_p(0x400000), None) == -1
+
+
+def _device_present():
+    import torch
+    return torch.cuda.is_available()
+
+
+@pytest.mark.skipif(_device_present(), reason="needs a host without a GPU: the call must reach a failing CUDA call")
+def test_cuda_failure_is_a_status_not_a_crash():
+    """Arguments that pass every host check reach the first CUDA runtime call
+    (the status reset), which fails here for want of a device: the call
+    returns EDIT_ERR_CUDA instead of crashing, for the layer, a variant and
+    MM-EDiT alike. (Skipped where a GPU exists: the fake pointers would then
+    reach a real device.)"""
+    s = fake_struct(ws_bytes=1 << 40)
+    assert fwd(s) == -6
+    assert vfwd(s, fake_variant("none", "none", "none", proj=True)) == -6
+    m = bd.MMEditWeights()
+    m.img = s
+    for k, n in enumerate(bd.TEXT_NAMES):
+        setattr(m, n, 0x800000 + 0x1000 * k)
+    m.workspace, m.workspace_bytes = 0x100000, 1 << 40
+    rc = bd.lib().mmedit_hybrid_forward(ctypes.c_void_p(0x200000), ctypes.c_void_p(0x300000), 1, 64, 64, 333, 1152,
+                                        16, ctypes.byref(m), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x500000), None)
+    assert rc == -6
+    assert bd.status_string(rc) == "CUDA error"
