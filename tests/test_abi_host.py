@@ -215,3 +215,47 @@ def test_cuda_failure_is_a_status_not_a_crash():
                                         16, ctypes.byref(m), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x500000), None)
     assert rc == -6
     assert bd.status_string(rc) == "CUDA error"
+
+
+def _regions(lay, B, H, W, C, heads, c_red, bf16, compress):
+    """(name, offset, bytes) of the intermediates the layout reports, sized as
+    the header documents them."""
+    es = 2 if bf16 else 4
+    N = H * W
+    M = ((H + 1) // 2) * ((W + 1) // 2) if compress else N
+    d = C // heads
+    size = {
+        "U": B * N * c_red * es, "G": B * N * c_red * es, "Q": B * N * C * es, "KVp": B * N * 2 * C * es,
+        "K": B * M * C * es, "V": B * M * C * es, "gn_stats": None, "Sz": B * heads * d * (d + 1) * 4,
+        "KT": B * C * lay["Mp"] * 2, "VTx": B * heads * lay["NP"] * lay["Mp"] * 2,
+    }
+    out = []
+    for name, nbytes in size.items():
+        off = lay[name]
+        if off < 0 or not nbytes:
+            continue
+        out.append((name, off, nbytes))
+    return out
+
+
+@pytest.mark.parametrize("dtype", [bd.EDIT_BF16, bd.EDIT_F32])
+def test_workspace_regions_disjoint_and_inside(dtype):
+    import itertools
+    shapes = [(1, 64, 64, 1152, 16, 288, 32), (2, 9, 7, 128, 2, 64, 8), (1, 1, 1, 128, 4, 64, 4),
+              (3, 12, 20, 384, 6, 256, 8), (1, 5, 130, 128, 1, 128, 8)]
+    if dtype == bd.EDIT_F32:
+        shapes = [(2, 5, 7, 48, 3, 12, 3), (1, 1, 1, 32, 2, 8, 2), (1, 11, 4, 72, 1, 24, 6)]
+    procs = [("cf", "sc", "sc"), ("cf", "cf", "none"), ("none", "sc", "sc"), ("cf", "none", "none"),
+             ("none", "none", "none")]
+    for (B, H, W, C, heads, cr, g), qkv, proj in itertools.product(shapes, procs, (False, True)):
+        s = fake_struct(dtype=dtype, c_red=cr, groups=g)
+        var = fake_variant(*qkv, proj=proj)
+        total = bd.edit_attn_variant_workspace_bytes(B, H, W, C, heads, s, var)
+        assert total > 0, (B, H, W, C, heads, qkv)
+        lay = bd.edit_attn_variant_workspace_layout(B, H, W, C, heads, s, var)
+        cr_used = cr if "cf" in qkv[:2] else 0   # U and G exist only when a ConvFusion runs
+        regs = _regions(lay, B, H, W, C, heads, cr_used, dtype == bd.EDIT_BF16, qkv[1] == "sc")
+        for name, off, nbytes in regs:
+            assert off % 256 == 0 and off + nbytes <= total, (name, off, nbytes, total)
+        for (n1, o1, b1), (n2, o2, b2) in itertools.combinations(regs, 2):
+            assert o1 + b1 <= o2 or o2 + b2 <= o1, (qkv, n1, o1, b1, n2, o2, b2)
