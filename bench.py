@@ -534,7 +534,8 @@ def run_ours(args, cfg):
                     "d2h_bytes_per_step": nbytes},
             "gpu_launches": launches,
         }
-        if args.workload == "px4096" and args.variant == "cf-sc-sc" and not args.no_side:
+        # side lines on one rank only (the others would wait at the final barrier)
+        if world == 1 and args.workload == "px4096" and args.variant == "cf-sc-sc" and not args.no_side:
             line["other_sizes"] = side_measurements(dev, peaks)
         if world == 1 and not args.no_cpu_baseline and args.variant == "cf-sc-sc":
             line["cpu_baseline"] = cpu_baseline(cfg)
