@@ -165,14 +165,22 @@ def blas_threads():
         return 1
 
 
-def oracle_rate(cfg, side, reps=1):
-    """tokens/s of the fp64 oracle on a side x side crop of the workload."""
+def oracle_layer(qkv=("cf", "sc", "sc"), proj=False):
+    """The fp64 oracle's layer with the given query/key/value processing."""
     import oracle.edit_oracle as O
+    if qkv == ("cf", "sc", "sc") and not proj:
+        return lambda d, sub: O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+    return lambda d, sub: O.edit_variant_forward(d["x"], sub["H"], sub["W"], d, sub["heads"], *qkv, out_proj=proj)
+
+
+def oracle_rate(cfg, side, reps=1, qkv=("cf", "sc", "sc"), proj=False):
+    """tokens/s of the fp64 oracle on a side x side crop of the workload."""
+    layer = oracle_layer(qkv, proj)
     sub = dict(cfg, B=1, H=min(side, cfg["H"]), W=min(side, cfg["W"]))
-    d = make_inputs(**sub)
+    d = make_inputs(**sub, variant_weights=qkv != ("cf", "sc", "sc") or proj)
     t0 = time.perf_counter()
     for _ in range(reps):
-        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+        layer(d, sub)
     dt = time.perf_counter() - t0
     return reps * sub["H"] * sub["W"] / dt, dt, sub
 
@@ -228,20 +236,20 @@ def run_reference(args, cfg):
     world, rank, _ = dist_setup()
     if rank != 0:
         return
-    import oracle.edit_oracle as O
+    layer = oracle_layer(args.qkv, args.proj)
     # size each step so that warm-up + steps fit in about two minutes
-    r16, _, _ = oracle_rate(cfg, 16)
+    r16, _, _ = oracle_rate(cfg, 16, qkv=args.qkv, proj=args.proj)
     per_step = 60.0 / max(1, args.steps + args.warmup)
     side = 2
     while side < min(cfg["H"], cfg["W"]) and (2 * side) ** 2 / r16 <= per_step:
         side *= 2
     sub = dict(cfg, B=1, H=min(side, cfg["H"]), W=min(side, cfg["W"]))
-    d = make_inputs(**sub)
+    d = make_inputs(**sub, variant_weights=args.qkv != ("cf", "sc", "sc") or args.proj)
     for _ in range(args.warmup):
-        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+        layer(d, sub)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        O.edit_forward(d["x"], sub["H"], sub["W"], d, sub["heads"])
+        layer(d, sub)
     dt = time.perf_counter() - t0
     tok = sub["H"] * sub["W"] * args.steps
     value = tok / dt
