@@ -34,16 +34,20 @@
  *            allocates, frees or synchronises (except edit_attn_read_status).
  *            Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *            default stream). Outputs must not alias inputs or the workspace.
- *            bf16 calls run part of their kernels on a second stream that
- *            the library creates for the calling thread and device at its
- *            first such call (kept until the process exits): the query's
- *            weight folding, and for layers of at most 32768 tokens (B*H*W)
- *            also the key/value branch and MM-EDiT's prompt-side attention.
- *            It is forked from `stream` and joined back into it within the
- *            call, so everything still completes in `stream` order and the
- *            call can be captured in a CUDA graph; make the first call
- *            before any stream capture. Stage events (below) and the
- *            key-ConvFusion variant keep every kernel on `stream`.
+ *            The library creates no streams or events either.
+ *   Streams: a caller may lend a second stream (side_stream, a cudaStream_t
+ *            of the same device, with EDIT_SIDE_EVENTS cudaEvent_t handles in
+ *            side_events, all owned by the caller). bf16 calls then run part
+ *            of their kernels there: the query's weight folding, and for
+ *            layers of at most 32768 tokens (B*H*W) also the key/value branch
+ *            and MM-EDiT's prompt-side attention. The side stream is forked
+ *            from `stream` and joined back into it within the call, so
+ *            everything still completes in `stream` order and the call can be
+ *            captured in a CUDA graph. Calls that share a side stream or its
+ *            events must be ordered on one `stream`. With side_stream NULL
+ *            every kernel runs on `stream`, one after the other (identical
+ *            results). Stage events (below) and the key-ConvFusion variant
+ *            also keep every kernel on `stream`.
  *   Workspace: caller-allocated device buffer of at least the size returned by
  *            the matching *_workspace_bytes query, 256-byte aligned. Distinct
  *            concurrent calls need distinct workspaces.
@@ -71,6 +75,9 @@ extern "C" {
 #endif
 
 typedef enum { EDIT_F32 = 0, EDIT_BF16 = 1 } edit_dtype;
+
+/* Events that go with a caller-provided side stream (see Streams above). */
+#define EDIT_SIDE_EVENTS 4
 
 enum {
   EDIT_OK = 0,
@@ -111,10 +118,14 @@ typedef struct {
   const void *vdw_w, *vdw_b;
   void *workspace; /* device, 256-byte aligned, >= edit_attn_workspace_bytes() */
   size_t workspace_bytes;
+  void *side_stream;                   /* optional cudaStream_t (see Streams), or NULL */
+  void *side_events[EDIT_SIDE_EVENTS]; /* cudaEvent_t handles; required with side_stream */
 } edit_attn_weights;
 
 /* Bytes of workspace edit_attn_forward needs for this shape (0 on a shape or
- * dtype error). Host-only; no CUDA call. */
+ * dtype error). Host-only: no allocation and no launch; the plan reads the
+ * current device's SM count (148 when no device is visible), so query with
+ * the device current that will run the layer. */
 EDIT_API size_t edit_attn_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights *w);
 
 /* One EDiT attention layer: out[B, H*W, C] from x[B, H*W, C] (equations
@@ -176,7 +187,8 @@ EDIT_API int edit_attn_variant_forward(const void *x, int B, int H, int W, int C
 /* Weights of the MM-EDiT hybrid: the EDiT image-stream weights (`img`, its
  * dtype field is the dtype of everything) plus the prompt-token projections
  * tq_w, tk_w, tv_w [C][C] (torch Linear layout) and their biases [C]. The
- * workspace fields of `img` are ignored; the ones here are used. */
+ * workspace and side-stream fields of `img` are ignored; the ones here are
+ * used. */
 typedef struct {
   edit_attn_weights img;
   const void *tq_w, *tq_b;
@@ -184,6 +196,8 @@ typedef struct {
   const void *tv_w, *tv_b;
   void *workspace;
   size_t workspace_bytes;
+  void *side_stream;
+  void *side_events[EDIT_SIDE_EVENTS];
 } mmedit_weights;
 
 EDIT_API size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights *w);
@@ -259,6 +273,23 @@ EDIT_API int edit_attn_set_stage_events(void *const *events, int n);
 
 EDIT_API uint64_t edit_attn_kernel_launches(void);
 
+/* Wait drill for the device-side failure path (no counterpart on the page).
+ *
+ * Every device-side wait in the library is bounded and reports
+ * EDIT_ERR_TIMEOUT through the workspace status word instead of hanging. This
+ * hook lets a test make one such wait run out on purpose, without a fault:
+ * while armed (gn_extra_arrivals > 0), the fused GroupNorm kernel of the
+ * calling thread's bf16 forward calls waits at its grid barrier for
+ * gn_extra_arrivals more blocks than it launched, and gives up after
+ * limit_ns nanoseconds (1e3 .. 2e9). Each block then records EDIT_ERR_TIMEOUT
+ * and the first one the wait site (word 1 = 30, word 3 = arrivals seen,
+ * word 4 = arrivals expected, word 5 = blocks launched) and returns without
+ * applying the normalisation; later kernels of the call still run, and their
+ * results are invalid. The GPU context stays usable. The fused kernel runs
+ * for bf16 layers with at least 8 channels per group and c_red <= 4096.
+ * (0, 0) disarms it. Returns EDIT_ERR_SHAPE for arguments out of range. */
+EDIT_API int edit_attn_set_wait_drill(int gn_extra_arrivals, uint64_t limit_ns);
+
 /* Linear attention step without any caller-provided scratch (the paper has
  * no counterpart; this is a deployment convenience).
  *
@@ -274,10 +305,12 @@ EDIT_API uint64_t edit_attn_kernel_launches(void);
  *   heads divide C; the call is asynchronous on `stream`.
  *
  * The scratch is a static device array of EDIT_NOALLOC_SCRATCH_BYTES bytes
- * that every GPU which loads the library keeps until the process exits. A
- * call needs B * heads * d * (d + 1) * 4 bytes for two chunks of partial sums
- * plus the combined [S | z] (d = C / heads, at least 3 such blocks in all);
- * larger requests return EDIT_ERR_SCRATCH without launching anything. The
+ * that every GPU which loads the library keeps until the process exits. Each
+ * [S | z] block is B * heads * d * (d + 1) * 4 bytes (d = C / heads); a call
+ * uses chunks + 1 such blocks (partial sums of each chunk of keys, then the
+ * combined one), at least 3, and they must fit in the scratch: larger
+ * requests return EDIT_ERR_SCRATCH without launching anything. d above 128,
+ * or B or heads above 65535, return EDIT_ERR_UNSUPPORTED. The
  * library never calls cudaMalloc, cudaFree or any allocating routine here.
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream

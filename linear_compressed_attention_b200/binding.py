@@ -22,22 +22,27 @@ TEXT_NAMES = ("tq_w", "tq_b", "tk_w", "tk_b", "tv_w", "tv_b")
 EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_bytes", "mmedit_hybrid_forward",
            "edit_attn_read_status", "edit_status_string", "edit_attn_workspace_layout",
            "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc",
-           "edit_attn_variant_workspace_bytes", "edit_attn_variant_forward", "edit_attn_variant_workspace_layout")
+           "edit_attn_variant_workspace_bytes", "edit_attn_variant_forward", "edit_attn_variant_workspace_layout",
+           "edit_attn_set_wait_drill")
 STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
 PROC = {"none": 0, "cf": 1, "sc": 2}
 VARIANT_NAMES = ("kcf3_w", "kcf3_b", "kgn_gamma", "kgn_beta", "kcf1_w", "kcf1_b", "o_w", "o_b")
+
+
+SIDE_EVENTS = 4
+_SIDE_FIELDS = [("side_stream", ctypes.c_void_p), ("side_events", ctypes.c_void_p * SIDE_EVENTS)]
 
 
 class EditAttnWeights(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("c_red", ctypes.c_int), ("gn_groups", ctypes.c_int),
                 ("gn_eps", ctypes.c_float), ("leaky_slope", ctypes.c_float), ("attn_eps", ctypes.c_float)] + \
                [(n, ctypes.c_void_p) for n in WEIGHT_NAMES] + \
-               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS
 
 
 class MMEditWeights(ctypes.Structure):
     _fields_ = [("img", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in TEXT_NAMES] + \
-               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS
 
 
 class EditAttnVariant(ctypes.Structure):
@@ -82,6 +87,8 @@ def lib():
     L.edit_attn_set_stage_events.restype = i
     L.edit_attn_kernel_launches.argtypes = []
     L.edit_attn_kernel_launches.restype = ctypes.c_uint64
+    L.edit_attn_set_wait_drill.argtypes = [i, ctypes.c_uint64]
+    L.edit_attn_set_wait_drill.restype = i
     L.edit_linear_attention_noalloc.argtypes = [p, p, p, i, i, i, i, i, i, ctypes.c_float, p, p]
     L.edit_linear_attention_noalloc.restype = i
     V = ctypes.POINTER(EditAttnVariant)
@@ -199,6 +206,36 @@ def edit_attn_kernel_launches() -> int:
     return int(lib().edit_attn_kernel_launches())
 
 
+def edit_attn_set_wait_drill(gn_extra_arrivals: int, limit_ns: int) -> int:
+    return int(lib().edit_attn_set_wait_drill(int(gn_extra_arrivals), int(limit_ns)))
+
+
+def set_side(struct, side) -> None:
+    """Lend a side stream to a weights struct: `side` is (stream, [4 events])
+    of torch.cuda objects, or None for none."""
+    if side is None:
+        struct.side_stream = None
+        for i in range(SIDE_EVENTS):
+            struct.side_events[i] = None
+        return
+    stream, events = side
+    struct.side_stream = stream.cuda_stream
+    for i, e in enumerate(events):
+        struct.side_events[i] = e.cuda_event
+
+
+def make_side(device=None):
+    """A side stream and its events for the library's concurrent branches,
+    owned by the caller (kept alive by the returned tuple)."""
+    import torch
+    stream = torch.cuda.Stream(device=device)
+    events = [torch.cuda.Event(enable_timing=False) for _ in range(SIDE_EVENTS)]
+    with torch.cuda.stream(stream):
+        for e in events:
+            e.record(stream)  # torch creates the event handle at its first record
+    return stream, events
+
+
 def make_variant_struct(q_proc="cf", k_proc="sc", v_proc="sc", w: dict | None = None) -> EditAttnVariant:
     """Processing names 'cf' / 'sc' / 'none'; `w` holds the key ConvFusion
     weights and/or the output Linear (o_w, o_b) as device tensors, or None."""
@@ -247,10 +284,12 @@ class EditAttention:
 
     def __init__(self, arrays: dict, B: int, H: int, W: int, C: int, heads: int, dtype: str = "bf16",
                  n_txt: int = 0, mm: bool | None = None, device="cuda", variant: tuple | None = None,
-                 out_proj: bool = False):
+                 out_proj: bool = False, side: bool = True):
         """``variant`` = (q_proc, k_proc, v_proc) names ('cf', 'sc', 'none') and/or
         ``out_proj`` select edit_attn_variant_forward; weights a variant does
-        not read are not copied to the device (NULL in the structs)."""
+        not read are not copied to the device (NULL in the structs). With
+        ``side`` the layer lends the library a side stream and its events
+        (created here, owned by this object) for the concurrent branches."""
         import torch
         self.torch = torch
         self.B, self.H, self.W, self.C, self.heads, self.n_txt = B, H, W, C, heads, int(n_txt or 0)
@@ -287,7 +326,16 @@ class EditAttention:
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.struct = make_weights_struct(self.w, self.code, workspace=self.workspace, **self.consts)
         self.mm_struct = make_mm_struct(self.struct, self.w, self.workspace) if self.mm else None
+        self.side = make_side(device) if side and self.code == EDIT_BF16 else None
+        self.set_side(self.side)
         self.layout = edit_attn_variant_workspace_layout(B, H, W, C, heads, self.struct, self.variant)
+
+    def set_side(self, side) -> None:
+        """Lend (stream, events) to the library, or None to run every kernel
+        on the call's stream."""
+        set_side(self.struct, side)
+        if self.mm_struct is not None:
+            set_side(self.mm_struct, side)
 
     def forward(self, x, out=None, stream=None):
         if out is None:

@@ -18,6 +18,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -132,17 +133,24 @@ bool map_grid(CUtensorMap* m, const void* base, int B, int H, int W, int C, int 
   return encode(m, 4, base, dims, st, box);
 }
 
+// SM count of the current device, read once per device (148, the B200's,
+// when no device is visible, so host-only queries still plan the same way).
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // ------------------------------------------------------------ plan
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Planning is host-only (no CUDA call), so chunking uses the B200 SM count.
-int num_sms_hint() { return 148; }
 
 // Layers of at most this many tokens (B * H * W) run their K/V branch
 // concurrently with the query branch (see run_edit).
@@ -245,7 +253,7 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     pl.conv_pair_tiles = (B * pl.tiles_h * pl.tiles_w + 1) / 2;
     pl.conv_ksplit = 1;
     if (pl.TW < 128) {
-      const int pairs = num_sms_hint() / 2, nkb = 9 * C / 64;
+      const int pairs = num_sms() / 2, nkb = 9 * C / 64;
       if (2 * pl.conv_pair_tiles <= pairs) {
         int k = pairs / pl.conv_pair_tiles;
         if (k > nkb / 9) k = nkb / 9;  // at least 9 k-blocks (one channel block of every tap) per part
@@ -277,7 +285,7 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
     long best = -1;
     for (int kb = 4; kb <= (total_kb > 4 ? total_kb : 4); ++kb) {
       const long chunks = (total_kb + kb - 1) / kb;
-      const long waves = (bh * chunks + num_sms_hint() - 1) / num_sms_hint();
+      const long waves = (bh * chunks + num_sms() - 1) / num_sms();
       const long cost = waves * (kb + 2);
       if (best < 0 || cost < best) {
         best = cost;
@@ -327,7 +335,7 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   if (pl.bf16 && NT > 0) {
     const long ctas = static_cast<long>(B) * heads * ((NT + 63) / 64);
     const int span = NT > 256 ? NT : 256;
-    if (ctas < 2L * num_sms_hint() && pl.M > span) {
+    if (ctas < 2L * num_sms() && pl.M > span) {
       pl.sdpa_split = (pl.M + span - 1) / span;
       pl.sdpapart = take(static_cast<size_t>(B) * heads * NT * (pl.sdpa_split + 1) * (pl.d + 2) * 4);
     }
@@ -383,6 +391,10 @@ namespace {
 thread_local void* const* g_stage_events = nullptr;
 thread_local int g_stage_n = 0;
 thread_local uint64_t g_launches = 0;
+// Wait drill (edit_attn_set_wait_drill): extra arrivals the fused GroupNorm's
+// grid barrier waits for, and its wait limit while armed.
+thread_local int g_drill_extra = 0;
+thread_local uint64_t g_drill_limit_ns = 0;
 
 void stage_mark(int i, cudaStream_t st) {
   if (g_stage_events && i < g_stage_n && g_stage_events[i])
@@ -392,42 +404,43 @@ void stage_mark(int i, cudaStream_t st) {
 // ------------------------------------------------------------ side stream
 // The K/V branch (steps 1-3) and the query branch (steps 4-7) of a layer share
 // no data. On small layers no kernel fills the GPU for long, so the K/V branch
-// runs on a second stream of the calling thread, forked from the caller's
-// stream after the status reset and joined back into it before the apply, and
-// the two branches' fixed latencies (launch, pipeline fill, last wave)
-// overlap. One non-blocking stream and two events per (thread, device),
-// created by the first such call and kept until the process exits.
+// runs on a second stream, forked from the caller's stream after the status
+// reset and joined back into it before the apply, and the two branches' fixed
+// latencies (launch, pipeline fill, last wave) overlap. The stream and its
+// four events belong to the caller (side_stream / side_events of the weights
+// struct); without them every kernel runs on the caller's stream in order.
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, fold = nullptr, kv = nullptr, join = nullptr;
-  bool failed = false;
 };
-constexpr int kMaxDevices = 64;
-thread_local SideStream g_side[kMaxDevices];
 
-SideStream* side_stream() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  SideStream& ss = g_side[dev];
-  if (ss.failed) return nullptr;
-  if (!ss.s) {
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fold, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.kv, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
-      (void)cudaGetLastError();
-      ss.failed = true;  // run the branches in order on the caller's stream instead
-      return nullptr;
-    }
-  }
-  return &ss;
+SideStream side_of(void* stream, void* const* ev) {
+  SideStream ss;
+  if (!stream) return ss;
+  ss.s = static_cast<cudaStream_t>(stream);
+  ss.fork = static_cast<cudaEvent_t>(ev[0]);
+  ss.fold = static_cast<cudaEvent_t>(ev[1]);
+  ss.kv = static_cast<cudaEvent_t>(ev[2]);
+  ss.join = static_cast<cudaEvent_t>(ev[3]);
+  return ss;
+}
+
+// A side stream comes with all four events.
+int check_side(void* stream, void* const* ev) {
+  if (!stream) return EDIT_OK;
+  for (int i = 0; i < EDIT_SIDE_EVENTS; ++i)
+    if (!ev[i]) return EDIT_ERR_NULL;
+  return EDIT_OK;
 }
 
 // ------------------------------------------------------------ launchers
 // Every library kernel launches with programmatic stream serialization: it may
 // start while the previous kernel drains and waits in pdl_wait() for that
-// kernel's memory. Errors surface through cudaGetLastError in last_launch().
+// kernel's memory. The launch's own return code is kept for last_launch()
+// (cudaGetLastError would also report, and clear, errors of the caller's
+// earlier calls).
+thread_local cudaError_t g_launch_err = cudaSuccess;
+
 template <typename... KArgs, typename... Args>
 void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg;
@@ -441,12 +454,14 @@ void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cuda
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  (void)cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  g_launch_err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 int last_launch() {
   ++g_launches;
-  return cudaGetLastError() == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
+  const cudaError_t e = g_launch_err;
+  g_launch_err = cudaSuccess;
+  return e == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
 }
 
 int grid_for(long total, int threads) {
@@ -615,7 +630,7 @@ int linear_bn(long rows, int N, int n_split, const void* const* biases, int nbia
   for (int s = 0; s < nbias; ++s)  // the 384 epilogue reads bias vectors 16 bytes at a time
     if (reinterpret_cast<uintptr_t>(biases[s]) % 16 != 0) return kPairBN;
   const long m_pairs = (ceil_div(rows, 128) + 1) / 2;
-  const long pairs = num_sms_hint() / 2;
+  const long pairs = num_sms() / 2;
   const long w256 = (m_pairs * ceil_div(N, 256) + pairs - 1) / pairs;
   const long w384 = (m_pairs * ceil_div(N, 384) + pairs - 1) / pairs;
   return w384 * 384 * 85 < w256 * 256 * 100 ? 384 : kPairBN;
@@ -880,9 +895,11 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
 
 // Cooperative launch of the fused GroupNorm (bf16): as many blocks as are
 // co-resident (at most gn_P, the partial buffer's capacity), 512 threads.
-// The grid barrier counter is the status-block word at byte barrier_off (16 for
-// the query's ConvFusion, 32 for the key's), which every call zeroes before its
-// first launch.
+// The grid barrier counter is the status-block word at byte barrier_off (64 for
+// the query's ConvFusion, 128 for the key's; clear of the status word and the
+// wait-site words 1-7), which every call zeroes before its first launch. The
+// barrier expects one arrival per block and gives up after EDIT_WAIT_TIMEOUT_NS,
+// unless this thread armed the wait drill (edit_attn_set_wait_drill).
 int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slope, int barrier_off, uint8_t* ws,
                     cudaStream_t st) {
   // two blocks per SM at most: more blocks only add partials to combine
@@ -890,13 +907,13 @@ int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slo
   if (nblk > pl.gn_P) nblk = pl.gn_P;
   if (nblk > GN_FUSED_MAXB) nblk = GN_FUSED_MAXB;
   const size_t smem = (512 * 4 + static_cast<size_t>(pl.Cr) * 4) * sizeof(float);
-  static bool attr_set = false;  // one device model per process
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gn_fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) !=
-        cudaSuccess)
-      return EDIT_ERR_CUDA;
-    attr_set = true;
-  }
+  // (a per-device function attribute; setting it on every launch keeps it
+  // right for whichever device and thread launches)
+  if (cudaFuncSetAttribute(gn_fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) !=
+      cudaSuccess)
+    return EDIT_ERR_CUDA;
+  const unsigned int expect = static_cast<unsigned int>(nblk + (g_drill_extra > 0 ? g_drill_extra : 0));
+  const uint64_t limit_ns = g_drill_extra > 0 ? g_drill_limit_ns : EDIT_WAIT_TIMEOUT_NS;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gn_fused_bf16_kernel, 512, smem) != cudaSuccess ||
       per_sm * num_sms() < nblk)
@@ -920,7 +937,7 @@ int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slo
                          slope, reinterpret_cast<float*>(ws + pl.gnpart),
                          reinterpret_cast<unsigned int*>(ws + pl.status + barrier_off), reinterpret_cast<float*>(ws + pl.gnstats),
                          reinterpret_cast<float*>(ws + pl.gnss), reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb),
-                         reinterpret_cast<int*>(ws + pl.status)) != cudaSuccess)
+                         reinterpret_cast<int*>(ws + pl.status), expect, limit_ns) != cudaSuccess)
     return EDIT_ERR_CUDA;
   return last_launch();
 }
@@ -1339,7 +1356,7 @@ struct MmPrompt {
 // from the attention output Y kept in the workspace (stage event 9).
 template <typename T>
 int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out, cudaStream_t st,
-             const edit_attn_variant* var = nullptr, MmPrompt* mm = nullptr) {
+             const SideStream& side, const edit_attn_variant* var = nullptr, MmPrompt* mm = nullptr) {
   if (cudaMemsetAsync(ws + pl.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
   stage_mark(0, st);
   // Side stream (bf16; stage events time the steps one after the other, so
@@ -1350,7 +1367,7 @@ int run_edit(const void* x, const Plan& pl, const edit_attn_weights* w, uint8_t*
   // depthwise conv leaves idle instead of delaying the GEMM's CTAs. The key
   // ConvFusion shares the folding buffers, so that variant stays serial.
   const bool side_fold = pl.bf16 && pl.q_proc == EDIT_PROC_CF && pl.k_proc != EDIT_PROC_CF;
-  SideStream* ss = (!g_stage_events && (pl.fork || side_fold)) ? side_stream() : nullptr;
+  const SideStream* ss = (!g_stage_events && (pl.fork || side_fold) && side.s) ? &side : nullptr;
   const bool fold_on_side = ss && side_fold;
   int rkv = EDIT_OK, rq = EDIT_OK, rs = EDIT_OK;
   if (ss && pl.fork) {
@@ -1409,7 +1426,7 @@ template <typename T>
 int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8_t* ws,
            void* out_img, void* out_txt, cudaStream_t st) {
   MmPrompt mm = {x_txt, w, out_txt, false};
-  EDIT_TRY(run_edit<T>(x_img, pl, &w->img, ws, out_img, st, nullptr, &mm));
+  EDIT_TRY(run_edit<T>(x_img, pl, &w->img, ws, out_img, st, side_of(w->side_stream, w->side_events), nullptr, &mm));
   if (pl.NT == 0) return EDIT_OK;  // eta = 1: the image rows are the EDiT layer
   if (!mm.done) EDIT_TRY(mm_project<T>(x_txt, pl, w, ws, st));
   EDIT_TRY(mm_image_rows<T>(pl, ws, out_img, st));
@@ -1442,9 +1459,12 @@ int edit_attn_forward(const void* x, int B, int H, int W, int C, int heads, cons
   Plan pl;
   EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl));
   EDIT_TRY(common_checks(x, out, w, w->workspace, w->workspace_bytes, pl));
+  EDIT_TRY(check_side(w->side_stream, w->side_events));
   uint8_t* ws = static_cast<uint8_t*>(w->workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st) : run_edit<float>(x, pl, w, ws, out, st);
+  const SideStream side = side_of(w->side_stream, w->side_events);
+  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st, side)
+                 : run_edit<float>(x, pl, w, ws, out, st, side);
 }
 
 size_t edit_attn_variant_workspace_bytes(int B, int H, int W, int C, int heads, const edit_attn_weights* w,
@@ -1460,9 +1480,12 @@ int edit_attn_variant_forward(const void* x, int B, int H, int W, int C, int hea
   Plan pl;
   EDIT_TRY(make_plan(B, H, W, C, heads, 0, w, pl, var));
   EDIT_TRY(common_checks(x, out, w, w->workspace, w->workspace_bytes, pl, var));
+  EDIT_TRY(check_side(w->side_stream, w->side_events));
   uint8_t* ws = static_cast<uint8_t*>(w->workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st, var) : run_edit<float>(x, pl, w, ws, out, st, var);
+  const SideStream side = side_of(w->side_stream, w->side_events);
+  return pl.bf16 ? run_edit<__nv_bfloat16>(x, pl, w, ws, out, st, side, var)
+                 : run_edit<float>(x, pl, w, ws, out, st, side, var);
 }
 
 size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights* w) {
@@ -1477,6 +1500,7 @@ int mmedit_hybrid_forward(const void* x_img, const void* x_txt, int B, int H, in
   Plan pl;
   EDIT_TRY(make_plan(B, H, W, C, heads, N_T, &w->img, pl));
   EDIT_TRY(common_checks(x_img, out_img, &w->img, w->workspace, w->workspace_bytes, pl));
+  EDIT_TRY(check_side(w->side_stream, w->side_events));
   if (N_T > 0) {
     if (!x_txt || !out_txt) return EDIT_ERR_NULL;
     if (!aligned(x_txt, 16) || !aligned(out_txt, 16)) return EDIT_ERR_ALIGN;
@@ -1554,5 +1578,13 @@ int edit_attn_set_stage_events(void* const* events, int n) {
 }
 
 uint64_t edit_attn_kernel_launches(void) { return g_launches; }
+
+int edit_attn_set_wait_drill(int gn_extra_arrivals, uint64_t limit_ns) {
+  if (gn_extra_arrivals < 0 || gn_extra_arrivals > 1024) return EDIT_ERR_SHAPE;
+  if (gn_extra_arrivals > 0 && (limit_ns < 1000ull || limit_ns > EDIT_WAIT_TIMEOUT_NS)) return EDIT_ERR_SHAPE;
+  g_drill_extra = gn_extra_arrivals;
+  g_drill_limit_ns = gn_extra_arrivals > 0 ? limit_ns : 0;
+  return EDIT_OK;
+}
 
 }  // extern "C"

@@ -35,6 +35,18 @@ int scratch_address(void** out) {
   return EDIT_OK;
 }
 
+// Plain launch on `st`; the launch's own return code (cudaGetLastError would
+// also report, and clear, errors left by the caller's earlier calls).
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
+}
+
 template <typename T>
 int run(const void* q, const void* k, const void* v, int B, int N, int M, int C, int heads, float eps, void* out,
         float* scratch, int chunks, cudaStream_t st) {
@@ -46,21 +58,21 @@ int run(const void* q, const void* k, const void* v, int B, int N, int M, int C,
   int threads = (nb * nb + 31) / 32 * 32;
   if (threads < d) threads = (d + 31) / 32 * 32;
   const size_t smem = 2 * 32 * static_cast<size_t>(d) * sizeof(float);
-  kv_state_partial_kernel<T><<<dim3(chunks, heads, B), threads, smem, st>>>(
-      static_cast<const T*>(k), static_cast<const T*>(v), M, C, heads, chunks, part);
-  if (cudaGetLastError() != cudaSuccess) return EDIT_ERR_CUDA;
+  int rc = launch(kv_state_partial_kernel<T>, dim3(chunks, heads, B), dim3(threads), smem, st,
+                  static_cast<const T*>(k), static_cast<const T*>(v), M, C, heads, chunks, part);
+  if (rc != EDIT_OK) return rc;
   const long total = static_cast<long>(B) * heads * per_head;
   const int grid = static_cast<int>((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-  kv_state_combine_kernel<<<grid, 256, 0, st>>>(part, chunks, static_cast<int>(per_head), total, Sz);
-  if (cudaGetLastError() != cudaSuccess) return EDIT_ERR_CUDA;
+  rc = launch(kv_state_combine_kernel, dim3(grid), dim3(256), 0, st, static_cast<const float*>(part), chunks,
+              static_cast<int>(per_head), total, Sz);
+  if (rc != EDIT_OK) return rc;
   const size_t asmem = static_cast<size_t>(per_head) * sizeof(float);
   if (asmem > 48 * 1024 &&
       cudaFuncSetAttribute(apply_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem) !=
           cudaSuccess)
     return EDIT_ERR_CUDA;
-  apply_simt_kernel<T><<<dim3((N + 127) / 128, heads, B), 128, asmem, st>>>(
-      static_cast<const T*>(q), Sz, N, C, heads, eps, static_cast<T*>(out));
-  return cudaGetLastError() == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
+  return launch(apply_simt_kernel<T>, dim3((N + 127) / 128, heads, B), dim3(128), asmem, st,
+                static_cast<const T*>(q), static_cast<const float*>(Sz), N, C, heads, eps, static_cast<T*>(out));
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -76,6 +88,7 @@ extern "C" int edit_linear_attention_noalloc(const void* q, const void* k, const
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return EDIT_ERR_ALIGN;
   const int d = C / heads;
   if (d > 128) return EDIT_ERR_UNSUPPORTED;
+  if (B > 65535 || heads > 65535) return EDIT_ERR_UNSUPPORTED;  // grid y/z limits
   // blocks of [S | z]: `chunks` partials per (image, head) plus the combined one
   const double block = static_cast<double>(B) * heads * d * (d + 1) * 4.0;
   const double cap = static_cast<double>(EDIT_NOALLOC_SCRATCH_BYTES);

@@ -153,8 +153,9 @@ __global__ void gn_partial_kernel(const T* __restrict__ U, int HW, int Cr, int g
 //  1. per-thread sums of 8-channel vectors (at most two groups per vector),
 //     fixed-order block reduction -> part[b][block][group][2];
 //  2. grid barrier: one arrival per block on a zeroed counter, then a bounded
-//     spin (EDIT_ERR_TIMEOUT after 2 s; the launch is cooperative, so every
-//     block is resident);
+//     spin until `expect` arrivals (gridDim.x in every forward call;
+//     EDIT_ERR_TIMEOUT and wait site 30 after `limit_ns`, 2 s in a forward
+//     call; the launch is cooperative, so every block is resident);
 //  3. per image: every block combines all blocks' partials in the same fixed
 //     order (one warp per group, fp64), forms the per-channel affine form
 //     scale = gamma * rstd, shift = beta - mean * scale, and applies
@@ -170,7 +171,8 @@ __global__ void __launch_bounds__(512) gn_fused_bf16_kernel(const __nv_bfloat16*
                                                             const __nv_bfloat16* __restrict__ beta, float slope,
                                                             float* __restrict__ part, unsigned int* arrive,
                                                             float* __restrict__ stats, float* __restrict__ ss,
-                                                            __nv_bfloat16* __restrict__ G, int* status) {
+                                                            __nv_bfloat16* __restrict__ G, int* status,
+                                                            unsigned int expect, uint64_t limit_ns) {
   pdl_wait();
   extern __shared__ float gf_sm[];
   float* red = gf_sm;                      // [blockDim][4]
@@ -244,9 +246,11 @@ __global__ void __launch_bounds__(512) gn_fused_bf16_kernel(const __nv_bfloat16*
     __threadfence();
     atomicAdd(arrive, 1u);
     const uint64_t w0 = globaltimer_ns();
-    while (*reinterpret_cast<volatile unsigned int*>(arrive) < static_cast<unsigned int>(nblk)) {
-      if (globaltimer_ns() - w0 > EDIT_WAIT_TIMEOUT_NS) {
+    unsigned int seen;
+    while ((seen = *reinterpret_cast<volatile unsigned int*>(arrive)) < expect) {
+      if (globaltimer_ns() - w0 > limit_ns) {
         record_status(status, EDIT_ERR_TIMEOUT);
+        record_wait_site(status, 30, static_cast<int>(seen), static_cast<int>(expect), nblk, 0);
         gf_abort = 1;
         break;
       }

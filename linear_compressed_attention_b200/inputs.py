@@ -126,3 +126,17 @@ def make_workload(name, **overrides):
     cfg = dict(WORKLOADS[name])
     cfg.update(overrides)
     return cfg, make_inputs(**cfg)
+
+
+def make_attention_inputs(B, N, M, C, seed, dtype="bf16"):
+    """Operands of the linear-attention step alone: q [B, N, C] and k [B, M, C]
+    non-negative (|N(0, 1)| draws, like the ReLU feature maps the layer feeds
+    it), v [B, M, C] ~ N(0, 1); drawn in that order from
+    ``numpy.random.default_rng(seed)`` and rounded once to bf16 for bf16."""
+    rng = np.random.default_rng(seed)
+    q = np.abs(rng.standard_normal((B, N, C), dtype=np.float32))
+    k = np.abs(rng.standard_normal((B, M, C), dtype=np.float32))
+    v = rng.standard_normal((B, M, C), dtype=np.float32)
+    if dtype == "bf16":
+        q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+    return q, k, v

@@ -106,6 +106,38 @@ def test_mm_rejects_bad_arguments():
     assert bd.mmedit_workspace_bytes(1, 64, 64, 333, 1536, 24, m) > bd.mmedit_workspace_bytes(1, 64, 64, 0, 1536, 24, m)
 
 
+def test_side_stream_is_optional_and_needs_its_events():
+    """A side stream is lent by the caller with its four events; NULL (the
+    default) is accepted and runs every kernel on the call's stream."""
+    s = fake_struct(ws_bytes=1024)
+    assert s.side_stream is None
+    assert fwd(s) == -5                     # NULL side stream passes validation up to the workspace
+    s = fake_struct()
+    s.side_stream = 0x7000
+    assert fwd(s) == -1                     # events missing
+    for i in range(bd.SIDE_EVENTS):
+        s.side_events[i] = 0x7100 + i
+    s.side_events[2] = None
+    assert fwd(s) == -1
+    m = bd.MMEditWeights()
+    m.img = fake_struct()
+    for k, n in enumerate(bd.TEXT_NAMES):
+        setattr(m, n, 0x800000 + 0x1000 * k)
+    m.workspace, m.workspace_bytes = 0x100000, 1 << 40
+    m.side_stream = 0x7000
+    rc = bd.lib().mmedit_hybrid_forward(ctypes.c_void_p(0x200000), ctypes.c_void_p(0x300000), 1, 64, 64, 333, 1536,
+                                        24, ctypes.byref(m), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x500000), None)
+    assert rc == -1
+
+
+def test_wait_drill_arguments():
+    assert bd.edit_attn_set_wait_drill(-1, 0) == -2
+    assert bd.edit_attn_set_wait_drill(1, 10) == -2            # limit below 1 us
+    assert bd.edit_attn_set_wait_drill(1, 3_000_000_000) == -2  # above the library's own 2 s
+    assert bd.edit_attn_set_wait_drill(1, 1_000_000) == 0
+    assert bd.edit_attn_set_wait_drill(0, 0) == 0
+
+
 def test_status_strings():
     assert bd.status_string(0) == "ok"
     assert bd.status_string(-7) == "device wait timed out"
@@ -133,6 +165,13 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     assert rc == -9 and bd.status_string(rc) == "request exceeds the library's fixed scratch"
     assert L.edit_linear_attention_noalloc(None, p(0x2000), p(0x3000), 1, 8, 4, 64, 2, 0, ctypes.c_float(1e-6),
                                            p(0x4000), None) == -1
+    # grid limits: more than 65535 images or heads is a shape error, not a failed launch
+    assert L.edit_linear_attention_noalloc(p(0x1000), p(0x2000), p(0x3000), 70000, 8, 4, 8, 2, 0,
+                                           ctypes.c_float(1e-6), p(0x4000), None) == -8
+    assert L.edit_linear_attention_noalloc(p(0x1000), p(0x2000), p(0x3000), 1, 8, 4, 70000, 70000, 0,
+                                           ctypes.c_float(1e-6), p(0x4000), None) == -8
+    assert L.edit_linear_attention_noalloc(p(0x1000), p(0x2000), p(0x3000), 1, 8, 4, 258, 1, 0,
+                                           ctypes.c_float(1e-6), p(0x4000), None) == -8   # d > 128
 
 
 def fake_variant(q="cf", k="sc", v="sc", proj=False, base=0x900000):

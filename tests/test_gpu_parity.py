@@ -265,15 +265,24 @@ def test_workload_px8192_sampled_rows():
 
 @pytest.mark.parametrize("name", ["px1024", "px4096"])
 def test_streams_serial_and_graph_paths_agree(name):
-    """The same layer through its three launch paths gives bit-identical
-    outputs: the default (K/V branch and weight folding on the library's side
-    stream), the serial order taken while stage events are recorded, and a
-    CUDA-graph capture of the default path replayed."""
+    """The same layer through its launch paths gives bit-identical outputs:
+    the default (K/V branch and weight folding on the side stream the layer
+    lends the library), no side stream (every kernel on the call's stream),
+    the serial order taken while stage events are recorded, and a CUDA-graph
+    capture of the default path replayed."""
     cfg = dict(WORKLOADS[name])
     d = make_inputs(**cfg)
     layer, x = gpu_layer(cfg, d)
     y0 = layer.forward(x).clone()
     torch.cuda.synchronize()
+    assert layer.side is not None
+    layer.set_side(None)
+    try:
+        ys = layer.forward(x).clone()
+    finally:
+        layer.set_side(layer.side)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, ys)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(bd.STAGE_EVENTS_EDIT)]
     for e in evs:
         e.record()

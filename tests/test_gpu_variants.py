@@ -65,6 +65,30 @@ def test_table_rows_px1024(qkv):
     print(qkv, check_variant(cfg, make_inputs(**cfg), qkv, qkv == ("cf", "sc", "sc")))
 
 
+@pytest.mark.parametrize("qkv", TABLE_ROWS, ids=lambda v: "-".join(v))
+def test_table_rows_px2048(qkv):
+    """The ablation table's four rows on the 16,384-token workload, the size
+    from which the plan takes the kernels the benchmark times at 65,536
+    tokens: the tap-reuse conv (W = 128), the 384-column ring GEMM (also for
+    the key ConvFusion's 2C-strided output and the output Linear) and the
+    uncompressed rows' operand transpose over 16,384 tokens."""
+    cfg = dict(WORKLOADS["px2048"], variant_weights=True)
+    print(qkv, check_variant(cfg, make_inputs(**cfg), qkv, qkv == ("cf", "sc", "sc")))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("qkv,proj", [(("cf", "none", "none"), False), (("cf", "cf", "none"), False),
+                                      (("cf", "sc", "sc"), True), (("none", "sc", "sc"), False)],
+                         ids=["cf-none-none", "cf-cf-none", "cf-sc-sc-proj", "none-sc-sc"])
+def test_table_rows_px4096_full_size(qkv, proj):
+    """The ablation rows at the size and in the launch configuration the
+    benchmark times them (65,536 tokens, 5% outlier tokens), every output
+    element and S, z against the oracle; the uncompressed rows sum over all
+    65,536 keys per head."""
+    cfg = dict(WORKLOADS["px4096"], variant_weights=True)
+    print(qkv, proj, check_variant(cfg, make_inputs(**cfg), qkv, proj))
+
+
 def test_default_variant_is_the_layer():
     cfg = dict(dtype="bf16", B=1, H=16, W=16, C=256, c_red=64, gn_groups=4, heads=4, seed=43, variant_weights=True)
     d = make_inputs(**cfg)
