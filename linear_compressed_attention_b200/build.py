@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 SRCS = [os.path.join(PKG, "csrc", "edit_attn.cu"), os.path.join(PKG, "csrc", "edit_noalloc.cu")]
 OUT = os.path.join(PKG, "libedit_attn.so")
 DEPS = [os.path.join(PKG, "csrc", f) for f in ("edit_attn.cu", "edit_noalloc.cu", "common.cuh", "tc_gemm.cuh",
-                                                "tc_conv.cuh", "simt_kernels.cuh", "sdpa_mma.cuh")]
+                                                "tc_conv.cuh", "simt_kernels.cuh", "sdpa_tc.cuh")]
 DEPS.append(os.path.join(ROOT, "include", "edit_attn.h"))
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -25,7 +25,7 @@
 #include <utility>
 
 #include "common.cuh"
-#include "sdpa_mma.cuh"
+#include "sdpa_tc.cuh"
 #include "simt_kernels.cuh"
 #include "tc_conv.cuh"
 #include "tc_gemm.cuh"
@@ -173,7 +173,7 @@ struct Plan {
   int kv_chunks;  // KV-state partials per (image, head)
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
-  int sdpa_split = 0;  // MM-EDiT prompt rows (bf16): ranges of the image keys per query tile, 0 = no split
+  int npv = 0, nkpI = 0, nkpP = 0;  // MM-EDiT (bf16): [V | 1]^T rows per head, image / prompt keys padded to 128
   bool fork = false;   // K/V branch on the calling thread's side stream, concurrent with the query branch
   int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
@@ -184,7 +184,7 @@ struct Plan {
   bool oproj = false;    // output Linear after the attention
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      fixpart, sdpapart, Y, total;
+      fixpart, VTi, VTp, Y, total;
 };
 
 int next_pow2(int v) {
@@ -328,17 +328,15 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
   pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
   pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
-  // MM-EDiT prompt rows walk all M image keys per query: when their query tiles
-  // fill less than two waves, split the image keys into ranges of about
-  // max(256, NT) keys (one more item takes the prompt keys) and merge after.
-  pl.sdpapart = 0;
+  // MM-EDiT softmax blocks (bf16): the image and prompt values as [V | 1]^T
+  // operands, [B][heads][npv][keys padded to 128]
+  pl.VTi = pl.VTp = 0;
   if (pl.bf16 && NT > 0) {
-    const long ctas = static_cast<long>(B) * heads * ((NT + 63) / 64);
-    const int span = NT > 256 ? NT : 256;
-    if (ctas < 2L * num_sms() && pl.M > span) {
-      pl.sdpa_split = (pl.M + span - 1) / span;
-      pl.sdpapart = take(static_cast<size_t>(B) * heads * NT * (pl.sdpa_split + 1) * (pl.d + 2) * 4);
-    }
+    pl.npv = pl.d + 1 <= 48 ? 48 : 80;
+    pl.nkpI = (pl.M + 127) / 128 * 128;
+    pl.nkpP = (NT + 127) / 128 * 128;
+    pl.VTi = take(static_cast<size_t>(B) * heads * pl.npv * pl.nkpI * 2);
+    pl.VTp = take(static_cast<size_t>(B) * heads * pl.npv * pl.nkpP * 2);
   }
   // fp32 halves of the conv tiles split in the last wave (tap-reuse conv only)
   pl.fixpart = (pl.bf16 && pl.TW == 128) ? take(static_cast<size_t>(kConvMaxSplit) * 4 * 128 * pl.Cr * 4) : 0;
@@ -1235,33 +1233,100 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
   return last_launch();
 }
 
-template <typename T, int D>
-int launch_sdpa(const SdpaParams& p, int B, cudaStream_t st) {
-  if (sizeof(T) == 2) {  // bf16: tensor-core flash-style kernel, 64 query rows per block
-    const int nitem = p.part ? p.nchunk1 + (p.n2 > 0 ? 1 : 0) : 1;
-    launch_pdl(sdpa_mma_kernel<D>, dim3(dim3(ceil_div(p.Nq, 64) * nitem, p.heads, B)), dim3(128), 0, st, p);
-    if (!p.part) return last_launch();
-    EDIT_TRY(last_launch());
-    launch_pdl(sdpa_combine_kernel, dim3(grid_for(static_cast<long>(B) * p.heads * p.Nq * 32, 256)), dim3(256), 0, st,
-               p);
-    return last_launch();
-  }
+template <int D>
+int launch_sdpa_simt(const SdpaParams& p, int B, cudaStream_t st) {
   const size_t smem = (128 * D + 128 * (D + 1)) * sizeof(float);
-  auto kern = sdpa_blend_kernel<T, D>;
+  auto kern = sdpa_blend_kernel<float, D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EDIT_ERR_CUDA;
   launch_pdl(kern, dim3(dim3(ceil_div(p.Nq, 128), p.heads, B)), dim3(128), smem, st, p);
   return last_launch();
 }
 
-template <typename T>
-int sdpa(const SdpaParams& p, int B, cudaStream_t st) {
+// fp32 softmax blocks on the CUDA cores.
+int sdpa_simt(const SdpaParams& p, int B, cudaStream_t st) {
   switch (p.d) {
-    case 32: return launch_sdpa<T, 32>(p, B, st);
-    case 64: return launch_sdpa<T, 64>(p, B, st);
-    case 72: return launch_sdpa<T, 72>(p, B, st);
+    case 32: return launch_sdpa_simt<32>(p, B, st);
+    case 64: return launch_sdpa_simt<64>(p, B, st);
+    case 72: return launch_sdpa_simt<72>(p, B, st);
   }
   return EDIT_ERR_UNSUPPORTED;
+}
+
+// One key set of a tensor-core softmax launch: K token-major (row stride ld
+// elements, n keys per image) and its [V | 1]^T operand (keys padded to nkp).
+struct SdpaSet {
+  const void* k;
+  long ld;
+  int n;
+  const void* vt;
+  int nkp;
+};
+
+// Token-major rows seen per head: [rows][heads][d] bf16, box 64 x 1 x 128
+// (columns past d, and rows past the end, read as zero).
+bool map_head_rows(CUtensorMap* m, const void* base, int d, int heads, long rows, long ld) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t st[2] = {(cuuint64_t)d * 2, (cuuint64_t)ld * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  return encode(m, 3, base, dims, st, box);
+}
+
+// bf16 softmax blocks on the tensor cores (sdpa_tc_kernel): one persistent
+// CTA per SM at most (512 TMEM columns, ~200 KB of shared memory each).
+template <int D>
+int launch_sdpa_tc(const void* q, long ldq, int Nq, const SdpaSet& s1, const SdpaSet* s2, SdpaTcParams p,
+                   const Plan& pl, cudaStream_t st) {
+  using Cfg = SdpaTcCfg<D>;
+  CUtensorMap mq, mk1, mv1, mk2, mv2;
+  const long B = pl.B, heads = pl.heads;
+  if (!map_head_rows(&mq, q, D, pl.heads, B * Nq, ldq) || !map_head_rows(&mk1, s1.k, D, pl.heads, B * s1.n, s1.ld) ||
+      !map_b(&mv1, s1.vt, s1.nkp, B * heads * Cfg::NPV, s1.nkp, Cfg::NPV))
+    return EDIT_ERR_CUDA;
+  if (s2) {
+    if (!map_head_rows(&mk2, s2->k, D, pl.heads, B * s2->n, s2->ld) ||
+        !map_b(&mv2, s2->vt, s2->nkp, B * heads * Cfg::NPV, s2->nkp, Cfg::NPV))
+      return EDIT_ERR_CUDA;
+  } else {
+    mk2 = mk1;
+    mv2 = mv1;
+  }
+  p.Nq = Nq;
+  p.heads = pl.heads;
+  p.nimg = pl.B;
+  p.n1 = s1.n;
+  p.n2 = s2 ? s2->n : 0;
+  auto kern = sdpa_tc_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+    return EDIT_ERR_CUDA;
+  const long items = B * heads * ceil_div(Nq, 128);
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  launch_pdl(kern, dim3(grid), dim3(192), Cfg::SMEM_BYTES, st, mq, mk1, mv1, mk2, mv2, p);
+  return last_launch();
+}
+
+int sdpa_tc(const void* q, long ldq, int Nq, const SdpaSet& s1, const SdpaSet* s2, const SdpaTcParams& p,
+            const Plan& pl, cudaStream_t st) {
+  switch (pl.d) {
+    case 32: return launch_sdpa_tc<32>(q, ldq, Nq, s1, s2, p, pl, st);
+    case 64: return launch_sdpa_tc<64>(q, ldq, Nq, s1, s2, p, pl, st);
+    case 72: return launch_sdpa_tc<72>(q, ldq, Nq, s1, s2, p, pl, st);
+  }
+  return EDIT_ERR_UNSUPPORTED;
+}
+
+// [V | 1]^T of one key set (vt_ones_kernel), keys padded to nkp.
+int vt_ones(const void* v, long ldv, int n, int nkp, const Plan& pl, void* vt, cudaStream_t st) {
+  const dim3 grid(nkp / 64, pl.heads, pl.B);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  auto* out = static_cast<__nv_bfloat16*>(vt);
+  switch (pl.d) {
+    case 32: launch_pdl(vt_ones_kernel<32, 48>, grid, dim3(256), 0, st, vb, ldv, n, nkp, pl.heads, out); break;
+    case 64: launch_pdl(vt_ones_kernel<64, 80>, grid, dim3(256), 0, st, vb, ldv, n, nkp, pl.heads, out); break;
+    case 72: launch_pdl(vt_ones_kernel<72, 80>, grid, dim3(256), 0, st, vb, ldv, n, nkp, pl.heads, out); break;
+    default: return EDIT_ERR_UNSUPPORTED;
+  }
+  return last_launch();
 }
 
 // MM-EDiT, prompt side: the prompt projections [Q_P | K_P | V_P] (stage 9).
@@ -1271,10 +1336,16 @@ int mm_project(const void* x_txt, const Plan& pl, const mmedit_weights* w, uint8
   const long trow = static_cast<long>(pl.B) * pl.NT;
   const void* wts[3] = {w->tq_w, w->tk_w, w->tv_w};
   const void* bs[3] = {w->tq_b, w->tk_b, w->tv_b};
-  if (pl.bf16)
+  if (pl.bf16) {
     EDIT_TRY(tc_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, 3L * pl.C, 0, status, st));
-  else
+    // [V | 1]^T operands of the softmax blocks: prompt values, then the image's
+    // compressed values (token-major V, written by the K/V branch)
+    const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
+    EDIT_TRY(vt_ones(qkv + 2 * pl.C, 3L * pl.C, pl.NT, pl.nkpP, pl, ws + pl.VTp, st));
+    EDIT_TRY(vt_ones(ws + pl.V, pl.C, pl.M, pl.nkpI, pl, ws + pl.VTi, st));
+  } else {
     EDIT_TRY(simt_linear(x_txt, trow, pl.C, wts, bs, 3, pl.C, ws + pl.QKVt, 3 * pl.C, 0, st));
+  }
   stage_mark(9, st);
   return EDIT_OK;
 }
@@ -1287,23 +1358,36 @@ template <typename T>
 int mm_image_rows(const Plan& pl, uint8_t* ws, void* out_img, cudaStream_t st) {
   const double eta = mm_eta(pl);
   const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
-  SdpaParams a;
-  std::memset(&a, 0, sizeof(a));
-  a.q = ws + pl.Q;
-  a.ldq = pl.C;
-  a.k1 = qkv + pl.C;
-  a.v1 = qkv + 2 * pl.C;
-  a.ld1 = 3L * pl.C;
-  a.n1 = pl.NT;
-  a.out = out_img;
-  a.ldo = pl.C;
-  a.Nq = static_cast<int>(pl.HW);
-  a.heads = pl.heads;
-  a.d = pl.d;
-  a.w0 = static_cast<float>(eta);
-  a.w1 = static_cast<float>(1.0 - eta);
-  a.blend_in = 1;
-  EDIT_TRY(sdpa<T>(a, pl.B, st));
+  if (pl.bf16) {
+    SdpaTcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.w0 = static_cast<float>(eta);
+    p.w1 = static_cast<float>(1.0 - eta);
+    p.blend_in = 1;
+    p.out = out_img;
+    p.ldo = pl.C;
+    p.status = reinterpret_cast<int*>(ws + pl.status);
+    const SdpaSet prompt = {qkv + pl.C, 3L * pl.C, pl.NT, ws + pl.VTp, pl.nkpP};
+    EDIT_TRY(sdpa_tc(ws + pl.Q, pl.C, static_cast<int>(pl.HW), prompt, nullptr, p, pl, st));
+  } else {
+    SdpaParams a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = ws + pl.Q;
+    a.ldq = pl.C;
+    a.k1 = qkv + pl.C;
+    a.v1 = qkv + 2 * pl.C;
+    a.ld1 = 3L * pl.C;
+    a.n1 = pl.NT;
+    a.out = out_img;
+    a.ldo = pl.C;
+    a.Nq = static_cast<int>(pl.HW);
+    a.heads = pl.heads;
+    a.d = pl.d;
+    a.w0 = static_cast<float>(eta);
+    a.w1 = static_cast<float>(1.0 - eta);
+    a.blend_in = 1;
+    EDIT_TRY(sdpa_simt(a, pl.B, st));
+  }
   stage_mark(10, st);
   return EDIT_OK;
 }
@@ -1313,31 +1397,39 @@ template <typename T>
 int mm_prompt_rows(const Plan& pl, uint8_t* ws, void* out_txt, cudaStream_t st) {
   const double eta = mm_eta(pl);
   const T* qkv = reinterpret_cast<const T*>(ws + pl.QKVt);
-  SdpaParams t;
-  std::memset(&t, 0, sizeof(t));
-  t.q = qkv;
-  t.ldq = 3L * pl.C;
-  t.k1 = ws + pl.K;
-  t.v1 = ws + pl.V;
-  t.ld1 = pl.C;
-  t.n1 = pl.M;
-  t.k2 = qkv + pl.C;
-  t.v2 = qkv + 2 * pl.C;
-  t.ld2 = 3L * pl.C;
-  t.n2 = pl.NT;
-  t.out = out_txt;
-  t.ldo = pl.C;
-  t.Nq = pl.NT;
-  t.heads = pl.heads;
-  t.d = pl.d;
-  t.w1 = static_cast<float>(eta);
-  t.w2 = static_cast<float>(1.0 - eta);
-  if (pl.sdpa_split > 0) {
-    t.nchunk1 = pl.sdpa_split;
-    t.nimg = pl.B;
-    t.part = reinterpret_cast<float*>(ws + pl.sdpapart);
+  if (pl.bf16) {
+    SdpaTcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.w1 = static_cast<float>(eta);
+    p.w2 = static_cast<float>(1.0 - eta);
+    p.out = out_txt;
+    p.ldo = pl.C;
+    p.status = reinterpret_cast<int*>(ws + pl.status);
+    const SdpaSet image = {ws + pl.K, pl.C, pl.M, ws + pl.VTi, pl.nkpI};
+    const SdpaSet prompt = {qkv + pl.C, 3L * pl.C, pl.NT, ws + pl.VTp, pl.nkpP};
+    EDIT_TRY(sdpa_tc(qkv, 3L * pl.C, pl.NT, image, &prompt, p, pl, st));
+  } else {
+    SdpaParams t;
+    std::memset(&t, 0, sizeof(t));
+    t.q = qkv;
+    t.ldq = 3L * pl.C;
+    t.k1 = ws + pl.K;
+    t.v1 = ws + pl.V;
+    t.ld1 = pl.C;
+    t.n1 = pl.M;
+    t.k2 = qkv + pl.C;
+    t.v2 = qkv + 2 * pl.C;
+    t.ld2 = 3L * pl.C;
+    t.n2 = pl.NT;
+    t.out = out_txt;
+    t.ldo = pl.C;
+    t.Nq = pl.NT;
+    t.heads = pl.heads;
+    t.d = pl.d;
+    t.w1 = static_cast<float>(eta);
+    t.w2 = static_cast<float>(1.0 - eta);
+    EDIT_TRY(sdpa_simt(t, pl.B, st));
   }
-  EDIT_TRY(sdpa<T>(t, pl.B, st));
   stage_mark(11, st);
   return EDIT_OK;
 }

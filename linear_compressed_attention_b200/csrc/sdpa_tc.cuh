@@ -1,0 +1,435 @@
+// Softmax attention blocks of MM-EDiT (section "MM-EDiT", eq. (A^Hybrid)) on
+// the 5th-generation tensor cores (tcgen05, accumulators in TMEM, operands
+// staged by TMA), bf16 in, fp32 accumulate:
+//
+//   out = [w0 * out] + sum_s w_s * softmax(q K_s^T / sqrt(d)) V_s
+//
+// over one or two key sets s, each normalised over its own keys.
+//
+// Work item: 128 query rows of one (image, head). A persistent CTA takes items
+// i, i + gridDim.x, ... and streams every key set of an item through one
+// pipeline in tiles of 128 keys; the tile sequence runs on across items.
+//   warp 0   TMA producer: the item's Q tile (once), then per key tile the K
+//            rows (token-major, K-major operand) and the V^T rows (channel-
+//            major with a ones row, K-major operand) into a STAGES-deep ring.
+//   warp 1   TMEM owner and MMA issuer: S_g = Q K_g^T (M = 128, N = 128) into
+//            one of two TMEM S buffers; then, for the previous tile,
+//            O_g = P_g [V_g | 1]^T (M = 128, N = NPV) into one of two TMEM O
+//            buffers. Column d of O is the row sum of P (the ones row of V^T),
+//            so numerator and denominator come from the same bf16 P.
+//   warps 2-5 softmax, one thread per query row (its TMEM lane): the row max
+//            of the tile (first pass over S), P = exp2(S c - m) rounded to bf16
+//            and written to shared memory as the K-major A operand of the
+//            second product (128-byte swizzle, second pass over S); then the
+//            running accumulator R = R 2^(m_prev - m) + O of the previous tile
+//            (deferred by one tile so that the next tile's exponentials overlap
+//            the product), R / R[d] at the end of a key set, and the blended
+//            output row at the end of the item.
+// Keys past the set's end (the zero-filled or next-image rows of a tile) get
+// P = 0. Every wait is bounded (EDIT_ERR_TIMEOUT in the status word).
+#pragma once
+
+#include "common.cuh"
+
+namespace edit {
+
+struct SdpaTcParams {
+  int Nq, heads, nimg;
+  int n1, n2;          // keys of the two sets (n2 = 0: one set)
+  float w0, w1, w2;    // out = [w0 * out] + w1 A_1 + w2 A_2
+  int blend_in;
+  void* out;
+  long ldo;
+  int* status;
+};
+
+template <int D>
+struct SdpaTcCfg {
+  static_assert(D == 32 || D == 64 || D == 72, "head width");
+  static constexpr int NBX = (D + 63) / 64;          // 64-column boxes of a Q / K row
+  static constexpr int KS = (D + 15) / 16;           // k-steps of q . k
+  static constexpr int NPV = (D + 1 <= 48) ? 48 : 80;  // [V | 1] rows: MMA N of the second product
+  static constexpr int STAGES = (D == 72) ? 2 : 3;
+  static constexpr int QB = (D == 72) ? 1 : 2;       // Q tile buffers
+  static constexpr int QBOX = 128 * 128;             // one 128-row x 128-byte box
+  static constexpr int Q_BYTES = QB * NBX * QBOX;
+  static constexpr int K_BYTES = STAGES * NBX * QBOX;
+  static constexpr int VBOX = NPV * 128;             // NPV rows x 64 keys
+  static constexpr int V_BYTES = STAGES * 2 * VBOX;
+  static constexpr int P_BYTES = 2 * 2 * QBOX;       // two P buffers of 128 rows x 128 keys
+  static constexpr int BAR_BYTES = (2 * QB + 2 * STAGES + 10) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + K_BYTES + V_BYTES + P_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128);
+  static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, NPV);
+  static constexpr int TMEM_COLS = 512;  // S buffers at 0, 128; O buffers at 256, 384
+};
+
+// 32 lanes x 32 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
+      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__ CUtensorMap mq,
+                                                         const __grid_constant__ CUtensorMap mk1,
+                                                         const __grid_constant__ CUtensorMap mv1,
+                                                         const __grid_constant__ CUtensorMap mk2,
+                                                         const __grid_constant__ CUtensorMap mv2,
+                                                         const SdpaTcParams p) {
+  using Cfg = SdpaTcCfg<D>;
+  constexpr int NBX = Cfg::NBX, KS = Cfg::KS, NPV = Cfg::NPV, STAGES = Cfg::STAGES, QB = Cfg::QB;
+  constexpr int QBOX = Cfg::QBOX, VBOX = Cfg::VBOX;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sQ = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = sQ + Cfg::Q_BYTES;
+  uint8_t* sV = sK + Cfg::K_BYTES;
+  uint8_t* sP = sV + Cfg::V_BYTES;
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + Cfg::P_BYTES);
+  uint64_t* q_empty = q_full + QB;
+  uint64_t* kv_full = q_empty + QB;
+  uint64_t* kv_empty = kv_full + STAGES;
+  uint64_t* s_full = kv_empty + STAGES;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_empty = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < QB; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);  // one arrival per softmax warp
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk1);
+    tma_prefetch_desc(&mv1);
+    if (p.n2 > 0) {
+      tma_prefetch_desc(&mk2);
+      tma_prefetch_desc(&mv2);
+    }
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+
+  const int qtiles = (p.Nq + 127) / 128;
+  const long nitems = static_cast<long>(p.nimg) * p.heads * qtiles;
+  const int T1 = (p.n1 + 127) / 128, T2 = (p.n2 + 127) / 128, T = T1 + T2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      long g = 0;
+      int li = 0;
+      bool ok = true;
+      for (long it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+        const int qt = static_cast<int>(it % qtiles);
+        const long bh = it / qtiles;
+        const int h = static_cast<int>(bh % p.heads), b = static_cast<int>(bh / p.heads);
+        const int qb = li % QB;
+        if (!mbar_wait(&q_empty[qb], ((li / QB) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&q_full[qb], NBX * QBOX);
+#pragma unroll
+        for (int bx = 0; bx < NBX; ++bx)
+          tma_load_3d(&mq, &q_full[qb], sQ + (qb * NBX + bx) * QBOX, 64 * bx, h, b * p.Nq + qt * 128);
+        for (int t = 0; t < T; ++t, ++g) {
+          const bool one = t < T1;
+          const int tt = one ? t : t - T1;
+          const int n = one ? p.n1 : p.n2;
+          const int st = static_cast<int>(g % STAGES);
+          if (!mbar_wait(&kv_empty[st], static_cast<uint32_t>((g / STAGES) & 1) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[st], NBX * QBOX + 2 * VBOX);
+#pragma unroll
+          for (int bx = 0; bx < NBX; ++bx)
+            tma_load_3d(one ? &mk1 : &mk2, &kv_full[st], sK + (st * NBX + bx) * QBOX, 64 * bx, h, b * n + tt * 128);
+#pragma unroll
+          for (int kx = 0; kx < 2; ++kx)
+            tma_load_2d(one ? &mv1 : &mv2, &kv_full[st], sV + (st * 2 + kx) * VBOX, tt * 128 + 64 * kx,
+                        (b * p.heads + h) * NPV);
+        }
+      }
+      if (*abort_flag) {  // let copies already issued land before the block exits
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      long g = 0;
+      int li = 0;
+      bool ok = true;
+      // O_gg = P_gg [V_gg | 1]^T for a tile whose P the softmax warps have written
+      auto issue_pv = [&](long gg) -> bool {
+        const int ob = static_cast<int>(gg & 1);
+        const uint32_t ph = static_cast<uint32_t>((gg >> 1) & 1);
+        if (!mbar_wait(&p_full[ob], ph, abort_flag, p.status)) return false;
+        if (!mbar_wait(&o_empty[ob], ph ^ 1u, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const int st = static_cast<int>(gg % STAGES);
+        const uint32_t pa = smem_u32(sP + ob * 2 * QBOX), va = smem_u32(sV + st * 2 * VBOX);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t ad = sdesc_kmajor_sw128(pa + (s >> 2) * QBOX + (s & 3) * 32);
+          const uint64_t bd = sdesc_kmajor_sw128(va + (s >> 2) * VBOX + (s & 3) * 32);
+          umma_bf16(tmem_base + 256 + 128 * ob, ad, bd, Cfg::IDESC_O, s > 0 ? 1u : 0u);
+        }
+        umma_commit(&o_full[ob]);
+        umma_commit(&kv_empty[st]);
+        return true;
+      };
+      for (long it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+        const int qb = li % QB;
+        if (!mbar_wait(&q_full[qb], (li / QB) & 1, abort_flag, p.status)) break;
+        const uint32_t qa = smem_u32(sQ + qb * NBX * QBOX);
+        for (int t = 0; t < T; ++t, ++g) {
+          const int st = static_cast<int>(g % STAGES);
+          const int sb = static_cast<int>(g & 1);
+          if (!mbar_wait(&kv_full[st], static_cast<uint32_t>((g / STAGES) & 1), abort_flag, p.status) ||
+              !mbar_wait(&s_empty[sb], static_cast<uint32_t>((g >> 1) & 1) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sK + st * NBX * QBOX);
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(qa + (kk >> 2) * QBOX + (kk & 3) * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(ka + (kk >> 2) * QBOX + (kk & 3) * 32);
+            umma_bf16(tmem_base + 128 * sb, ad, bd, Cfg::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[sb]);
+          if (t == T - 1) umma_commit(&q_empty[qb]);  // the item's last reads of its Q tile
+          if (g > 0 && !issue_pv(g - 1)) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (ok && g > 0) issue_pv(g - 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / output
+    const int q4 = warp & 3;  // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16);
+    const float c = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e): exp2 below
+    const uint32_t prow = static_cast<uint32_t>(row) * 128u;
+    const uint32_t psw = static_cast<uint32_t>(row & 7);
+    long g = 0;
+    bool ok = true;
+    float R[D + 1];
+    float acc[D];
+    for (long it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int qt = static_cast<int>(it % qtiles);
+      const long bh = it / qtiles;
+      const int h = static_cast<int>(bh % p.heads), b = static_cast<int>(bh / p.heads);
+#pragma unroll
+      for (int i = 0; i < D; ++i) acc[i] = 0.f;
+      for (int set = 0; set < 2 && ok; ++set) {
+        const int n = set == 0 ? p.n1 : p.n2;
+        const int Ts = set == 0 ? T1 : T2;
+        if (Ts == 0) continue;
+#pragma unroll
+        for (int i = 0; i <= D; ++i) R[i] = 0.f;
+        float m_run = -INFINITY, m_acc = -INFINITY, m_pend = -INFINITY;
+        // R = R 2^(m_acc - m_j) + O_j for tile gg whose P used the max m_j
+        auto accumulate = [&](long gg, float m_j) -> bool {
+          const int ob = static_cast<int>(gg & 1);
+          if (!warp_wait(&o_full[ob], static_cast<uint32_t>((gg >> 1) & 1), abort_flag, p.status)) return false;
+          tc_fence_after();
+          const float alpha = exp2f(m_acc - m_j);
+          m_acc = m_j;
+#pragma unroll
+          for (int ch = 0; ch < (D + 16) / 16; ++ch) {
+            float v[16];
+            tmem_ld16(t_lane + 256 + 128 * ob + 16 * ch, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (16 * ch + i <= D) R[16 * ch + i] = fmaf(R[16 * ch + i], alpha, v[i]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[ob]);
+          return true;
+        };
+        for (int tt = 0; tt < Ts; ++tt, ++g) {
+          const int sb = static_cast<int>(g & 1);
+          if (!warp_wait(&s_full[sb], static_cast<uint32_t>((g >> 1) & 1), abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nvalid = n - tt * 128 < 128 ? n - tt * 128 : 128;
+          // pass 1: the tile's row max over its valid keys
+          float mt = -INFINITY;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            if (32 * ch < nvalid) {
+              float v[32];
+              tmem_ld32(t_lane + 128 * sb + 32 * ch, v);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (32 * ch + i < nvalid) mt = fmaxf(mt, v[i]);
+            }
+          }
+          const float m_new = fmaxf(m_run, mt * c);
+          m_run = m_new;
+          // pass 2: P = 2^(S c - m) in bf16, 128-byte-swizzled K-major rows
+          uint8_t* pb = sP + sb * 2 * QBOX;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            float v[32];
+            if (32 * ch < nvalid) tmem_ld32(t_lane + 128 * sb + 32 * ch, v);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float e[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int key = 32 * ch + 8 * q8 + i;
+                e[i] = key < nvalid ? exp2f(fmaf(v[8 * q8 + i], c, -m_new)) : 0.f;
+              }
+              uint4 w;
+              w.x = pack_bf16x2(e[0], e[1]);
+              w.y = pack_bf16x2(e[2], e[3]);
+              w.z = pack_bf16x2(e[4], e[5]);
+              w.w = pack_bf16x2(e[6], e[7]);
+              const int key0 = 32 * ch + 8 * q8;               // first key of this 16-byte chunk
+              const uint32_t chunk = static_cast<uint32_t>((key0 & 63) >> 3);
+              *reinterpret_cast<uint4*>(pb + (key0 >> 6) * QBOX + prow + ((chunk ^ psw) << 4)) = w;
+            }
+          }
+          fence_proxy_async_smem();  // P is read by the tensor cores (async proxy)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&s_empty[sb]);
+            mbar_arrive(&p_full[sb]);
+          }
+          if (tt > 0 && !accumulate(g - 1, m_pend)) {
+            ok = false;
+            break;
+          }
+          m_pend = m_new;
+          if (tt == Ts - 1 && !accumulate(g, m_new)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        const float w = set == 0 ? p.w1 : p.w2;
+        const float sc = R[D] > 0.f ? w / R[D] : 0.f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) acc[i] = fmaf(R[i], sc, acc[i]);
+      }
+      if (!ok) break;
+      const int r = qt * 128 + row;
+      if (r < p.Nq) {
+        __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D;
+#pragma unroll
+        for (int c8 = 0; c8 < D; c8 += 8) {
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = acc[c8 + i];
+          if (p.blend_in) {
+            const uint4 old = *reinterpret_cast<const uint4*>(og + c8);
+            const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              o[2 * i] = fmaf(p.w0, __uint_as_float(ow[i] << 16), o[2 * i]);
+              o[2 * i + 1] = fmaf(p.w0, __uint_as_float(ow[i] & 0xffff0000u), o[2 * i + 1]);
+            }
+          }
+          uint4 wv;
+          wv.x = pack_bf16x2(o[0], o[1]);
+          wv.y = pack_bf16x2(o[2], o[3]);
+          wv.z = pack_bf16x2(o[4], o[5]);
+          wv.w = pack_bf16x2(o[6], o[7]);
+          *reinterpret_cast<uint4*>(og + c8) = wv;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// [V | 1]^T operand of the softmax blocks: VT[b][h][c][j] = V[b][j][h d + c]
+// for c < d, row d = 1 for the set's n keys, every other row and every key
+// j >= n zero; rows NPV per head, keys padded to nkp (a multiple of 128).
+// One block per (64 keys, head, image): the 64 token rows are read with
+// 16-byte loads into shared memory and written out transposed, 16 bytes per
+// thread.
+template <int D, int NPV>
+__global__ void __launch_bounds__(256) vt_ones_kernel(const __nv_bfloat16* __restrict__ V, long ldv, int n, int nkp,
+                                                     int heads, __nv_bfloat16* __restrict__ VT) {
+  pdl_wait();
+  __shared__ __align__(16) __nv_bfloat16 tile[64][D + 8];
+  const int j0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z;
+  for (int e = threadIdx.x; e < 64 * (D / 8); e += blockDim.x) {
+    const int r = e / (D / 8), c8 = (e - r * (D / 8)) * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j0 + r < n) v = *reinterpret_cast<const uint4*>(V + (static_cast<long>(b) * n + j0 + r) * ldv + h * D + c8);
+    *reinterpret_cast<uint4*>(&tile[r][c8]) = v;
+  }
+  __syncthreads();
+  const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
+  for (int e = threadIdx.x; e < NPV * 8; e += blockDim.x) {
+    const int c = e >> 3, k8 = (e & 7) * 8;
+    __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = j0 + k8 + i < n;
+      o[i] = c < D ? (in ? tile[k8 + i][c] : zero) : (c == D && in ? one : zero);
+    }
+    *reinterpret_cast<uint4*>(VT + ((static_cast<long>(b) * heads + h) * NPV + c) * nkp + j0 + k8) =
+        *reinterpret_cast<const uint4*>(o);
+  }
+}
+
+}  // namespace edit

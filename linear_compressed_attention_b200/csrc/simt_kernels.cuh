@@ -6,9 +6,29 @@
 #pragma once
 
 #include "common.cuh"
-#include "sdpa_mma.cuh"  // SdpaParams
 
 namespace edit {
+
+// Parameters of one softmax-attention launch of the CUDA-core path (fp32),
+// token-major operands: out = [w0 * out] + w1 softmax(q k1^T / sqrt(d)) v1
+// (+ w2 softmax(q k2^T / sqrt(d)) v2 when n2 > 0).
+struct SdpaParams {
+  const void* q;
+  long ldq;
+  const void* k1;
+  const void* v1;
+  long ld1;
+  int n1;
+  const void* k2;
+  const void* v2;
+  long ld2;
+  int n2;
+  void* out;
+  long ldo;
+  int Nq, heads, d;
+  float w0, w1, w2;
+  int blend_in;
+};
 namespace {  // internal linkage: each translation unit that uses these keeps its own copy
 
 // ====================================================================== GEMM
