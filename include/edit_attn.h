@@ -249,6 +249,55 @@ EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, c
 EDIT_API int edit_attn_variant_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
                                                 const edit_attn_variant *v, edit_ws_layout *layout);
 
+/* Row bands: one image split over several ranks (sequence parallelism).
+ *
+ * The notes page scales EDiT to 8192 x 8192 images (section 延迟分析, the
+ * latency table); one such layer is 262,144 tokens. Its only global steps are
+ * two reductions: the GroupNorm statistics of U = Conv3x3(X) (eq. (Q^EDiT))
+ * and the per-head sums S = sum_j K_j^T V_j, z = sum_j K_j of eq. (y_i).
+ * Everything else reads at most a 3 x 3 neighbourhood of a pixel. So the rows
+ * of one image can be split into bands, one per rank:
+ *   1. each rank takes its band of x plus one halo row above and one below
+ *      from its neighbours (none at the image borders) and calls
+ *      edit_attn_band_partials, which writes the band's record of partial
+ *      sums;
+ *   2. the ranks all-gather the records, in band order;
+ *   3. each rank calls edit_attn_band_finish with all records, which sums them
+ *      in band order (so every rank forms the same totals) and writes the
+ *      band's rows of out.
+ * Shapes and rules:
+ *   band   rows [row0, row0 + rows) of an image of H rows: row0 even, and
+ *          row0 + rows even unless it equals H, so that no stride-2 key/value
+ *          token straddles two bands.
+ *   x_ext  [rows + top + bottom][W][C]: the band with its halo rows, top = 1
+ *          when row0 > 0, bottom = 1 when row0 + rows < H (else 0).
+ *   record device buffer of edit_attn_band_record_bytes, 256-byte aligned:
+ *          fp64 GroupNorm sums [gn_groups][2] (sum, sum of squares of the
+ *          band's U), then, at the next 256-byte boundary, the band's fp32
+ *          [S | z] [heads][d][d + 1].
+ *   records the records of all nrecords bands, in band order, each
+ *          edit_attn_band_record_bytes apart (256-byte aligned).
+ *   out    [rows][W][C]: the band's rows of the layer output.
+ * bf16 only (EDIT_ERR_UNSUPPORTED for fp32), one image. The workspace
+ * (w->workspace, at least edit_attn_band_workspace_bytes) carries the band's
+ * intermediates from the first call to the second: pass the same band, x_ext
+ * and workspace to both, on the same stream. Errors as for edit_attn_forward;
+ * a band that breaks the rules above is EDIT_ERR_SHAPE. */
+typedef struct {
+  int H;    /* rows of the whole image */
+  int row0; /* first row of this band */
+  int rows; /* rows of this band */
+} edit_band;
+
+EDIT_API size_t edit_attn_band_workspace_bytes(int W, int C, int heads, const edit_band *band,
+                                               const edit_attn_weights *w);
+EDIT_API size_t edit_attn_band_record_bytes(int C, int heads, const edit_attn_weights *w);
+EDIT_API int edit_attn_band_partials(const void *x_ext, int W, int C, int heads, const edit_band *band,
+                                     const edit_attn_weights *w, void *record, void *stream);
+EDIT_API int edit_attn_band_finish(const void *x_ext, int W, int C, int heads, const edit_band *band,
+                                   const edit_attn_weights *w, const void *records, int nrecords, void *out,
+                                   void *stream);
+
 /* Measurement hooks (no counterpart on the page; used by the benchmark).
  *
  * edit_attn_set_stage_events: when `events` is non-NULL, the next forward

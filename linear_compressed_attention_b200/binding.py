@@ -23,7 +23,8 @@ EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_b
            "edit_attn_read_status", "edit_status_string", "edit_attn_workspace_layout",
            "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc",
            "edit_attn_variant_workspace_bytes", "edit_attn_variant_forward", "edit_attn_variant_workspace_layout",
-           "edit_attn_set_wait_drill")
+           "edit_attn_set_wait_drill", "edit_attn_band_workspace_bytes", "edit_attn_band_record_bytes",
+           "edit_attn_band_partials", "edit_attn_band_finish")
 STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
 PROC = {"none": 0, "cf": 1, "sc": 2}
 VARIANT_NAMES = ("kcf3_w", "kcf3_b", "kgn_gamma", "kgn_beta", "kcf1_w", "kcf1_b", "o_w", "o_b")

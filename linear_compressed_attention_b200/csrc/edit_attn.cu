@@ -613,7 +613,6 @@ int gemm_conv_reuse(TcGemmParams& p, int cr, cudaStream_t st, bool* split) {
 }
 
 // Box rows of a B map = the MMA N of one instruction (half of it per CTA in a pair).
-int linear_chunk(int bn) { return bn; }
 int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
 
 // Linear GEMMs on CTA pairs: 256 x 256 pair tiles (one N = 256 MMA per
@@ -752,6 +751,77 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
 // Spatial Compressor (the EDiT layer) K = ReLU(DW(Linear_K(X))), V = DW(Linear_V(X));
 // without it the keys and values keep all N tokens: K = ReLU(Linear_K(X)) or the
 // key's own ConvFusion feature map, V = Linear_V(X).
+// Per-head partial [S | z] sums of the channel-major K, V operands (KT, VTx)
+// over chunks of tokens: tensor-core GEMM Kᵀ [V | 1] into kvpart.
+int kv_state_tc(const Plan& pl, uint8_t* ws, cudaStream_t st) {
+  const __nv_bfloat16* KT = reinterpret_cast<const __nv_bfloat16*>(ws + pl.KT);
+  const __nv_bfloat16* VTx = reinterpret_cast<const __nv_bfloat16*>(ws + pl.VTx);
+  TcGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!map_a(&p.a0, KT, pl.Mp, static_cast<long>(pl.B) * pl.C, 1, pl.Mp, static_cast<long>(pl.B) * pl.C * pl.Mp))
+    return EDIT_ERR_CUDA;
+  p.a1 = p.a0;
+  if (!map_b(&p.b0, VTx, pl.Mp, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.Mp, pl.NP)) return EDIT_ERR_CUDA;
+  p.b1 = p.b2 = p.bk = p.b0;
+  p.num_kb = (pl.Mp + 63) / 64;
+  p.kb_split = p.num_kb;
+  p.kb_per_chunk = pl.kv_kb;
+  p.num_chunks = pl.kv_chunks;
+  p.num_m_tiles = pl.kv_chunks;
+  p.num_tiles = pl.B * pl.heads * pl.kv_chunks;
+  p.num_n_tiles = 1;
+  p.n_split = pl.NP;
+  p.N = pl.NP;
+  p.d = pl.d;
+  p.heads = pl.heads;
+  p.kv_rows_per_img = pl.C;
+  p.kv_part = reinterpret_cast<float*>(ws + pl.kvpart);
+  p.status = reinterpret_cast<int*>(ws + pl.status);
+  return gemm_kvstate(p, pl.NP, st);
+}
+
+// Depthwise stride-2 conv of the token-major K'|V' rows (an image of `rows`
+// rows, the first `row_shift` of them a halo above the output rows) into the
+// channel-major KT, VTx operands (and token-major K, V when the plan keeps
+// them): output row i reads K'|V' rows 2i - 1 + row_shift .. 2i + 1 + row_shift.
+int dwconv_tc(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, int rows, int row_shift, cudaStream_t st) {
+  __nv_bfloat16* KT = reinterpret_cast<__nv_bfloat16*>(ws + pl.KT);
+  __nv_bfloat16* VTx = reinterpret_cast<__nv_bfloat16*>(ws + pl.VTx);
+  DwTmaMaps mp;
+  std::memset(&mp, 0, sizeof(mp));
+  const long C2 = 2L * pl.C;
+  cuuint64_t d_in[4] = {(cuuint64_t)C2, (cuuint64_t)pl.W, (cuuint64_t)rows, (cuuint64_t)pl.B};
+  cuuint64_t s_in[3] = {(cuuint64_t)C2 * 2, (cuuint64_t)pl.W * C2 * 2, (cuuint64_t)rows * pl.W * C2 * 2};
+  cuuint32_t b_in[4] = {64, 65, 3, 1};
+  cuuint64_t d_kt[2] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.B * pl.C};
+  cuuint64_t s_kt[1] = {(cuuint64_t)pl.Mp * 2};
+  cuuint32_t b_kt[2] = {32, 64};
+  cuuint64_t d_vt[3] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.NP, (cuuint64_t)pl.B * pl.heads};
+  cuuint64_t s_vt[2] = {(cuuint64_t)pl.Mp * 2, (cuuint64_t)pl.NP * pl.Mp * 2};
+  cuuint32_t b_vt[3] = {32, 8, 1};
+  if (!encode(&mp.in, 4, ws + pl.KVp, d_in, s_in, b_in, SWZ_NONE) ||
+      !encode(&mp.kt, 2, KT, d_kt, s_kt, b_kt, SWZ_64) || !encode(&mp.vtx, 3, VTx, d_vt, s_vt, b_vt, SWZ_64))
+    return EDIT_ERR_CUDA;
+  const int tokmajor = pl.K ? 1 : 0;
+  if (tokmajor) {
+    cuuint64_t d_t[4] = {(cuuint64_t)pl.C, (cuuint64_t)pl.Wo, (cuuint64_t)pl.Ho, (cuuint64_t)pl.B};
+    cuuint64_t s_t[3] = {(cuuint64_t)pl.C * 2, (cuuint64_t)pl.Wo * pl.C * 2, (cuuint64_t)pl.Ho * pl.Wo * pl.C * 2};
+    cuuint32_t b_t[4] = {64, 32, 1, 1};
+    if (!encode(&mp.ktok, 4, ws + pl.K, d_t, s_t, b_t, SWZ_NONE) ||
+        !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
+      return EDIT_ERR_CUDA;
+  }
+  launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, mp, rows,
+             pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
+             static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
+             static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, row_shift, reinterpret_cast<int*>(ws + pl.status));
+  EDIT_TRY(last_launch());
+  const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
+  launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP,
+             pl.Mp);
+  return last_launch();
+}
+
 template <typename T>
 int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit_attn_variant* var, uint8_t* ws,
            cudaStream_t st, cudaEvent_t after_linear = nullptr) {
@@ -792,67 +862,15 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
                  dim3(256), 0, st, reinterpret_cast<const __nv_bfloat16*>(ws + pl.KVp), static_cast<long>(pl.HW),
                  pl.C, pl.d, pl.heads, pl.NP, static_cast<long>(pl.Mp), KT, VTx);
       EDIT_TRY(last_launch());
-    } else {
-      DwTmaMaps mp;
-      std::memset(&mp, 0, sizeof(mp));
-      const long C2 = 2L * pl.C;
-      cuuint64_t d_in[4] = {(cuuint64_t)C2, (cuuint64_t)pl.W, (cuuint64_t)pl.H, (cuuint64_t)pl.B};
-      cuuint64_t s_in[3] = {(cuuint64_t)C2 * 2, (cuuint64_t)pl.W * C2 * 2, (cuuint64_t)pl.H * pl.W * C2 * 2};
-      cuuint32_t b_in[4] = {64, 65, 3, 1};
-      cuuint64_t d_kt[2] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.B * pl.C};
-      cuuint64_t s_kt[1] = {(cuuint64_t)pl.Mp * 2};
-      cuuint32_t b_kt[2] = {32, 64};
-      cuuint64_t d_vt[3] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.NP, (cuuint64_t)pl.B * pl.heads};
-      cuuint64_t s_vt[2] = {(cuuint64_t)pl.Mp * 2, (cuuint64_t)pl.NP * pl.Mp * 2};
-      cuuint32_t b_vt[3] = {32, 8, 1};
-      if (!encode(&mp.in, 4, ws + pl.KVp, d_in, s_in, b_in, SWZ_NONE) ||
-          !encode(&mp.kt, 2, KT, d_kt, s_kt, b_kt, SWZ_64) || !encode(&mp.vtx, 3, VTx, d_vt, s_vt, b_vt, SWZ_64))
-        return EDIT_ERR_CUDA;
-      const int tokmajor = pl.K ? 1 : 0;
-      if (tokmajor) {
-        cuuint64_t d_t[4] = {(cuuint64_t)pl.C, (cuuint64_t)pl.Wo, (cuuint64_t)pl.Ho, (cuuint64_t)pl.B};
-        cuuint64_t s_t[3] = {(cuuint64_t)pl.C * 2, (cuuint64_t)pl.Wo * pl.C * 2,
-                             (cuuint64_t)pl.Ho * pl.Wo * pl.C * 2};
-        cuuint32_t b_t[4] = {64, 32, 1, 1};
-        if (!encode(&mp.ktok, 4, ws + pl.K, d_t, s_t, b_t, SWZ_NONE) ||
-            !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
-          return EDIT_ERR_CUDA;
-      }
-      launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, 
-          mp, pl.H, pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
-          static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
-          static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, reinterpret_cast<int*>(ws + pl.status));
-      EDIT_TRY(last_launch());
-    }
-    {
       const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
       launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d,
                  pl.NP, pl.Mp);
       EDIT_TRY(last_launch());
+    } else {
+      EDIT_TRY(dwconv_tc(pl, w, ws, pl.H, 0, st));  // (writes the VTx padding rows too)
     }
     stage_mark(2, st);
-    TcGemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    if (!map_a(&p.a0, KT, pl.Mp, static_cast<long>(pl.B) * pl.C, 1, pl.Mp, static_cast<long>(pl.B) * pl.C * pl.Mp))
-      return EDIT_ERR_CUDA;
-    p.a1 = p.a0;
-    if (!map_b(&p.b0, VTx, pl.Mp, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.Mp, pl.NP)) return EDIT_ERR_CUDA;
-    p.b1 = p.b2 = p.bk = p.b0;
-    p.num_kb = (pl.Mp + 63) / 64;
-    p.kb_split = p.num_kb;
-    p.kb_per_chunk = pl.kv_kb;
-    p.num_chunks = pl.kv_chunks;
-    p.num_m_tiles = pl.kv_chunks;
-    p.num_tiles = pl.B * pl.heads * pl.kv_chunks;
-    p.num_n_tiles = 1;
-    p.n_split = pl.NP;
-    p.N = pl.NP;
-    p.d = pl.d;
-    p.heads = pl.heads;
-    p.kv_rows_per_img = pl.C;
-    p.kv_part = reinterpret_cast<float*>(ws + pl.kvpart);
-    p.status = reinterpret_cast<int*>(ws + pl.status);
-    EDIT_TRY(gemm_kvstate(p, pl.NP, st));
+    EDIT_TRY(kv_state_tc(pl, ws, st));
   } else {
     if (pl.compress) {
       const long total = static_cast<long>(pl.B) * pl.M * (2 * pl.C);
@@ -889,6 +907,97 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
   }
   stage_mark(3, st);
   return EDIT_OK;
+}
+
+// Step 5 on the tensor cores: U = Conv3x3(X) + b for the plan's image grid
+// (stage event 5 after the conv kernel when `marks`).
+int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, cudaStream_t st, bool marks) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  const int C = pl.C, Cr = pl.Cr;
+  TcGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!map_grid(&p.a0, x, pl.B, pl.H, pl.W, C, pl.TW, pl.TH)) return EDIT_ERR_CUDA;
+  p.a1 = p.a0;
+  if (!map_b(&p.b0, cf.cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr) / 2)) return EDIT_ERR_CUDA;
+  p.b1 = p.b2 = p.bk = p.b0;
+  p.num_kb = 9 * C / 64;
+  p.kb_split = p.num_kb;
+  p.kb_per_tap = C / 64;
+  p.n_split = Cr;
+  p.N = Cr;
+  p.num_n_tiles = 1;
+  p.H = pl.H;
+  p.W = pl.W;
+  p.TH = pl.TH;
+  p.TW = pl.TW;
+  p.tiles_h = pl.tiles_h;
+  p.tiles_w = pl.tiles_w;
+  p.num_m_tiles = pl.B * pl.tiles_h * pl.tiles_w;
+  p.out = ws + pl.U;
+  p.ldo = Cr;
+  if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
+  p.bias[0] = cf.cf3_b;
+  p.status = status;
+  if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
+    if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
+    p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
+    bool split = false;
+    EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
+    if (marks) stage_mark(5, st);
+    if (split) {
+      const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
+      launch_pdl(conv_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, 
+          p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
+          static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+      EDIT_TRY(last_launch());
+    }
+  } else {
+    p.ksplit = pl.conv_ksplit;
+    p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
+    EDIT_TRY(gemm_conv(p, Cr, st));
+    if (marks) stage_mark(5, st);
+    if (pl.conv_ksplit > 1) {
+      const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
+      launch_pdl(conv_splitk_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit,
+                 pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
+                 static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+      EDIT_TRY(last_launch());
+    }
+  }
+  return EDIT_OK;
+}
+
+// Step 7 on the tensor cores: out = ReLU([X | G] [Wl | Wl W1]^T + Wl b1 + bl)
+// for `tok` token rows of x and g, with the folded weights of the plan's
+// workspace (Wqw1, bfold); rows ldo elements apart.
+int query_gemm_tc(const void* x, long tok, const Plan& pl, const CfWeights& cf, const void* g, uint8_t* ws, void* qout,
+                  long ldo, cudaStream_t st) {
+  int* status = reinterpret_cast<int*>(ws + pl.status);
+  const int C = pl.C, Cr = pl.Cr;
+  TcGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!map_a(&p.a0, x, C, tok, 1, C, tok * C)) return EDIT_ERR_CUDA;
+  if (!map_a(&p.a1, g, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
+  const void* qb = ws + pl.bfold;
+  const int lbn = linear_bn(tok, C, 1 << 30, &qb, 1);
+  if (!map_b(&p.b0, cf.lin_w, C, C, C, linear_box(lbn))) return EDIT_ERR_CUDA;
+  if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, linear_box(lbn))) return EDIT_ERR_CUDA;
+  p.b1 = p.b2 = p.b0;
+  p.R = static_cast<int>(tok);
+  p.m_tiles_per_img = ceil_div(tok, 128);
+  p.num_m_tiles = p.m_tiles_per_img;
+  p.kb_split = C / 64;
+  p.num_kb = C / 64 + ceil_div(Cr, 64);
+  p.n_split = 1 << 30;  // one weight source; rows past C read as zeros
+  p.N = C;
+  p.out = qout;
+  p.ldo = ldo;
+  if (!map_out2d(&p.out_map, qout, C, tok, ldo)) return EDIT_ERR_CUDA;
+  p.bias[0] = ws + pl.bfold;
+  p.bias_f32 = 1;
+  p.relu = 1;
+  p.status = status;
+  return gemm_linear_pair(p, lbn, st);
 }
 
 // Cooperative launch of the fused GroupNorm (bf16): as many blocks as are
@@ -1000,7 +1109,6 @@ int run_fold(const Plan& pl, const CfWeights& cf, uint8_t* ws, cudaStream_t st) 
 template <typename T>
 int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_eps, float slope, void* qout, long ldo,
                    int barrier_off, bool marks, uint8_t* ws, cudaStream_t st, bool fold, cudaEvent_t fold_ready) {
-  int* status = reinterpret_cast<int*>(ws + pl.status);
   auto mark = [&](int i) {
     if (marks) stage_mark(i, st);
   };
@@ -1012,56 +1120,7 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
   float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
   bool gn_fused = false;
   if (pl.bf16) {
-    TcGemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    if (!map_grid(&p.a0, x, pl.B, pl.H, pl.W, C, pl.TW, pl.TH)) return EDIT_ERR_CUDA;
-    p.a1 = p.a0;
-    if (!map_b(&p.b0, cf.cf3_w, 9L * C, Cr, 9L * C, conv_chunk(Cr) / 2)) return EDIT_ERR_CUDA;
-    p.b1 = p.b2 = p.bk = p.b0;
-    p.num_kb = 9 * C / 64;
-    p.kb_split = p.num_kb;
-    p.kb_per_tap = C / 64;
-    p.n_split = Cr;
-    p.N = Cr;
-    p.num_n_tiles = 1;
-    p.H = pl.H;
-    p.W = pl.W;
-    p.TH = pl.TH;
-    p.TW = pl.TW;
-    p.tiles_h = pl.tiles_h;
-    p.tiles_w = pl.tiles_w;
-    p.num_m_tiles = pl.B * pl.tiles_h * pl.tiles_w;
-    p.out = ws + pl.U;
-    p.ldo = Cr;
-    if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
-    p.bias[0] = cf.cf3_b;
-    p.status = status;
-    if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
-      if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
-      p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
-      bool split = false;
-      EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
-      mark(5);
-      if (split) {
-        const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
-        launch_pdl(conv_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, 
-            p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
-            static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
-        EDIT_TRY(last_launch());
-      }
-    } else {
-      p.ksplit = pl.conv_ksplit;
-      p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
-      EDIT_TRY(gemm_conv(p, Cr, st));
-      mark(5);
-      if (pl.conv_ksplit > 1) {
-        const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
-        launch_pdl(conv_splitk_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit,
-                   pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
-                   static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
-        EDIT_TRY(last_launch());
-      }
-    }
+    EDIT_TRY(conv3x3_tc(x, pl, cf, ws, st, marks));
     if ((Cr / pl.G) >= 8 && Cr / 8 <= 512) {
       // 6. G = LeakyReLU(GN(U)) in one cooperative grid: statistics, grid barrier, apply
       const int r = launch_gn_fused(pl, cf, gn_eps, slope, barrier_off, ws, st);
@@ -1123,30 +1182,7 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
   // 7. Q
   if (fold_ready && cudaStreamWaitEvent(st, fold_ready, 0) != cudaSuccess) return EDIT_ERR_CUDA;
   if (pl.bf16) {
-    TcGemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    if (!map_a(&p.a0, x, C, tok, 1, C, tok * C)) return EDIT_ERR_CUDA;
-    if (!map_a(&p.a1, ws + pl.Gb, Cr, tok, 1, Cr, tok * Cr)) return EDIT_ERR_CUDA;
-    const void* qb = ws + pl.bfold;
-    const int lbn = linear_bn(tok, C, 1 << 30, &qb, 1);
-    if (!map_b(&p.b0, cf.lin_w, C, C, C, linear_box(lbn))) return EDIT_ERR_CUDA;
-    if (!map_b(&p.bk, ws + pl.Wqw1, Cr, C, Cr, linear_box(lbn))) return EDIT_ERR_CUDA;
-    p.b1 = p.b2 = p.b0;
-    p.R = static_cast<int>(tok);
-    p.m_tiles_per_img = ceil_div(tok, 128);
-    p.num_m_tiles = p.m_tiles_per_img;
-    p.kb_split = C / 64;
-    p.num_kb = C / 64 + ceil_div(Cr, 64);
-    p.n_split = 1 << 30;  // one weight source; rows past C read as zeros
-    p.N = C;
-    p.out = qout;
-    p.ldo = ldo;
-    if (!map_out2d(&p.out_map, qout, C, tok, ldo)) return EDIT_ERR_CUDA;
-    p.bias[0] = ws + pl.bfold;
-    p.bias_f32 = 1;
-    p.relu = 1;
-    p.status = status;
-    EDIT_TRY(gemm_linear_pair(p, lbn, st));
+    EDIT_TRY(query_gemm_tc(x, tok, pl, cf, ws + pl.Gb, ws, qout, ldo, st));
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -1296,12 +1332,12 @@ int launch_sdpa_tc(const void* q, long ldq, int Nq, const SdpaSet& s1, const Sdp
   p.nimg = pl.B;
   p.n1 = s1.n;
   p.n2 = s2 ? s2->n : 0;
-  auto kern = sdpa_tc_kernel<D>;
+  auto kern = s2 ? sdpa_tc_kernel<D, 2> : sdpa_tc_kernel<D, 1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
     return EDIT_ERR_CUDA;
   const long items = B * heads * ceil_div(Nq, 128);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  launch_pdl(kern, dim3(grid), dim3(192), Cfg::SMEM_BYTES, st, mq, mk1, mv1, mk2, mv2, p);
+  launch_pdl(kern, dim3(grid), dim3(320), Cfg::SMEM_BYTES, st, mq, mk1, mv1, mk2, mv2, p);
   return last_launch();
 }
 
@@ -1526,6 +1562,137 @@ int run_mm(const void* x_img, const void* x_txt, const Plan& pl, const mmedit_we
   return EDIT_OK;
 }
 
+// ------------------------------------------------------------ row bands
+// One image split into horizontal bands of rows, one per rank. Layout of a
+// band's workspace: the plan `pe` of the band with its halo rows as one image
+// (conv3x3, U, G, GroupNorm partials, weight folding, K'|V' of the band and its
+// upper halo row), then the plan `pq` of the band's own rows (compressed K, V,
+// KV state, Q, the apply operand), whose offsets are shifted past pe's.
+struct BandPlan {
+  Plan pe, pq;
+  int H, row0, rows, top, bot;
+  size_t rec_bytes, sz_off, total;
+};
+
+// The record a band contributes to the two global reductions: fp64 GroupNorm
+// sums [groups][2] at byte 0, fp32 [S | z] [heads][d][d + 1] at sz_off.
+size_t band_record_layout(int groups, int heads, int d, size_t* sz_off) {
+  *sz_off = align_up(static_cast<size_t>(groups) * 2 * sizeof(double), 256);
+  return align_up(*sz_off + static_cast<size_t>(heads) * d * (d + 1) * sizeof(float), 256);
+}
+
+int make_band_plan(int W, int C, int heads, const edit_band* band, const edit_attn_weights* w, BandPlan& bp) {
+  if (!band || !w) return EDIT_ERR_NULL;
+  if (w->dtype != EDIT_F32 && w->dtype != EDIT_BF16) return EDIT_ERR_DTYPE;
+  if (w->dtype != EDIT_BF16) return EDIT_ERR_UNSUPPORTED;
+  const int H = band->H, r0 = band->row0, rows = band->rows;
+  if (H < 1 || rows < 1 || r0 < 0 || r0 > H - rows) return EDIT_ERR_SHAPE;
+  // band boundaries on even rows: no stride-2 key/value token straddles two bands
+  if (r0 % 2 != 0 || (r0 + rows != H && (r0 + rows) % 2 != 0)) return EDIT_ERR_SHAPE;
+  bp.H = H;
+  bp.row0 = r0;
+  bp.rows = rows;
+  bp.top = r0 > 0 ? 1 : 0;
+  bp.bot = r0 + rows < H ? 1 : 0;
+  EDIT_TRY_CHECK(make_plan(1, rows + bp.top + bp.bot, W, C, heads, 0, w, bp.pe));
+  EDIT_TRY_CHECK(make_plan(1, rows, W, C, heads, 0, w, bp.pq));
+  const size_t sh = bp.pe.total;
+  Plan& q = bp.pq;
+  q.status = bp.pe.status;
+  q.KT += sh;
+  q.VTx += sh;
+  q.kvpart += sh;
+  q.Sz += sh;
+  q.SzT += sh;
+  q.Q += sh;
+  bp.total = bp.pe.total + q.total;
+  bp.rec_bytes = band_record_layout(bp.pe.G, heads, bp.pe.d, &bp.sz_off);
+  return EDIT_OK;
+}
+
+// Band step 1: its rows' compressed K, V and partial [S | z]; U of the band
+// with its halo rows and the band rows' GroupNorm sums. Writes the record.
+int run_band_partials(const void* x, const BandPlan& bp, const edit_attn_weights* w, uint8_t* ws, uint8_t* rec,
+                      cudaStream_t st) {
+  const Plan& pe = bp.pe;
+  const Plan& pq = bp.pq;
+  int* status = reinterpret_cast<int*>(ws + pe.status);
+  if (cudaMemsetAsync(ws + pe.status, 0, 256, st) != cudaSuccess) return EDIT_ERR_CUDA;
+  const int W = pe.W, C = pe.C, Cr = pe.Cr;
+  // K'|V' of the band's rows and its upper halo row; the depthwise conv reads
+  // them with that halo as row 0 (output row i: rows 2i - 1 + top .. 2i + 1 + top)
+  const long tokkv = static_cast<long>(bp.rows + bp.top) * W;
+  const void* wts[2] = {w->k_w, w->v_w};
+  const void* bs[2] = {w->k_b, w->v_b};
+  EDIT_TRY(tc_linear(x, tokkv, C, wts, bs, 2, C, ws + pe.KVp, 2L * C, 0, status, st));
+  Plan pk = pq;  // the K'|V' rows live in pe's buffer
+  pk.KVp = pe.KVp;
+  EDIT_TRY(dwconv_tc(pk, w, ws, bp.rows + bp.top, bp.top, st));
+  EDIT_TRY(kv_state_tc(pq, ws, st));
+  const int per_head = pq.d * (pq.d + 1);
+  const long total = static_cast<long>(pq.heads) * per_head;
+  launch_pdl(kv_state_combine_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st,
+             reinterpret_cast<const float*>(ws + pq.kvpart), pq.kv_chunks, per_head, total,
+             reinterpret_cast<float*>(rec + bp.sz_off));
+  EDIT_TRY(last_launch());
+  // U of the band with its halo rows (the halo rows' own outputs are not used)
+  EDIT_TRY(conv3x3_tc(x, pe, query_cf(w), ws, st, false));
+  const __nv_bfloat16* Ub = reinterpret_cast<const __nv_bfloat16*>(ws + pe.U) + static_cast<long>(bp.top) * W * Cr;
+  float* gnpart = reinterpret_cast<float*>(ws + pe.gnpart);
+  launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pq.gn_P, 1)), dim3(256), 0, st, Ub,
+             static_cast<int>(pq.HW), Cr, pe.G, pq.gn_P, gnpart);
+  EDIT_TRY(last_launch());
+  launch_pdl(gn_band_sums_kernel, dim3(pe.G), dim3(256), 0, st, static_cast<const float*>(gnpart), pq.gn_P, pe.G,
+             reinterpret_cast<double*>(rec));
+  return last_launch();
+}
+
+// Band step 2: the global GroupNorm statistics and [S | z] from every band's
+// record (summed in band order), then G, the query and the attention output of
+// the band's rows.
+int run_band_finish(const void* x, const BandPlan& bp, const edit_attn_weights* w, uint8_t* ws, const uint8_t* recs,
+                    int nrec, void* out, cudaStream_t st) {
+  const Plan& pe = bp.pe;
+  const Plan& pq = bp.pq;
+  const int W = pe.W, C = pe.C, Cr = pe.Cr;
+  const long count = static_cast<long>(bp.H) * W * (Cr / pe.G);
+  launch_pdl(gn_band_finalize_kernel, dim3(pe.G), dim3(64), 0, st, recs, nrec, static_cast<long>(bp.rec_bytes), pe.G,
+             Cr, count, w->gn_eps, static_cast<const __nv_bfloat16*>(w->gn_gamma),
+             static_cast<const __nv_bfloat16*>(w->gn_beta), reinterpret_cast<float*>(ws + pe.gnstats),
+             reinterpret_cast<float*>(ws + pe.gnss));
+  EDIT_TRY(last_launch());
+  const long tok = pq.HW;
+  {
+    const int nvec = Cr / 8;
+    const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
+    launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(per_block * nvec), 0, st,
+               reinterpret_cast<const __nv_bfloat16*>(ws + pe.U) + static_cast<long>(bp.top) * W * Cr,
+               reinterpret_cast<const float*>(ws + pe.gnss), tok, Cr, w->leaky_slope,
+               reinterpret_cast<__nv_bfloat16*>(ws + pe.Gb), tok);
+    EDIT_TRY(last_launch());
+  }
+  const CfWeights cf = query_cf(w);
+  EDIT_TRY(run_fold<__nv_bfloat16>(pe, cf, ws, st));
+  const void* xb = static_cast<const __nv_bfloat16*>(x) + static_cast<long>(bp.top) * W * C;
+  EDIT_TRY(query_gemm_tc(xb, tok, pe, cf, ws + pe.Gb, ws, ws + pq.Q, C, st));
+  const long total_t = static_cast<long>(pq.heads) * pq.NP * pq.KP;
+  launch_pdl(sz_band_combine_pack_kernel, dim3(grid_for(total_t, 256)), dim3(256), 0, st, recs, nrec,
+             static_cast<long>(bp.rec_bytes), static_cast<long>(bp.sz_off), pq.d, pq.NP, pq.KP, total_t,
+             reinterpret_cast<float*>(ws + pq.Sz), reinterpret_cast<__nv_bfloat16*>(ws + pq.SzT));
+  EDIT_TRY(last_launch());
+  return run_apply<__nv_bfloat16>(pq, w, ws, out, st);
+}
+
+int band_checks(const void* x, const edit_attn_weights* w, const BandPlan& bp) {
+  if (!x) return EDIT_ERR_NULL;
+  EDIT_TRY_CHECK(check_weights(w, bp.pe));
+  if (!aligned(x, 16)) return EDIT_ERR_ALIGN;
+  if (!w->workspace) return EDIT_ERR_NULL;
+  if (!aligned(w->workspace, 256)) return EDIT_ERR_ALIGN;
+  if (w->workspace_bytes < bp.total) return EDIT_ERR_WORKSPACE;
+  return EDIT_OK;
+}
+
 int common_checks(const void* x, const void* out, const edit_attn_weights* w, void* ws, size_t ws_bytes,
                   const Plan& pl, const edit_attn_variant* var = nullptr) {
   if (!x || !out || !ws) return EDIT_ERR_NULL;
@@ -1615,6 +1782,40 @@ int edit_attn_read_status(const void* workspace, void* stream, int* status) {
     return EDIT_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return EDIT_ERR_CUDA;
   return EDIT_OK;
+}
+
+size_t edit_attn_band_workspace_bytes(int W, int C, int heads, const edit_band* band, const edit_attn_weights* w) {
+  BandPlan bp;
+  return make_band_plan(W, C, heads, band, w, bp) == EDIT_OK ? bp.total : 0;
+}
+
+size_t edit_attn_band_record_bytes(int C, int heads, const edit_attn_weights* w) {
+  if (!w || heads < 1 || C % heads != 0 || w->gn_groups < 1) return 0;
+  size_t sz_off = 0;
+  return band_record_layout(w->gn_groups, heads, C / heads, &sz_off);
+}
+
+int edit_attn_band_partials(const void* x_ext, int W, int C, int heads, const edit_band* band,
+                            const edit_attn_weights* w, void* record, void* stream) {
+  BandPlan bp;
+  EDIT_TRY(make_band_plan(W, C, heads, band, w, bp));
+  EDIT_TRY(band_checks(x_ext, w, bp));
+  if (!record) return EDIT_ERR_NULL;
+  if (!aligned(record, 256)) return EDIT_ERR_ALIGN;
+  return run_band_partials(x_ext, bp, w, static_cast<uint8_t*>(w->workspace), static_cast<uint8_t*>(record),
+                           static_cast<cudaStream_t>(stream));
+}
+
+int edit_attn_band_finish(const void* x_ext, int W, int C, int heads, const edit_band* band,
+                          const edit_attn_weights* w, const void* records, int nrecords, void* out, void* stream) {
+  BandPlan bp;
+  EDIT_TRY(make_band_plan(W, C, heads, band, w, bp));
+  EDIT_TRY(band_checks(x_ext, w, bp));
+  if (!records || !out) return EDIT_ERR_NULL;
+  if (nrecords < 1 || nrecords > (bp.H + 1) / 2) return EDIT_ERR_SHAPE;
+  if (!aligned(records, 256) || !aligned(out, 16)) return EDIT_ERR_ALIGN;
+  return run_band_finish(x_ext, bp, w, static_cast<uint8_t*>(w->workspace), static_cast<const uint8_t*>(records),
+                         nrecords, out, static_cast<cudaStream_t>(stream));
 }
 
 const char* edit_status_string(int status) {

@@ -17,14 +17,15 @@
 //            O_g = P_g [V_g | 1]^T (M = 128, N = NPV) into one of two TMEM O
 //            buffers. Column d of O is the row sum of P (the ones row of V^T),
 //            so numerator and denominator come from the same bf16 P.
-//   warps 2-5 softmax, one thread per query row (its TMEM lane): the row max
-//            of the tile (first pass over S), P = exp2(S c - m) rounded to bf16
-//            and written to shared memory as the K-major A operand of the
-//            second product (128-byte swizzle, second pass over S); then the
-//            running accumulator R = R 2^(m_prev - m) + O of the previous tile
-//            (deferred by one tile so that the next tile's exponentials overlap
-//            the product), R / R[d] at the end of a key set, and the blended
-//            output row at the end of the item.
+//   warps 2-9 softmax, two threads per query row (its TMEM lane), one per
+//            64-key half of the tile: the half's row max, exchanged with the
+//            partner through shared memory; P = 2^(S c - m) rounded to bf16 and
+//            written to shared memory as the K-major A operand of the second
+//            product (128-byte swizzle); then, for half of the accumulator
+//            columns, the running accumulator R = R 2^(m_prev - m) + O of the
+//            previous tile (deferred by one tile so that the next tile's
+//            exponentials overlap the product), R / l at the end of a key set,
+//            and the blended output row at the end of the item.
 // Keys past the set's end (the zero-filled or next-image rows of a tile) get
 // P = 0. Every wait is bounded (EDIT_ERR_TIMEOUT in the status word).
 #pragma once
@@ -57,34 +58,50 @@ struct SdpaTcCfg {
   static constexpr int VBOX = NPV * 128;             // NPV rows x 64 keys
   static constexpr int V_BYTES = STAGES * 2 * VBOX;
   static constexpr int P_BYTES = 2 * 2 * QBOX;       // two P buffers of 128 rows x 128 keys
+  static constexpr int XCH_BYTES = (2 * 2 * 128 + 128) * 4;  // row-max exchange (2 tiles x 2 halves), l exchange
   static constexpr int BAR_BYTES = (2 * QB + 2 * STAGES + 10) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + K_BYTES + V_BYTES + P_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + K_BYTES + V_BYTES + P_BYTES + XCH_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, NPV);
   static constexpr int TMEM_COLS = 512;  // S buffers at 0, 128; O buffers at 256, 384
+  static constexpr int OC = (D + 16) / 16;    // 16-column chunks of [O | l] (d + 1 columns)
+  static constexpr int OC0 = (OC + 1) / 2;    // chunks of the first softmax half
+  static constexpr int OCH = OC0;             // most chunks a half holds
 };
 
-// 32 lanes x 32 consecutive fp32 columns.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
-      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+// 2^x with the SFU's approximate exponential (flushes denormals; P is rounded
+// to bf16 right after, far coarser than its error).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-template <int D>
-__global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__ CUtensorMap mq,
+// 32 lanes x N consecutive fp32 columns (N = 32 or 64), waited for.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld_cols<64>(uint32_t taddr, float (&v)[64]) {
+  tmem_ld64(taddr, v);
+}
+template <>
+__device__ __forceinline__ void tmem_ld_cols<32>(uint32_t taddr, float (&v)[32]) {
+  float a[16], b[16];
+  tmem_ld16(taddr, a);
+  tmem_ld16(taddr + 16, b);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = a[i];
+    v[16 + i] = b[i];
+  }
+}
+
+// NSET: number of key sets (1: image rows, 2: prompt rows). With two sets
+// the first set's share is kept in registers, so S is read 32 columns at a
+// time (twice) to stay within the register budget of 10 warps.
+template <int D, int NSET>
+__global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__ CUtensorMap mq,
                                                          const __grid_constant__ CUtensorMap mk1,
                                                          const __grid_constant__ CUtensorMap mv1,
                                                          const __grid_constant__ CUtensorMap mk2,
@@ -92,13 +109,16 @@ __global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__
                                                          const SdpaTcParams p) {
   using Cfg = SdpaTcCfg<D>;
   constexpr int NBX = Cfg::NBX, KS = Cfg::KS, NPV = Cfg::NPV, STAGES = Cfg::STAGES, QB = Cfg::QB;
-  constexpr int QBOX = Cfg::QBOX, VBOX = Cfg::VBOX;
+  constexpr int QBOX = Cfg::QBOX, VBOX = Cfg::VBOX, OC = Cfg::OC, OC0 = Cfg::OC0, OCH = Cfg::OCH;
+  constexpr int CW = NSET == 1 ? 64 : 32, NCW = 64 / CW;  // S columns read at a time
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sQ = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = sQ + Cfg::Q_BYTES;
   uint8_t* sV = sK + Cfg::K_BYTES;
   uint8_t* sP = sV + Cfg::V_BYTES;
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + Cfg::P_BYTES);
+  float* mx = reinterpret_cast<float*>(sP + Cfg::P_BYTES);  // [2 tiles][2 halves][128 rows]
+  float* lsum = mx + 2 * 2 * 128;                          // [128 rows]
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + Cfg::P_BYTES + Cfg::XCH_BYTES);
   uint64_t* q_empty = q_full + QB;
   uint64_t* kv_full = q_empty + QB;
   uint64_t* kv_empty = kv_full + STAGES;
@@ -122,10 +142,10 @@ __global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);  // one arrival per softmax warp
-      mbar_init(&p_full[i], 4);
+      mbar_init(&s_empty[i], 8);  // one arrival per softmax warp
+      mbar_init(&p_full[i], 8);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 4);
+      mbar_init(&o_empty[i], 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -250,43 +270,49 @@ __global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / output
-    const int q4 = warp & 3;  // TMEM lane quarter of this warp
+    // Two warps per TMEM lane quarter: half hf of the warps takes keys
+    // 64 hf .. 64 hf + 63 of every tile (one 64-key sub-buffer of P) and the
+    // accumulator columns [16 OC0 hf, ...) (the l column d lies in half 1).
+    const int q4 = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int row = q4 * 32 + lane;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16);
-    const float c = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e): exp2 below
-    const uint32_t prow = static_cast<uint32_t>(row) * 128u;
+    const float c = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e): base-2 exponent
     const uint32_t psw = static_cast<uint32_t>(row & 7);
+    uint8_t* prow = sP + hf * QBOX + row * 128;  // + sb * 2 * QBOX: P buffer of the tile
+    const int col0 = hf ? 16 * OC0 : 0;  // first accumulator column of this half
+    const int nch = hf ? OC - OC0 : OC0;  // its 16-column chunks
     long g = 0;
     bool ok = true;
-    float R[D + 1];
-    float acc[D];
+    float R[16 * OCH];
+    float acc[NSET == 2 ? 16 * OCH : 1];  // the first set's share (two sets only)
     for (long it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
       const int qt = static_cast<int>(it % qtiles);
       const long bh = it / qtiles;
       const int h = static_cast<int>(bh % p.heads), b = static_cast<int>(bh / p.heads);
-#pragma unroll
-      for (int i = 0; i < D; ++i) acc[i] = 0.f;
-      for (int set = 0; set < 2 && ok; ++set) {
+      float sc = 0.f;
+      for (int set = 0; set < NSET && ok; ++set) {
         const int n = set == 0 ? p.n1 : p.n2;
         const int Ts = set == 0 ? T1 : T2;
         if (Ts == 0) continue;
 #pragma unroll
-        for (int i = 0; i <= D; ++i) R[i] = 0.f;
+        for (int i = 0; i < 16 * OCH; ++i) R[i] = 0.f;
         float m_run = -INFINITY, m_acc = -INFINITY, m_pend = -INFINITY;
-        // R = R 2^(m_acc - m_j) + O_j for tile gg whose P used the max m_j
+        // R = R 2^(m_acc - m_j) + O_j (this half's columns) for tile gg whose P used the max m_j
         auto accumulate = [&](long gg, float m_j) -> bool {
           const int ob = static_cast<int>(gg & 1);
           if (!warp_wait(&o_full[ob], static_cast<uint32_t>((gg >> 1) & 1), abort_flag, p.status)) return false;
           tc_fence_after();
-          const float alpha = exp2f(m_acc - m_j);
+          const float alpha = ex2_approx(m_acc - m_j);
           m_acc = m_j;
 #pragma unroll
-          for (int ch = 0; ch < (D + 16) / 16; ++ch) {
-            float v[16];
-            tmem_ld16(t_lane + 256 + 128 * ob + 16 * ch, v);
+          for (int ch = 0; ch < OCH; ++ch) {
+            if (ch < nch) {
+              float v[16];
+              tmem_ld16(t_lane + 256 + 128 * ob + col0 + 16 * ch, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (16 * ch + i <= D) R[16 * ch + i] = fmaf(R[16 * ch + i], alpha, v[i]);
+              for (int i = 0; i < 16; ++i) R[16 * ch + i] = fmaf(R[16 * ch + i], alpha, v[i]);
+            }
           }
           tc_fence_before();
           __syncwarp();
@@ -300,43 +326,53 @@ __global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__
             break;
           }
           tc_fence_after();
-          const int nvalid = n - tt * 128 < 128 ? n - tt * 128 : 128;
-          // pass 1: the tile's row max over its valid keys
+          // valid keys of this half: 0 .. nv - 1
+          int nv = n - tt * 128 - 64 * hf;
+          nv = nv < 0 ? 0 : (nv > 64 ? 64 : nv);
+          const uint32_t s_addr = t_lane + 128 * sb + 64 * hf;
+          float v[CW];
           float mt = -INFINITY;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            if (32 * ch < nvalid) {
-              float v[32];
-              tmem_ld32(t_lane + 128 * sb + 32 * ch, v);
+          for (int k = 0; k < NCW; ++k) {
+            if (nv > CW * k) {
+              tmem_ld_cols<CW>(s_addr + CW * k, v);
+              if (nv == 64) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (32 * ch + i < nvalid) mt = fmaxf(mt, v[i]);
+                for (int i = 0; i < CW; ++i) mt = fmaxf(mt, v[i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < CW; ++i)
+                  if (CW * k + i < nv) mt = fmaxf(mt, v[i]);
+              }
             }
           }
-          const float m_new = fmaxf(m_run, mt * c);
+          // the row max of the tile: both halves exchange theirs
+          float* mxb = mx + (g & 1) * 256;
+          mxb[hf * 128 + row] = mt;
+          named_bar_sync(1 + q4, 64);
+          const float m_new = fmaxf(m_run, fmaxf(mt, mxb[(hf ^ 1) * 128 + row]) * c);
           m_run = m_new;
-          // pass 2: P = 2^(S c - m) in bf16, 128-byte-swizzled K-major rows
-          uint8_t* pb = sP + sb * 2 * QBOX;
+          // P = 2^(S c - m) in bf16, 128-byte-swizzled K-major rows of this half's sub-buffer
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            float v[32];
-            if (32 * ch < nvalid) tmem_ld32(t_lane + 128 * sb + 32 * ch, v);
+          for (int k = 0; k < NCW; ++k) {
+            if (NCW > 1 && nv > CW * k) tmem_ld_cols<CW>(s_addr + CW * k, v);  // (one chunk held at a time)
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
+            for (int q8 = 0; q8 < CW / 8; ++q8) {
               float e[8];
+              const int key0 = CW * k + 8 * q8;
+              if (nv == 64) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int key = 32 * ch + 8 * q8 + i;
-                e[i] = key < nvalid ? exp2f(fmaf(v[8 * q8 + i], c, -m_new)) : 0.f;
+                for (int i = 0; i < 8; ++i) e[i] = ex2_approx(fmaf(v[8 * q8 + i], c, -m_new));
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) e[i] = key0 + i < nv ? ex2_approx(fmaf(v[8 * q8 + i], c, -m_new)) : 0.f;
               }
               uint4 w;
               w.x = pack_bf16x2(e[0], e[1]);
               w.y = pack_bf16x2(e[2], e[3]);
               w.z = pack_bf16x2(e[4], e[5]);
               w.w = pack_bf16x2(e[6], e[7]);
-              const int key0 = 32 * ch + 8 * q8;               // first key of this 16-byte chunk
-              const uint32_t chunk = static_cast<uint32_t>((key0 & 63) >> 3);
-              *reinterpret_cast<uint4*>(pb + (key0 >> 6) * QBOX + prow + ((chunk ^ psw) << 4)) = w;
+              *reinterpret_cast<uint4*>(prow + sb * 2 * QBOX + ((static_cast<uint32_t>(key0 >> 3) ^ psw) << 4)) = w;
             }
           }
           fence_proxy_async_smem();  // P is read by the tensor cores (async proxy)
@@ -357,35 +393,46 @@ __global__ void __launch_bounds__(192, 1) sdpa_tc_kernel(const __grid_constant__
           }
         }
         if (!ok) break;
+        // l = column d (half 1) to both halves, then acc += w R / l
+        if (hf) lsum[row] = R[D - 16 * OC0];
+        named_bar_sync(1 + q4, 64);
+        const float l = lsum[row];
+        named_bar_sync(1 + q4, 64);  // (lsum is rewritten at the next set's end)
         const float w = set == 0 ? p.w1 : p.w2;
-        const float sc = R[D] > 0.f ? w / R[D] : 0.f;
+        sc = l > 0.f ? w / l : 0.f;
+        if (NSET == 2 && set == 0) {
 #pragma unroll
-        for (int i = 0; i < D; ++i) acc[i] = fmaf(R[i], sc, acc[i]);
+          for (int i = 0; i < 16 * OCH; ++i) acc[NSET == 2 ? i : 0] = R[i] * sc;
+        }
       }
       if (!ok) break;
       const int r = qt * 128 + row;
       if (r < p.Nq) {
-        __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D;
+        __nv_bfloat16* og =
+            reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D + col0;
 #pragma unroll
-        for (int c8 = 0; c8 < D; c8 += 8) {
-          float o[8];
+        for (int c8 = 0; c8 < 16 * OCH; c8 += 8) {
+          if (col0 + c8 < D) {
+            float o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = acc[c8 + i];
-          if (p.blend_in) {
-            const uint4 old = *reinterpret_cast<const uint4*>(og + c8);
-            const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+            for (int i = 0; i < 8; ++i)
+              o[i] = NSET == 2 ? fmaf(R[c8 + i], sc, acc[NSET == 2 ? c8 + i : 0]) : R[c8 + i] * sc;
+            if (p.blend_in) {
+              const uint4 old = *reinterpret_cast<const uint4*>(og + c8);
+              const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              o[2 * i] = fmaf(p.w0, __uint_as_float(ow[i] << 16), o[2 * i]);
-              o[2 * i + 1] = fmaf(p.w0, __uint_as_float(ow[i] & 0xffff0000u), o[2 * i + 1]);
+              for (int i = 0; i < 4; ++i) {
+                o[2 * i] = fmaf(p.w0, __uint_as_float(ow[i] << 16), o[2 * i]);
+                o[2 * i + 1] = fmaf(p.w0, __uint_as_float(ow[i] & 0xffff0000u), o[2 * i + 1]);
+              }
             }
+            uint4 wv;
+            wv.x = pack_bf16x2(o[0], o[1]);
+            wv.y = pack_bf16x2(o[2], o[3]);
+            wv.z = pack_bf16x2(o[4], o[5]);
+            wv.w = pack_bf16x2(o[6], o[7]);
+            *reinterpret_cast<uint4*>(og + c8) = wv;
           }
-          uint4 wv;
-          wv.x = pack_bf16x2(o[0], o[1]);
-          wv.y = pack_bf16x2(o[2], o[3]);
-          wv.z = pack_bf16x2(o[4], o[5]);
-          wv.w = pack_bf16x2(o[6], o[7]);
-          *reinterpret_cast<uint4*>(og + c8) = wv;
         }
       }
     }

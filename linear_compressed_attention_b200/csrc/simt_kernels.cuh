@@ -646,7 +646,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
                                                             const __nv_bfloat16* __restrict__ kb,
                                                             const __nv_bfloat16* __restrict__ vw,
                                                             const __nv_bfloat16* __restrict__ vb, int tokmajor,
-                                                            int* status) {
+                                                            int row_shift, int* status) {
   pdl_wait();
   constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
   __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&m.in);
     mbar_arrive_expect_tx(&bar, 3 * PW * CB * 2);
-    tma_load_4d(&m.in, &bar, &in_s[0][0][0], gc0, 2 * j0 - 1, 2 * i - 1, b);
+    tma_load_4d(&m.in, &bar, &in_s[0][0][0], gc0, 2 * j0 - 1, 2 * i - 1 + row_shift, b);
   }
   const int c = threadIdx.x & (CB - 1);
   const int tg = threadIdx.x >> 6;  // tokens 8*tg .. 8*tg + 7
@@ -1100,6 +1100,101 @@ __global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
     float v = res[c];
     if (p.blend_in) v = fmaf(p.w0, to_f32(op[c]), v);
     op[c] = from_f32<T>(v);
+  }
+}
+
+// ================================================================ row bands
+// One image split into row bands over several ranks (edit_attn_band_*): each
+// band contributes partial sums to the layer's two global reductions, the
+// GroupNorm statistics of U and the per-head [S | z]; every rank then sums all
+// bands' records in band order.
+
+// Band GroupNorm sums: (sum, sum of squares) per group over this band's
+// tokens, from the gn_partial_kernel partials part [P][groups][2] (one image),
+// in fp64 with a fixed order (thread t sums partials t, t + 256, ..., then a
+// fixed tree). One block of 256 threads per group.
+__global__ void __launch_bounds__(256) gn_band_sums_kernel(const float* __restrict__ part, int P, int groups,
+                                                          double* __restrict__ out) {
+  pdl_wait();
+  __shared__ double r1[256], r2[256];
+  const int g = blockIdx.x, t = threadIdx.x;
+  double s1 = 0.0, s2 = 0.0;
+  for (int i = t; i < P; i += 256) {
+    const float2 q = *reinterpret_cast<const float2*>(part + (static_cast<long>(i) * groups + g) * 2);
+    s1 += q.x;
+    s2 += q.y;
+  }
+  r1[t] = s1;
+  r2[t] = s2;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (t < w) {
+      r1[t] += r1[t + w];
+      r2[t] += r2[t + w];
+    }
+    __syncthreads();
+  }
+  if (t == 0) {
+    out[g * 2] = r1[0];
+    out[g * 2 + 1] = r2[0];
+  }
+}
+
+// Global GroupNorm from all bands' records (rec_stride bytes apart, the fp64
+// sums first): totals summed in band order in fp64, then mean, biased
+// variance, rstd over `count` elements per group and the per-channel affine
+// form scale = gamma * rstd, shift = beta - mean * scale. One block per group.
+__global__ void __launch_bounds__(64) gn_band_finalize_kernel(const uint8_t* __restrict__ recs, int nrec,
+                                                             long rec_stride, int groups, int Cr, long count, float eps,
+                                                             const __nv_bfloat16* __restrict__ gamma,
+                                                             const __nv_bfloat16* __restrict__ beta,
+                                                             float* __restrict__ stats, float* __restrict__ ss) {
+  pdl_wait();
+  const int g = blockIdx.x;
+  double s1 = 0.0, s2 = 0.0;
+  for (int r = 0; r < nrec; ++r) {
+    const double* q = reinterpret_cast<const double*>(recs + r * rec_stride) + 2 * g;
+    s1 += q[0];
+    s2 += q[1];
+  }
+  const double mean = s1 / static_cast<double>(count);
+  double var = s2 / static_cast<double>(count) - mean * mean;
+  if (var < 0.0) var = 0.0;
+  const double rstd = 1.0 / sqrt(var + static_cast<double>(eps));
+  if (threadIdx.x == 0) {
+    stats[g * 2] = static_cast<float>(mean);
+    stats[g * 2 + 1] = static_cast<float>(rstd);
+  }
+  const int cpg = Cr / groups;
+  for (int c = g * cpg + threadIdx.x; c < (g + 1) * cpg; c += blockDim.x) {
+    const double sc = static_cast<double>(__bfloat162float(gamma[c])) * rstd;
+    ss[c * 2] = static_cast<float>(sc);
+    ss[c * 2 + 1] = static_cast<float>(static_cast<double>(__bfloat162float(beta[c])) - mean * sc);
+  }
+}
+
+// Global [S | z] from all bands' records (the fp32 [heads][d][d + 1] block at
+// byte sz_off of each record), summed in band order; writes Sz and the bf16
+// apply operand SzT [heads][NP][KP] (SzT[h][c][a] = [S | z]_h[a][c], zero
+// outside c <= d, a < d), as kv_state_combine_pack_kernel does for one image.
+__global__ void sz_band_combine_pack_kernel(const uint8_t* __restrict__ recs, int nrec, long rec_stride, long sz_off,
+                                            int d, int NP, int KP, long total, float* __restrict__ Sz,
+                                            __nv_bfloat16* __restrict__ SzT) {
+  pdl_wait();
+  const int per_head = d * (d + 1);
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int a = static_cast<int>(i % KP);
+    const long r = i / KP;
+    const int c = static_cast<int>(r % NP);
+    const long h = r / NP;
+    float s = 0.f;
+    if (c <= d && a < d) {
+      const long e = h * per_head + a * (d + 1) + c;
+      for (int k = 0; k < nrec; ++k) s += reinterpret_cast<const float*>(recs + k * rec_stride + sz_off)[e];
+      Sz[e] = s;
+    }
+    SzT[i] = __float2bfloat16_rn(s);
   }
 }
 

@@ -298,3 +298,27 @@ def test_workspace_regions_disjoint_and_inside(dtype):
             assert off % 256 == 0 and off + nbytes <= total, (name, off, nbytes, total)
         for (n1, o1, b1), (n2, o2, b2) in itertools.combinations(regs, 2):
             assert o1 + b1 <= o2 or o2 + b2 <= o1, (qkv, n1, o1, b1, n2, o2, b2)
+
+
+def test_band_entry_points_validate_on_the_host():
+    from linear_compressed_attention_b200 import seqpar
+    s = fake_struct(ws_bytes=1024)
+    L = seqpar._lib()
+    ok = seqpar.EditBand(64, 32, 32)
+    assert seqpar.band_workspace_bytes(64, 1152, 16, ok, s) > 0
+    assert seqpar.band_record_bytes(1152, 16, s) % 256 == 0
+    assert seqpar.band_record_bytes(1152, 16, s) >= 32 * 2 * 8 + 16 * 72 * 73 * 4
+    for bad in ((64, 1, 31), (64, 0, 33), (64, 40, 30), (0, 0, 1), (64, 0, 0)):
+        assert seqpar.band_workspace_bytes(64, 1152, 16, seqpar.EditBand(*bad), s) == 0, bad
+    assert seqpar.band_workspace_bytes(64, 1152, 16, seqpar.EditBand(63, 32, 31), s) > 0   # last band may be odd
+    f = fake_struct(dtype=bd.EDIT_F32, c_red=16, groups=4)
+    assert seqpar.band_workspace_bytes(16, 64, 2, seqpar.EditBand(16, 0, 8), f) == 0          # bf16 only
+    p = ctypes.c_void_p
+    rc = L.edit_attn_band_partials(p(0x200000), 64, 1152, 16, ctypes.byref(ok), ctypes.byref(s), p(0x300000), None)
+    assert rc == -5                                    # workspace too small, nothing launched
+    s = fake_struct()
+    rc = L.edit_attn_band_partials(p(0x200000), 64, 1152, 16, ctypes.byref(ok), ctypes.byref(s), p(0x300010), None)
+    assert rc == -3                                    # record not 256-byte aligned
+    rc = L.edit_attn_band_finish(p(0x200000), 64, 1152, 16, ctypes.byref(ok), ctypes.byref(s), p(0x300000), 0,
+                                 p(0x400000), None)
+    assert rc == -2                                    # no records
