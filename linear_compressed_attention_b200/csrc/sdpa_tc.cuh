@@ -97,9 +97,8 @@ __device__ __forceinline__ void tmem_ld_cols<32>(uint32_t taddr, float (&v)[32])
   }
 }
 
-// NSET: number of key sets (1: image rows, 2: prompt rows). With two sets
-// the first set's share is kept in registers, so S is read 32 columns at a
-// time (twice) to stay within the register budget of 10 warps.
+// NSET: number of key sets (1: image rows, 2: prompt rows); with two sets
+// the first set's share waits in registers for the second's.
 template <int D, int NSET>
 __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__ CUtensorMap mq,
                                                          const __grid_constant__ CUtensorMap mk1,
@@ -110,7 +109,8 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
   using Cfg = SdpaTcCfg<D>;
   constexpr int NBX = Cfg::NBX, KS = Cfg::KS, NPV = Cfg::NPV, STAGES = Cfg::STAGES, QB = Cfg::QB;
   constexpr int QBOX = Cfg::QBOX, VBOX = Cfg::VBOX, OC = Cfg::OC, OC0 = Cfg::OC0, OCH = Cfg::OCH;
-  constexpr int CW = NSET == 1 ? 64 : 32, NCW = 64 / CW;  // S columns read at a time
+  constexpr int CW = 32, NCW = 2;  // S columns read at a time (a chunk at a time keeps registers for the rest)
+  constexpr int NOLD = 16 * OCH / 8;  // 16-byte pieces of a thread's share of an output row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sQ = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = sQ + Cfg::Q_BYTES;
@@ -291,6 +291,20 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
       const long bh = it / qtiles;
       const int h = static_cast<int>(bh % p.heads), b = static_cast<int>(bh / p.heads);
       float sc = 0.f;
+      // the output row's current values (blended in at the end), fetched now
+      // so that their latency hides behind the item's tiles
+      const int r = qt * 128 + row;
+      __nv_bfloat16* og =
+          reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D + col0;
+      // (one key set only: with two, the registers hold the first set's share)
+      uint4 oldv[NSET == 1 ? NOLD : 1];
+      if (NSET == 1) {
+#pragma unroll
+        for (int k = 0; k < NOLD; ++k)
+          oldv[NSET == 1 ? k : 0] = (p.blend_in && r < p.Nq && col0 + 8 * k < D)
+                                        ? *reinterpret_cast<const uint4*>(og + 8 * k)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+      }
       for (int set = 0; set < NSET && ok; ++set) {
         const int n = set == 0 ? p.n1 : p.n2;
         const int Ts = set == 0 ? T1 : T2;
@@ -406,10 +420,7 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
         }
       }
       if (!ok) break;
-      const int r = qt * 128 + row;
       if (r < p.Nq) {
-        __nv_bfloat16* og =
-            reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long>(b) * p.Nq + r) * p.ldo + h * D + col0;
 #pragma unroll
         for (int c8 = 0; c8 < 16 * OCH; c8 += 8) {
           if (col0 + c8 < D) {
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
             for (int i = 0; i < 8; ++i)
               o[i] = NSET == 2 ? fmaf(R[c8 + i], sc, acc[NSET == 2 ? c8 + i : 0]) : R[c8 + i] * sc;
             if (p.blend_in) {
-              const uint4 old = *reinterpret_cast<const uint4*>(og + c8);
+              const uint4 old = NSET == 1 ? oldv[NSET == 1 ? c8 / 8 : 0] : *reinterpret_cast<const uint4*>(og + c8);
               const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
