@@ -184,11 +184,27 @@ EDIT_API int edit_attn_variant_forward(const void *x, int B, int H, int W, int C
                                        const edit_attn_weights *w, const edit_attn_variant *v, void *out,
                                        void *stream);
 
+/* Mixing weights of the MM-EDiT hybrid (eta_mode below).
+ *   EDIT_ETA_RATIO  the page's approximation: eta_I = eta_P = N_I / (N_I + N_T)
+ *                   (section "MM-EDiT", the sentence after eq. (A^Hybrid)).
+ *   EDIT_ETA_EXACT  the normaliser that ratio stands in for (the page calls it
+ *                   the exact computation but does not write it out; reading
+ *                   used here): each query normalises once over all keys.
+ *                   Image row i, head h: eta = (Q_i z + eps) /
+ *                   (Q_i z + eps + sum_P exp(q.k/sqrt(d))), i.e. image keys
+ *                   weighted by the linear kernel Q_i . K_j and prompt keys by
+ *                   exp(q . k / sqrt(d)) under one denominator. Prompt row:
+ *                   eta = Z_I / (Z_I + Z_P) with Z the sums of
+ *                   exp(q . k / sqrt(d)) over the image / prompt keys, i.e.
+ *                   one softmax over both key sets. */
+enum { EDIT_ETA_RATIO = 0, EDIT_ETA_EXACT = 1 };
+
 /* Weights of the MM-EDiT hybrid: the EDiT image-stream weights (`img`, its
  * dtype field is the dtype of everything) plus the prompt-token projections
  * tq_w, tk_w, tv_w [C][C] (torch Linear layout) and their biases [C]. The
  * workspace and side-stream fields of `img` are ignored; the ones here are
- * used. */
+ * used. eta_mode: EDIT_ETA_RATIO (0, the page's choice) or EDIT_ETA_EXACT;
+ * anything else returns EDIT_ERR_UNSUPPORTED. */
 typedef struct {
   edit_attn_weights img;
   const void *tq_w, *tq_b;
@@ -198,6 +214,7 @@ typedef struct {
   size_t workspace_bytes;
   void *side_stream;
   void *side_events[EDIT_SIDE_EVENTS];
+  int eta_mode;
 } mmedit_weights;
 
 EDIT_API size_t mmedit_workspace_bytes(int B, int H, int W, int N_T, int C, int heads, const mmedit_weights *w);

@@ -41,9 +41,13 @@ class EditAttnWeights(ctypes.Structure):
                [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS
 
 
+EDIT_ETA_RATIO, EDIT_ETA_EXACT = 0, 1
+
+
 class MMEditWeights(ctypes.Structure):
     _fields_ = [("img", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in TEXT_NAMES] + \
-               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS
+               [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS + \
+               [("eta_mode", ctypes.c_int)]
 
 
 class EditAttnVariant(ctypes.Structure):
@@ -285,12 +289,13 @@ class EditAttention:
 
     def __init__(self, arrays: dict, B: int, H: int, W: int, C: int, heads: int, dtype: str = "bf16",
                  n_txt: int = 0, mm: bool | None = None, device="cuda", variant: tuple | None = None,
-                 out_proj: bool = False, side: bool = True):
+                 out_proj: bool = False, side: bool = True, eta: str = "ratio"):
         """``variant`` = (q_proc, k_proc, v_proc) names ('cf', 'sc', 'none') and/or
         ``out_proj`` select edit_attn_variant_forward; weights a variant does
         not read are not copied to the device (NULL in the structs). With
         ``side`` the layer lends the library a side stream and its events
-        (created here, owned by this object) for the concurrent branches."""
+        (created here, owned by this object) for the concurrent branches.
+        ``eta`` ('ratio' | 'exact') picks MM-EDiT's mixing weights."""
         import torch
         self.torch = torch
         self.B, self.H, self.W, self.C, self.heads, self.n_txt = B, H, W, C, heads, int(n_txt or 0)
@@ -327,6 +332,8 @@ class EditAttention:
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.struct = make_weights_struct(self.w, self.code, workspace=self.workspace, **self.consts)
         self.mm_struct = make_mm_struct(self.struct, self.w, self.workspace) if self.mm else None
+        if self.mm_struct is not None:
+            self.mm_struct.eta_mode = {"ratio": EDIT_ETA_RATIO, "exact": EDIT_ETA_EXACT}[eta]
         self.side = make_side(device) if side and self.code == EDIT_BF16 else None
         self.set_side(self.side)
         self.layout = edit_attn_variant_workspace_layout(B, H, W, C, heads, self.struct, self.variant)

@@ -174,6 +174,7 @@ struct Plan {
   int NP, KP;     // apply operand padding: [S|z] rows (N) and K
   int bn_lin;     // tile N of the Linear GEMMs
   int npv = 0, nkpI = 0, nkpP = 0;  // MM-EDiT (bf16): [V | 1]^T rows per head, image / prompt keys padded to 128
+  bool exact_eta = false;  // MM-EDiT: exact mixing weights (the apply keeps its normaliser in `den`)
   bool fork = false;   // K/V branch on the calling thread's side stream, concurrent with the query branch
   int Wop, Mp;    // bf16 KV state: padded compressed grid width and token count
   int kv_kb;      // bf16 KV state: 64-token k-blocks per chunk
@@ -184,7 +185,7 @@ struct Plan {
   bool oproj = false;    // output Linear after the attention
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      fixpart, VTi, VTp, Y, total;
+      fixpart, VTi, VTp, den, Y, total;
 };
 
 int next_pow2(int v) {
@@ -328,6 +329,9 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   pl.Sz = take(static_cast<size_t>(B) * heads * pl.d * (pl.d + 1) * 4);
   pl.SzT = pl.bf16 ? take(static_cast<size_t>(B) * heads * pl.NP * pl.KP * 2) : 0;
   pl.QKVt = NT > 0 ? take(static_cast<size_t>(B) * NT * 3 * C * es) : 0;
+  // MM-EDiT: the linear part's normaliser Q z + eps per image row and head
+  // (read by the image rows' exact mixing weights)
+  pl.den = NT > 0 ? take(static_cast<size_t>(B) * pl.HW * heads * 4) : 0;
   // MM-EDiT softmax blocks (bf16): the image and prompt values as [V | 1]^T
   // operands, [B][heads][npv][keys padded to 128]
   pl.VTi = pl.VTp = 0;
@@ -1257,6 +1261,7 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
     p.ldo = pl.C;
     if (!map_out_heads(&p.out_map, out, pl.C, pl.HW, pl.B, pl.d)) return EDIT_ERR_CUDA;
     p.status = status;
+    p.den_out = pl.exact_eta ? reinterpret_cast<float*>(ws + pl.den) : nullptr;
     return gemm_apply(p, pl.NP, st);
   }
   const size_t smem = static_cast<size_t>(pl.d) * (pl.d + 1) * sizeof(float);
@@ -1265,7 +1270,8 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
     return EDIT_ERR_CUDA;
   launch_pdl(apply_simt_kernel<T>, dim3(dim3(ceil_div(pl.HW, 128), pl.heads, pl.B)), dim3(128), smem, st, 
       reinterpret_cast<const T*>(ws + pl.Q), reinterpret_cast<const float*>(ws + pl.Sz), static_cast<int>(pl.HW),
-      pl.C, pl.heads, w->attn_eps, static_cast<T*>(out));
+      pl.C, pl.heads, w->attn_eps, static_cast<T*>(out),
+      pl.exact_eta ? reinterpret_cast<float*>(ws + pl.den) : static_cast<float*>(nullptr));
   return last_launch();
 }
 
@@ -1403,6 +1409,8 @@ int mm_image_rows(const Plan& pl, uint8_t* ws, void* out_img, cudaStream_t st) {
     p.out = out_img;
     p.ldo = pl.C;
     p.status = reinterpret_cast<int*>(ws + pl.status);
+    p.exact = pl.exact_eta ? 1 : 0;
+    p.den = reinterpret_cast<const float*>(ws + pl.den);
     const SdpaSet prompt = {qkv + pl.C, 3L * pl.C, pl.NT, ws + pl.VTp, pl.nkpP};
     EDIT_TRY(sdpa_tc(ws + pl.Q, pl.C, static_cast<int>(pl.HW), prompt, nullptr, p, pl, st));
   } else {
@@ -1422,6 +1430,8 @@ int mm_image_rows(const Plan& pl, uint8_t* ws, void* out_img, cudaStream_t st) {
     a.w0 = static_cast<float>(eta);
     a.w1 = static_cast<float>(1.0 - eta);
     a.blend_in = 1;
+    a.exact = pl.exact_eta ? 1 : 0;
+    a.den = reinterpret_cast<const float*>(ws + pl.den);
     EDIT_TRY(sdpa_simt(a, pl.B, st));
   }
   stage_mark(10, st);
@@ -1441,6 +1451,7 @@ int mm_prompt_rows(const Plan& pl, uint8_t* ws, void* out_txt, cudaStream_t st) 
     p.out = out_txt;
     p.ldo = pl.C;
     p.status = reinterpret_cast<int*>(ws + pl.status);
+    p.exact = pl.exact_eta ? 1 : 0;
     const SdpaSet image = {ws + pl.K, pl.C, pl.M, ws + pl.VTi, pl.nkpI};
     const SdpaSet prompt = {qkv + pl.C, 3L * pl.C, pl.NT, ws + pl.VTp, pl.nkpP};
     EDIT_TRY(sdpa_tc(qkv, 3L * pl.C, pl.NT, image, &prompt, p, pl, st));
@@ -1464,6 +1475,7 @@ int mm_prompt_rows(const Plan& pl, uint8_t* ws, void* out_txt, cudaStream_t st) 
     t.d = pl.d;
     t.w1 = static_cast<float>(eta);
     t.w2 = static_cast<float>(1.0 - eta);
+    t.exact = pl.exact_eta ? 1 : 0;
     EDIT_TRY(sdpa_simt(t, pl.B, st));
   }
   stage_mark(11, st);
@@ -1769,6 +1781,8 @@ int mmedit_hybrid_forward(const void* x_img, const void* x_txt, int B, int H, in
       if (!aligned(p, 16)) return EDIT_ERR_ALIGN;
     }
   }
+  if (w->eta_mode != EDIT_ETA_RATIO && w->eta_mode != EDIT_ETA_EXACT) return EDIT_ERR_UNSUPPORTED;
+  pl.exact_eta = w->eta_mode == EDIT_ETA_EXACT && N_T > 0;
   uint8_t* ws = static_cast<uint8_t*>(w->workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return pl.bf16 ? run_mm<__nv_bfloat16>(x_img, x_txt, pl, w, ws, out_img, out_txt, st)

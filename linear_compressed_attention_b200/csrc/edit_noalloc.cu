@@ -72,7 +72,8 @@ int run(const void* q, const void* k, const void* v, int B, int N, int M, int C,
           cudaSuccess)
     return EDIT_ERR_CUDA;
   return launch(apply_simt_kernel<T>, dim3((N + 127) / 128, heads, B), dim3(128), asmem, st,
-                static_cast<const T*>(q), static_cast<const float*>(Sz), N, C, heads, eps, static_cast<T*>(out));
+                static_cast<const T*>(q), static_cast<const float*>(Sz), N, C, heads, eps, static_cast<T*>(out),
+                static_cast<float*>(nullptr));
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -42,6 +42,11 @@ struct SdpaTcParams {
   void* out;
   long ldo;
   int* status;
+  // exact mixing weights instead of w0..w2: one key set with blend_in mixes
+  // with the linear part, whose normaliser (Q z + eps) is den [img][row][head];
+  // two key sets mix by their softmax normalisers (one softmax over both)
+  int exact;
+  const float* den;
 };
 
 template <int D>
@@ -305,6 +310,9 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
                                         ? *reinterpret_cast<const uint4*>(og + 8 * k)
                                         : make_uint4(0u, 0u, 0u, 0u);
       }
+      // exact: log2 of the other part's normaliser (the linear part's den, one set)
+      float lz_other = 0.f, lz0 = 0.f;
+      if (NSET == 1 && p.exact && r < p.Nq) lz_other = log2f(p.den[(static_cast<long>(b) * p.Nq + r) * p.heads + h]);
       for (int set = 0; set < NSET && ok; ++set) {
         const int n = set == 0 ? p.n1 : p.n2;
         const int Ts = set == 0 ? T1 : T2;
@@ -412,8 +420,10 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
         named_bar_sync(1 + q4, 64);
         const float l = lsum[row];
         named_bar_sync(1 + q4, 64);  // (lsum is rewritten at the next set's end)
-        const float w = set == 0 ? p.w1 : p.w2;
+        const float w = p.exact ? 1.f : (set == 0 ? p.w1 : p.w2);
         sc = l > 0.f ? w / l : 0.f;
+        if (set == 0) lz0 = m_run + log2f(l);  // log2 of the set's normaliser sum_j exp(q.k_j / sqrt(d))
+        if (NSET == 2 && set == 1) lz_other = m_run + log2f(l);
         if (NSET == 2 && set == 0) {
 #pragma unroll
           for (int i = 0; i < 16 * OCH; ++i) acc[NSET == 2 ? i : 0] = R[i] * sc;
@@ -421,20 +431,32 @@ __global__ void __launch_bounds__(320, 1) sdpa_tc_kernel(const __grid_constant__
       }
       if (!ok) break;
       if (r < p.Nq) {
+        float w0e = p.w0;  // weight of the blended-in values (eta when exact)
 #pragma unroll
         for (int c8 = 0; c8 < 16 * OCH; c8 += 8) {
           if (col0 + c8 < D) {
             float o[8];
+            if (p.exact) {
+              // eta = A / (A + B) as 1 / (1 + 2^(log2 B - log2 A)): one set, A = the linear
+              // part's normaliser, B = this set's; two sets, A = the first's, B = the second's
+              const float eta = NSET == 2 ? 1.f / (1.f + exp2f(lz_other - lz0)) : 1.f / (1.f + exp2f(lz0 - lz_other));
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o[i] = NSET == 2 ? fmaf(R[c8 + i], sc, acc[NSET == 2 ? c8 + i : 0]) : R[c8 + i] * sc;
+              for (int i = 0; i < 8; ++i)
+                o[i] = NSET == 2 ? eta * acc[NSET == 2 ? c8 + i : 0] + (1.f - eta) * R[c8 + i] * sc
+                                 : (1.f - eta) * R[c8 + i] * sc;
+              w0e = eta;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = NSET == 2 ? fmaf(R[c8 + i], sc, acc[NSET == 2 ? c8 + i : 0]) : R[c8 + i] * sc;
+            }
             if (p.blend_in) {
               const uint4 old = NSET == 1 ? oldv[NSET == 1 ? c8 / 8 : 0] : *reinterpret_cast<const uint4*>(og + c8);
               const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                o[2 * i] = fmaf(p.w0, __uint_as_float(ow[i] << 16), o[2 * i]);
-                o[2 * i + 1] = fmaf(p.w0, __uint_as_float(ow[i] & 0xffff0000u), o[2 * i + 1]);
+                o[2 * i] = fmaf(w0e, __uint_as_float(ow[i] << 16), o[2 * i]);
+                o[2 * i + 1] = fmaf(w0e, __uint_as_float(ow[i] & 0xffff0000u), o[2 * i + 1]);
               }
             }
             uint4 wv;

@@ -28,6 +28,11 @@ struct SdpaParams {
   int Nq, heads, d;
   float w0, w1, w2;
   int blend_in;
+  // exact mixing weights instead of w0..w2 (one key set with blend_in: eta
+  // from den [b][row][head] = the linear part's normaliser; two key sets:
+  // eta from the two softmax normalisers)
+  int exact;
+  const float* den;
 };
 namespace {  // internal linkage: each translation unit that uses these keeps its own copy
 
@@ -996,7 +1001,7 @@ __global__ void kv_state_combine_pack_kernel(const float* __restrict__ part, int
 // One block per (token block, head, batch); [S_h | z_h] staged in shared memory.
 template <typename T>
 __global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restrict__ Sz, int N, int C, int heads,
-                                  float eps, T* __restrict__ out) {
+                                  float eps, T* __restrict__ out, float* __restrict__ den_out) {
   pdl_wait();
   const int d = C / heads;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -1011,6 +1016,7 @@ __global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restri
   float den = 0.f;
   for (int a = 0; a < d; ++a) den = fmaf(to_f32(q[a]), ap_sm[a * (d + 1) + d], den);
   const float inv = 1.f / (den + eps);
+  if (den_out) den_out[(static_cast<long>(b) * N + n) * heads + h] = den + eps;  // [b][n][head]
   for (int c = 0; c < d; ++c) {
     float s = 0.f;
     for (int a = 0; a < d; ++a) s = fmaf(to_f32(q[a]), ap_sm[a * (d + 1) + c], s);
@@ -1029,7 +1035,8 @@ __global__ void apply_simt_kernel(const T* __restrict__ Q, const float* __restri
 // q rows live in shared memory (qs, stride D + 1), one row per thread.
 template <typename T, int D>
 __device__ __forceinline__ void sdpa_one_set(const T* kb, const T* vb, long ld, int nk, const float* qrow,
-                                             bool active, float w, float (&res)[D], float* ks, float* vs, int h) {
+                                             bool active, float w, float (&res)[D], float* ks, float* vs, int h,
+                                             float* lz = nullptr) {
   constexpr int KT = 64;
   float m = -INFINITY, l = 0.f;
   float acc[D];
@@ -1067,6 +1074,7 @@ __device__ __forceinline__ void sdpa_one_set(const T* kb, const T* vb, long ld, 
   const float sc = l > 0.f ? w / l : 0.f;
 #pragma unroll
   for (int c = 0; c < D; ++c) res[c] = fmaf(acc[c], sc, res[c]);
+  if (lz) *lz = m + log2f(l);  // log2 of the set's normaliser sum_j exp(q.k_j / sqrt(d))
 }
 
 template <typename T, int D>
@@ -1083,22 +1091,32 @@ __global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
   float* qrow = qs + threadIdx.x * (D + 1);
   const T* qp = reinterpret_cast<const T*>(p.q) + (static_cast<long>(b) * p.Nq + (active ? i : 0)) * p.ldq + h * D;
   for (int c = 0; c < D; ++c) qrow[c] = active ? to_f32(qp[c]) * qscale : 0.f;
-  float res[D];
+  float res[D], res2[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c) res[c] = 0.f;
+  for (int c = 0; c < D; ++c) res[c] = res2[c] = 0.f;
+  float lz1 = 0.f, lz2 = 0.f;
   sdpa_one_set<T, D>(reinterpret_cast<const T*>(p.k1) + static_cast<long>(b) * p.n1 * p.ld1,
                      reinterpret_cast<const T*>(p.v1) + static_cast<long>(b) * p.n1 * p.ld1, p.ld1, p.n1, qrow,
-                     active, p.w1, res, ks, vs, h);
+                     active, p.exact ? 1.f : p.w1, res, ks, vs, h, &lz1);
   if (p.n2 > 0)
     sdpa_one_set<T, D>(reinterpret_cast<const T*>(p.k2) + static_cast<long>(b) * p.n2 * p.ld2,
                        reinterpret_cast<const T*>(p.v2) + static_cast<long>(b) * p.n2 * p.ld2, p.ld2, p.n2, qrow,
-                       active, p.w2, res, ks, vs, h);
+                       active, p.exact ? 1.f : p.w2, p.exact ? res2 : res, ks, vs, h, &lz2);
   if (!active) return;
   T* op = reinterpret_cast<T*>(p.out) + (static_cast<long>(b) * p.Nq + i) * p.ldo + h * D;
+  // exact: eta = A / (A + B) as 1 / (1 + 2^(log2 B - log2 A)); one set blends with the
+  // linear part (A = den), two sets share one softmax (A, B their normalisers)
+  float eta = 0.f;
+  if (p.exact) {
+    const float lza = p.n2 > 0 ? lz1 : log2f(p.den[(static_cast<long>(b) * p.Nq + i) * p.heads + h]);
+    eta = 1.f / (1.f + exp2f((p.n2 > 0 ? lz2 : lz1) - lza));
+  }
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     float v = res[c];
-    if (p.blend_in) v = fmaf(p.w0, to_f32(op[c]), v);
+    if (p.exact)
+      v = p.n2 > 0 ? eta * res[c] + (1.f - eta) * res2[c] : (1.f - eta) * res[c];
+    if (p.blend_in) v = fmaf(p.exact ? eta : p.w0, to_f32(op[c]), v);
     op[c] = from_f32<T>(v);
   }
 }

@@ -78,6 +78,7 @@ struct TcGemmParams {
   int bias_f32;
   int relu;
   int* status;
+  float* den_out;  // EPI_APPLY: when set, den + eps per row and head, [img][R][heads] fp32
 };
 
 template <int BN, int NSPLIT, int STAGES, int STG = 0>
@@ -281,6 +282,11 @@ __device__ __forceinline__ void epilogue_apply_staged(const TcGemmParams& p, con
   for (int i = 0; i < 16; ++i)
     if (i == d % 16) den = dv[i];
   const float inv = 1.f / (den + p.eps);
+  if (p.den_out) {
+    const int row = tc.r0 + q * 32 + lane;
+    if (tc.m_tile < p.num_m_tiles && row < p.R)
+      p.den_out[(static_cast<long>(tc.img) * p.R + row) * p.heads + tc.n_tile] = den + p.eps;
+  }
   if (lane == 0) bulk_wait_read<1>();
   __syncwarp();
   uint8_t* buf = stg + sbuf * (32 * d * 2);

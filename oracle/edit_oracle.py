@@ -19,7 +19,7 @@ Linear Compressed Attention" (ICCV 2025, arXiv 2503.16726), section
   depthwise conv of stride 2 (4x fewer key/value tokens).
 * Linear attention, eq. (y_i): y_i = Q_i (sum_j K_j^T V_j) / (Q_i sum_j K_j).
 * MM-EDiT, eq. (A^Hybrid) and the token-ratio approximation
-  eta = N_I / (N_I + N_T).
+  eta = N_I / (N_I + N_T), or the exact normaliser it stands in for.
 
 Everything is float64, computed from the given (possibly bf16-rounded) inputs
 with no intermediate rounding. Library primitives used as steps: numpy matmul
@@ -198,6 +198,27 @@ def sdpa(q, k, v, heads):
     return out
 
 
+def softmax_log_normaliser(q, k, heads):
+    """log sum_j exp(q . k_j / sqrt(d)) per query row and head, the
+    normaliser of sdpa() [R12]. q: [B, Nq, C]; k: [B, Nk, C]. Returns
+    [B, Nq, heads]; -inf for an empty key set."""
+    q, k = _f64(q), _f64(k)
+    B, Nq, C = q.shape
+    Nk = k.shape[1]
+    d = C // heads
+    out = np.full((B, Nq, heads), -np.inf)
+    if Nk == 0:
+        return out
+    scale = 1.0 / math.sqrt(d)
+    for bi in range(B):
+        for h in range(heads):
+            sl = slice(h * d, (h + 1) * d)
+            s = (q[bi, :, sl] @ k[bi, :, sl].T) * scale
+            m = s.max(axis=1)
+            out[bi, :, h] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    return out
+
+
 def mix_ratio(N_I, N_T):
     """eta = N_I / (N_I + N_T): eq. (A^Hybrid) normaliser approximated by
     the token-count ratio (eta_I and eta_P both take it [R13])."""
@@ -273,14 +294,23 @@ def edit_forward(x, H, W, w, heads, return_intermediates=False):
 # MM-EDiT hybrid
 # --------------------------------------------------------------------------
 
-def mmedit_forward(x_img, x_txt, H, W, w, heads, return_intermediates=False):
-    """MM-EDiT hybrid attention, eq. (A^Hybrid) with eta = N_I/(N_I+N_T).
+def mmedit_forward(x_img, x_txt, H, W, w, heads, return_intermediates=False, eta="ratio"):
+    """MM-EDiT hybrid attention, eq. (A^Hybrid).
 
     Image rows: eta * A_lin(Q_I, K_I, V_I) + (1 - eta) * A(Q_I, K_P, V_P).
     Text rows:  eta * A(Q_P, K_I, V_I)     + (1 - eta) * A(Q_P, K_P, V_P).
     Q_I, K_I, V_I are the EDiT query and the compressed keys/values; the
     prompt side uses plain Linear projections, A is softmax attention with
     scale 1/sqrt(d) normalised per block [R12].
+
+    eta="ratio": the page's approximation eta = N_I / (N_I + N_T) for both
+    rows [R13]. eta="exact": the normaliser the page says the ratio stands in
+    for [R22]: each query normalises once over all keys, image keys weighted by
+    the linear kernel (Q_i . K_j, plus the layer's eps) and prompt keys by
+    exp(q . k / sqrt(d)). Per query row and head that is
+      image rows: eta_i = (Q_i z + eps) / (Q_i z + eps + sum_P exp(q.k/sqrt(d)))
+      text rows:  eta_i = Z_I / (Z_I + Z_P), Z = sum_j exp(q.k_j/sqrt(d)) over
+                  the image (I) or prompt (P) keys, i.e. one softmax over both.
     Returns (out_img [B, N_I, C], out_txt [B, N_T, C]).
     """
     x_txt = _f64(x_txt)
@@ -291,12 +321,30 @@ def mmedit_forward(x_img, x_txt, H, W, w, heads, return_intermediates=False):
     Qp = linear(x_txt, w["tq_w"], w["tq_b"])
     Kp = linear(x_txt, w["tk_w"], w["tk_b"])
     Vp = linear(x_txt, w["tv_w"], w["tv_b"])
-    eta = mix_ratio(N_I, N_T)
     a_ip = sdpa(br["Q"], Kp, Vp, heads)
     a_pi = sdpa(Qp, br["K"], br["V"], heads)
     a_pp = sdpa(Qp, Kp, Vp, heads)
-    out_img = eta * y_lin + (1.0 - eta) * a_ip
-    out_txt = eta * a_pi + (1.0 - eta) * a_pp
+    if eta == "ratio":
+        eta = mix_ratio(N_I, N_T)
+        out_img = eta * y_lin + (1.0 - eta) * a_ip
+        out_txt = eta * a_pi + (1.0 - eta) * a_pp
+    elif eta == "exact":
+        d = C // heads
+        Q = br["Q"]
+        den = np.empty((B, N_I, heads))           # Q_i z + eps, the linear part's normaliser
+        for h in range(heads):
+            sl = slice(h * d, (h + 1) * d)
+            den[:, :, h] = np.einsum("bnc,bc->bn", Q[:, :, sl], z[:, h]) + w["attn_eps"]
+        # eta = A / (A + B) written as 1 / (1 + exp(log B - log A)), which stays finite
+        eta_i = 1.0 / (1.0 + np.exp(softmax_log_normaliser(Q, Kp, heads) - np.log(den)))
+        eta_p = 1.0 / (1.0 + np.exp(softmax_log_normaliser(Qp, Kp, heads) -
+                                    softmax_log_normaliser(Qp, br["K"], heads)))
+        per_col = lambda e: np.repeat(e, d, axis=2)  # noqa: E731  (heads -> their d columns)
+        out_img = per_col(eta_i) * y_lin + (1.0 - per_col(eta_i)) * a_ip
+        out_txt = per_col(eta_p) * a_pi + (1.0 - per_col(eta_p)) * a_pp
+        eta = (eta_i, eta_p)
+    else:
+        raise ValueError(f"eta must be 'ratio' or 'exact', not {eta!r}")
     if return_intermediates:
         br.update({"S": S, "z": z, "y": y_lin, "Qp": Qp, "Kp_txt": Kp,
                    "Vp_txt": Vp, "A_ip": a_ip, "A_pi": a_pi, "A_pp": a_pp,

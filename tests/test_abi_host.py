@@ -103,6 +103,9 @@ def test_mm_rejects_bad_arguments():
     assert call(xt=0) == -1
     assert call(ot=0x500002) == -3
     assert call(heads=12) == -8        # d = 128: no SDPA kernel for it
+    m.eta_mode = 7
+    assert call() == -8                # unknown mixing-weight mode
+    m.eta_mode = bd.EDIT_ETA_EXACT
     assert bd.mmedit_workspace_bytes(1, 64, 64, 333, 1536, 24, m) > bd.mmedit_workspace_bytes(1, 64, 64, 0, 1536, 24, m)
 
 

@@ -20,9 +20,9 @@ def max_rel(g, o):
     return float(np.max(np.abs(g - o)) / max(np.max(np.abs(o)), 1e-30))
 
 
-def gpu_layer(cfg, d):
+def gpu_layer(cfg, d, eta="ratio"):
     layer = bd.EditAttention(d, cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"], cfg["dtype"],
-                             n_txt=cfg.get("n_txt") or 0, mm=cfg.get("n_txt") is not None)
+                             n_txt=cfg.get("n_txt") or 0, mm=cfg.get("n_txt") is not None, eta=eta)
     x = torch.from_numpy(d["x"]).to("cuda", layer.tdtype)
     return layer, x
 
@@ -149,14 +149,14 @@ def test_shared_kv_weights_literal_reading():
 
 # ------------------------------------------------------------------ MM-EDiT
 
-def check_mm(cfg, d):
-    layer, xi = gpu_layer(cfg, d)
+def check_mm(cfg, d, eta="ratio"):
+    layer, xi = gpu_layer(cfg, d, eta)
     nt = cfg.get("n_txt") or 0
     xt = torch.from_numpy(d["x_txt"]).to("cuda", layer.tdtype) if nt else None
     oi, ot = layer.forward_mm(xi, xt)
     torch.cuda.synchronize()
     assert layer.status() == 0
-    ri, rt = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, cfg["heads"])
+    ri, rt = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, cfg["heads"], eta=eta)
     tol = TOL[cfg["dtype"]]
     errs = {"img": max_rel(oi.float().cpu().numpy(), ri)}
     if nt:
@@ -179,6 +179,18 @@ MM_SMALL = [
 def test_mm_small(shape):
     cfg = dict(shape, seed=31, nonzero_affine=True)
     check_mm(cfg, make_inputs(**cfg))
+
+
+@pytest.mark.parametrize("shape", MM_SMALL, ids=lambda s: f"{s['dtype']}-{s['C']}-{s['n_txt']}")
+def test_mm_small_exact_eta(shape):
+    """The exact mixing weights (one normalisation per query over all keys)."""
+    cfg = dict(shape, seed=33, nonzero_affine=True)
+    check_mm(cfg, make_inputs(**cfg), eta="exact")
+
+
+def test_mm_workload_exact_eta():
+    cfg = dict(WORKLOADS["mm1024"])
+    print("mm1024 exact", check_mm(cfg, make_inputs(**cfg), eta="exact"))
 
 
 def test_mm_without_prompt_tokens_is_edit():

@@ -352,6 +352,55 @@ def test_mmedit_without_text_is_edit():
     assert np.array_equal(oi, y)
 
 
+def test_mmedit_exact_eta_prompt_rows_are_one_softmax_over_all_keys():
+    """Exact eta, prompt rows: one softmax over the image and prompt keys
+    together (PyTorch CPU fp64 scaled_dot_product_attention on the
+    concatenated key and value sets)."""
+    cfg = small_cfg(n_txt=5)
+    d = make_inputs(**cfg)
+    B, C, heads = cfg["B"], cfg["C"], cfg["heads"]
+    _, op, it = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, heads, return_intermediates=True,
+                                 eta="exact")
+    dh = C // heads
+    sh = lambda a: torch.as_tensor(a).reshape(B, -1, heads, dh).transpose(1, 2)  # noqa: E731
+    k = np.concatenate([it["K"], it["Kp_txt"]], axis=1)
+    v = np.concatenate([it["V"], it["Vp_txt"]], axis=1)
+    ref = F.scaled_dot_product_attention(sh(it["Qp"]), sh(k), sh(v)).transpose(1, 2).reshape(B, -1, C).numpy()
+    assert rel(op, ref) < 1e-12
+
+
+def test_mmedit_exact_eta_image_rows_brute_force():
+    """Exact eta, image rows, pure-Python loops on a tiny case: every key
+    weighted once, image keys by Q_i . K_j, prompt keys by
+    exp(q . k / sqrt(d)), one normalisation with the layer's eps:
+    out_i = (sum_j w_j v_j) / (sum_j w_j + eps)."""
+    cfg = dict(B=1, H=3, W=3, C=8, c_red=4, gn_groups=2, heads=2, dtype="f32", seed=71, n_txt=3,
+               nonzero_affine=True)
+    d = make_inputs(**cfg)
+    oi, _, it = O.mmedit_forward(d["x"], d["x_txt"], 3, 3, d, 2, return_intermediates=True, eta="exact")
+    Q, K, V, Kp, Vp = (np.asarray(it[n])[0] for n in ("Q", "K", "V", "Kp_txt", "Vp_txt"))
+    dh, eps = 4, d["attn_eps"]
+    for i in range(Q.shape[0]):
+        for h in range(2):
+            cols = range(h * dh, (h + 1) * dh)
+            dot = lambda a, b: sum(a[c] * b[c] for c in cols)  # noqa: E731
+            ws = [dot(Q[i], K[j]) for j in range(K.shape[0])] + \
+                 [math.exp(dot(Q[i], Kp[j]) / math.sqrt(dh)) for j in range(Kp.shape[0])]
+            vs = [V[j] for j in range(V.shape[0])] + [Vp[j] for j in range(Vp.shape[0])]
+            tot = sum(ws) + eps
+            for c in cols:
+                want = sum(wj * vj[c] for wj, vj in zip(ws, vs)) / tot
+                assert abs(oi[0, i, c] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_mmedit_exact_eta_without_prompt_tokens_is_edit():
+    cfg = small_cfg(n_txt=0)
+    d = make_inputs(**cfg)
+    oi, op = O.mmedit_forward(d["x"], d["x_txt"], cfg["H"], cfg["W"], d, cfg["heads"], eta="exact")
+    assert np.array_equal(oi, O.edit_forward(d["x"], cfg["H"], cfg["W"], d, cfg["heads"]))
+    assert op.shape == (cfg["B"], 0, cfg["C"])
+
+
 # ------------------------------------------ planted mistakes must be caught
 
 def _mutant_layer(monkeypatch, name, fn):
