@@ -15,9 +15,10 @@ tv_w (fan_in C). Biases are 0, GroupNorm gamma = 1 and beta = 0, unless
 stream above is unchanged). ``variant_weights`` adds, drawn after all of
 that, the key's own ConvFusion weights kcf3_w, kcf1_w (fan_in 9C, Cr) and the
 output projection o_w (fan_in C), then (with ``nonzero_affine``) their
-biases and GroupNorm affine. bf16 workloads round every array once to bf16
-(round-to-nearest-even) and hand out float32 arrays holding exactly those
-values.
+biases and GroupNorm affine. ``dit_block`` (dict with n_cap, hidden) adds,
+after all of that, the DiT block's inputs and weights (see make_inputs). bf16
+workloads round every array once to bf16 (round-to-nearest-even) and hand out
+float32 arrays holding exactly those values.
 """
 from __future__ import annotations
 
@@ -57,7 +58,8 @@ def _normal(rng, shape, var):
 
 
 def make_inputs(B, H, W, C, c_red, gn_groups, heads, seed, dtype="bf16",
-                outliers=False, n_txt=None, nonzero_affine=False, variant_weights=False, **_ignored):
+                outliers=False, n_txt=None, nonzero_affine=False, variant_weights=False, dit_block=None,
+                **_ignored):
     """Draw one workload. Returns a dict with x (and x_txt) plus every weight
     under the C header's names and the declared constants; arrays are float32
     (bf16-exact for bf16 workloads). Shapes: x [B, H*W, C]; cf3_w [Cr, 3, 3, C];
@@ -116,9 +118,34 @@ def make_inputs(B, H, W, C, c_red, gn_groups, heads, seed, dtype="bf16",
             d["kgn_beta"] = _normal(rng, (c_red,), 0.01)
             d["kcf1_b"] = _normal(rng, (C,), 0.01)
             d["o_b"] = _normal(rng, (C,), 0.01)
+    if dit_block:
+        # the DiT block around the attention: caption tokens y [B, n_cap, C], the
+        # sample's timestep modulation t6 [B, 6, C] (N(0, 0.1^2)), the block's
+        # modulation table sst [6, C] (N(0, 1/C)), the attention's output Linear,
+        # the cross-attention Linears and the MLP (hidden units), fan-in variances
+        n_cap, hidden = dit_block["n_cap"], dit_block["hidden"]
+        d["y"] = rng.standard_normal((B, n_cap, C), dtype=np.float32)
+        d["t6"] = _normal(rng, (B, 6, C), 0.01)
+        d["sst"] = _normal(rng, (6, C), 1.0 / C)
+        if "o_w" not in d:
+            d["o_w"] = _normal(rng, (C, C), 1.0 / C)
+            d["o_b"] = zeros(C)
+        for n in ("cq_w", "ck_w", "cv_w", "co_w"):
+            d[n] = _normal(rng, (C, C), 1.0 / C)
+        d["fc1_w"] = _normal(rng, (hidden, C), 1.0 / C)
+        d["fc2_w"] = _normal(rng, (C, hidden), 1.0 / hidden)
+        for n in ("cq_b", "ck_b", "cv_b", "co_b", "fc2_b"):
+            d[n] = zeros(C)
+        d["fc1_b"] = zeros(hidden)
+        if nonzero_affine:
+            for n in ("cq_b", "ck_b", "cv_b", "co_b", "fc2_b", "o_b"):
+                d[n] = _normal(rng, (C,), 0.01)
+            d["fc1_b"] = _normal(rng, (hidden,), 0.01)
     if dtype == "bf16":
         d = {k: round_bf16(v) for k, v in d.items()}
     d.update(dict(c_red=c_red, gn_groups=gn_groups, **DECLARED))
+    if dit_block:
+        d["ln_eps"] = 1e-6
     return d
 
 

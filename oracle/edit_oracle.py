@@ -419,3 +419,50 @@ def edit_variant_forward(x, H, W, w, heads, q_proc=PROC_CF, k_proc=PROC_SC, v_pr
         it.update({"Q": Q, "K": K, "V": V, "S": S, "z": z, "y": y})
         return out, it
     return out
+
+
+# --------------------------------------------------------------------------
+# The DiT block around the attention [R23]
+# --------------------------------------------------------------------------
+
+def layer_norm(x, eps):
+    """LayerNorm over the last axis without affine weights: (x - mean) /
+    sqrt(biased var + eps)."""
+    x = _f64(x)
+    mean = x.mean(axis=-1, keepdims=True)
+    var = ((x - mean) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mean) / np.sqrt(var + eps)
+
+
+def gelu_tanh(x):
+    """GELU with the tanh approximation: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = _f64(x)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def dit_block_forward(x, y, t6, H, W, w, heads):
+    """One text-to-image DiT block of the PixArt-Sigma kind with EDiT as its
+    self-attention [R23] (the notes page: EDiT replaces the attention of
+    PixArt-Sigma's blocks; the block itself is that model's, not the page's).
+
+    x: [B, N, C] image tokens; y: [B, N_T, C] caption tokens; t6: [B, 6, C]
+    the sample's timestep modulation. With m = sst + t6 split into
+    (shift_a, scale_a, gate_a, shift_f, scale_f, gate_f):
+      x1 = x + gate_a * (EDiT(LN(x) (1 + scale_a) + shift_a) o_w^T + o_b)
+      x2 = x1 + (A(x1 cq_w^T + cq_b, y ck_w^T + ck_b, y cv_w^T + cv_b) co_w^T + co_b)
+      out = x2 + gate_f * (GELU(LN(x2) (1 + scale_f) + shift_f) fc1_w^T + fc1_b) fc2_w^T + fc2_b)
+    with LN the LayerNorm without affine (eps w["ln_eps"]), A softmax attention
+    per head (scale 1/sqrt(d)) and GELU the tanh form."""
+    x, y, t6 = _f64(x), _f64(y), _f64(t6)
+    m = _f64(w["sst"])[None] + t6                      # [B, 6, C]
+    sh_a, sc_a, g_a, sh_f, sc_f, g_f = (m[:, k][:, None, :] for k in range(6))
+    h1 = layer_norm(x, w["ln_eps"]) * (1.0 + sc_a) + sh_a
+    a = linear(edit_forward(h1, H, W, w, heads), w["o_w"], w["o_b"])
+    x1 = x + g_a * a
+    q = linear(x1, w["cq_w"], w["cq_b"])
+    k = linear(y, w["ck_w"], w["ck_b"])
+    v = linear(y, w["cv_w"], w["cv_b"])
+    x2 = x1 + linear(sdpa(q, k, v, heads), w["co_w"], w["co_b"])
+    h2 = layer_norm(x2, w["ln_eps"]) * (1.0 + sc_f) + sh_f
+    f = gelu_tanh(linear(h2, w["fc1_w"], w["fc1_b"]))
+    return x2 + g_f * linear(f, w["fc2_w"], w["fc2_b"])

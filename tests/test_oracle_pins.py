@@ -583,3 +583,66 @@ def test_variant_planted_mistake_is_caught(monkeypatch, mutant):
     assert rel(O.edit_variant_forward(d["x"], 4, 5, d, cfg["heads"], *qkv, out_proj=True), ref) < 1e-11
     monkeypatch.setattr(O, name, make(getattr(O, name)))
     assert rel(O.edit_variant_forward(d["x"], 4, 5, d, cfg["heads"], *qkv, out_proj=True), ref) > 1e-3, mutant
+
+
+# ------------------------------------------------ the DiT block around EDiT
+
+DIT = dict(n_cap=7, hidden=64)
+
+
+def _torch_dit_block(d, cfg):
+    """The block from PyTorch CPU float64 library routines: layer_norm,
+    linear, scaled_dot_product_attention, gelu(approximate='tanh'), and the
+    EDiT layer's own torch composition for the self-attention."""
+    B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+    t = {k: torch.tensor(np.asarray(v, np.float64)) for k, v in d.items() if isinstance(v, np.ndarray)}
+    m = t["sst"][None] + t["t6"]
+    sh_a, sc_a, g_a, sh_f, sc_f, g_f = (m[:, k][:, None, :] for k in range(6))
+    x = t["x"]
+    h1 = F.layer_norm(x, (C,), eps=d["ln_eps"]) * (1 + sc_a) + sh_a
+    y_att, _, _, _ = _torch_edit_layer(dict(d, x=h1.numpy()), cfg)
+    x1 = x + g_a * F.linear(torch.tensor(y_att), t["o_w"], t["o_b"])
+    dh = C // heads
+    sh = lambda a: a.reshape(B, -1, heads, dh).transpose(1, 2)  # noqa: E731
+    q = F.linear(x1, t["cq_w"], t["cq_b"])
+    k = F.linear(t["y"], t["ck_w"], t["ck_b"])
+    v = F.linear(t["y"], t["cv_w"], t["cv_b"])
+    a = F.scaled_dot_product_attention(sh(q), sh(k), sh(v)).transpose(1, 2).reshape(B, -1, C)
+    x2 = x1 + F.linear(a, t["co_w"], t["co_b"])
+    h2 = F.layer_norm(x2, (C,), eps=d["ln_eps"]) * (1 + sc_f) + sh_f
+    f = F.gelu(F.linear(h2, t["fc1_w"], t["fc1_b"]), approximate="tanh")
+    return (x2 + g_f * F.linear(f, t["fc2_w"], t["fc2_b"])).numpy()
+
+
+@pytest.mark.parametrize("cfgkw", [dict(), dict(H=5, W=7, B=1), dict(H=4, W=4, heads=4)])
+def test_dit_block_vs_torch_composition(cfgkw):
+    cfg = small_cfg(**cfgkw)
+    d = make_inputs(**cfg, dit_block=DIT)
+    out = O.dit_block_forward(d["x"], d["y"], d["t6"], cfg["H"], cfg["W"], d, cfg["heads"])
+    assert rel(out, _torch_dit_block(d, cfg)) < 1e-11
+
+
+def test_layer_norm_and_gelu_vs_torch():
+    x = np.random.default_rng(5).standard_normal((3, 7, 24))
+    assert rel(O.layer_norm(x, 1e-6), F.layer_norm(torch.tensor(x), (24,), eps=1e-6).numpy()) < 1e-13
+    assert rel(O.gelu_tanh(x), F.gelu(torch.tensor(x), approximate="tanh").numpy()) < 1e-13
+
+
+def test_dit_block_special_cases():
+    """Zero gates and a zero cross-attention output Linear leave x unchanged;
+    with zero gates only, the block is x plus the cross-attention alone."""
+    cfg = small_cfg()
+    d = make_inputs(**cfg, dit_block=DIT)
+    H, W, heads = cfg["H"], cfg["W"], cfg["heads"]
+    z = dict(d)
+    z["t6"] = d["t6"].copy()
+    z["t6"][:, 2] = -d["sst"][2]
+    z["t6"][:, 5] = -d["sst"][5]
+    z["co_w"] = np.zeros_like(d["co_w"])
+    z["co_b"] = np.zeros_like(d["co_b"])
+    assert np.array_equal(O.dit_block_forward(d["x"], d["y"], z["t6"], H, W, z, heads), np.asarray(d["x"], float))
+    z2 = dict(z, co_w=d["co_w"], co_b=d["co_b"])
+    q = O.linear(d["x"], d["cq_w"], d["cq_b"])
+    k, v = O.linear(d["y"], d["ck_w"], d["ck_b"]), O.linear(d["y"], d["cv_w"], d["cv_b"])
+    want = np.asarray(d["x"], float) + O.linear(O.sdpa(q, k, v, heads), d["co_w"], d["co_b"])
+    assert rel(O.dit_block_forward(d["x"], d["y"], z2["t6"], H, W, z2, heads), want) < 1e-13
