@@ -266,6 +266,45 @@ EDIT_API int edit_attn_workspace_layout(int B, int H, int W, int C, int heads, c
 EDIT_API int edit_attn_variant_workspace_layout(int B, int H, int W, int C, int heads, const edit_attn_weights *w,
                                                 const edit_attn_variant *v, edit_ws_layout *layout);
 
+/* The DiT block around the attention (a text-to-image transformer block of
+ * the PixArt-Sigma kind with EDiT as its self-attention; the notes page says
+ * EDiT replaces the attention of PixArt-Sigma's blocks, section 整体框架 /
+ * overall framework, but does not spell the block out: the block used here is
+ * that model family's, read as follows).
+ *   m = sst + t6[b] = (shift_a, scale_a, gate_a, shift_f, scale_f, gate_f)
+ *   x1 = x + gate_a * (EDiT(LN(x) (1 + scale_a) + shift_a) o_w^T + o_b)
+ *   x2 = x1 + softmax-attention(x1 cq_w^T + cq_b, y ck_w^T + ck_b, y cv_w^T + cv_b) co_w^T + co_b
+ *   out = x2 + gate_f * (GELU(LN(x2) (1 + scale_f) + shift_f) fc1_w^T + fc1_b) fc2_w^T + fc2_b)
+ * LN: LayerNorm over C without affine weights (eps ln_eps); GELU: the tanh
+ * form; the cross-attention is per head with scale 1/sqrt(d), over the N_T
+ * caption tokens y. Shapes (row-major, dtype of attn.dtype):
+ *   x, out [B, H*W, C]; y [B, N_T, C] (N_T >= 1); t6 [B, 6, C] (the sample's
+ *   timestep modulation); sst [6][C]; o_w, cq_w, ck_w, cv_w, co_w [C][C] and
+ *   their biases [C]; fc1_w [hidden][C], fc1_b [hidden], fc2_w [C][hidden],
+ *   fc2_b [C].
+ * The EDiT attention weights and constants are those of `attn` (its workspace
+ * and side-stream fields are ignored; the ones here are used). bf16 needs
+ * hidden % 128 == 0 and head widths d of 32, 64 or 72 (the softmax kernel's);
+ * other shapes return EDIT_ERR_UNSUPPORTED. */
+typedef struct {
+  edit_attn_weights attn;
+  const void *o_w, *o_b;
+  const void *sst;
+  const void *cq_w, *cq_b, *ck_w, *ck_b, *cv_w, *cv_b, *co_w, *co_b;
+  const void *fc1_w, *fc1_b, *fc2_w, *fc2_b;
+  int hidden;
+  float ln_eps;
+  void *workspace;
+  size_t workspace_bytes;
+  void *side_stream;
+  void *side_events[EDIT_SIDE_EVENTS];
+} edit_dit_block_weights;
+
+EDIT_API size_t edit_dit_block_workspace_bytes(int B, int H, int W, int N_T, int C, int heads,
+                                               const edit_dit_block_weights *w);
+EDIT_API int edit_dit_block_forward(const void *x, const void *y, const void *t6, int B, int H, int W, int N_T, int C,
+                                    int heads, const edit_dit_block_weights *w, void *out, void *stream);
+
 /* Row bands: one image split over several ranks (sequence parallelism).
  *
  * The notes page scales EDiT to 8192 x 8192 images (section 延迟分析, the

@@ -24,7 +24,8 @@ EXPORTS = ("edit_attn_workspace_bytes", "edit_attn_forward", "mmedit_workspace_b
            "edit_attn_set_stage_events", "edit_attn_kernel_launches", "edit_linear_attention_noalloc",
            "edit_attn_variant_workspace_bytes", "edit_attn_variant_forward", "edit_attn_variant_workspace_layout",
            "edit_attn_set_wait_drill", "edit_attn_band_workspace_bytes", "edit_attn_band_record_bytes",
-           "edit_attn_band_partials", "edit_attn_band_finish")
+           "edit_attn_band_partials", "edit_attn_band_finish", "edit_dit_block_workspace_bytes",
+           "edit_dit_block_forward")
 STAGE_EVENTS_EDIT, STAGE_EVENTS_MM = 9, 12
 PROC = {"none": 0, "cf": 1, "sc": 2}
 VARIANT_NAMES = ("kcf3_w", "kcf3_b", "kgn_gamma", "kgn_beta", "kcf1_w", "kcf1_b", "o_w", "o_b")
@@ -48,6 +49,16 @@ class MMEditWeights(ctypes.Structure):
     _fields_ = [("img", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in TEXT_NAMES] + \
                [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS + \
                [("eta_mode", ctypes.c_int)]
+
+
+DIT_NAMES = ("o_w", "o_b", "sst", "cq_w", "cq_b", "ck_w", "ck_b", "cv_w", "cv_b", "co_w", "co_b",
+             "fc1_w", "fc1_b", "fc2_w", "fc2_b")
+
+
+class DitBlockWeights(ctypes.Structure):
+    _fields_ = [("attn", EditAttnWeights)] + [(n, ctypes.c_void_p) for n in DIT_NAMES] + \
+               [("hidden", ctypes.c_int), ("ln_eps", ctypes.c_float), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)] + _SIDE_FIELDS
 
 
 class EditAttnVariant(ctypes.Structure):
@@ -96,6 +107,11 @@ def lib():
     L.edit_attn_set_wait_drill.restype = i
     L.edit_linear_attention_noalloc.argtypes = [p, p, p, i, i, i, i, i, i, ctypes.c_float, p, p]
     L.edit_linear_attention_noalloc.restype = i
+    DW = ctypes.POINTER(DitBlockWeights)
+    L.edit_dit_block_workspace_bytes.argtypes = [i, i, i, i, i, i, DW]
+    L.edit_dit_block_workspace_bytes.restype = sz
+    L.edit_dit_block_forward.argtypes = [p, p, p, i, i, i, i, i, i, DW, p, p]
+    L.edit_dit_block_forward.restype = i
     V = ctypes.POINTER(EditAttnVariant)
     L.edit_attn_variant_workspace_bytes.argtypes = [i, i, i, i, i, W, V]
     L.edit_attn_variant_workspace_bytes.restype = sz
@@ -379,3 +395,59 @@ class EditAttention:
         n = int(np.prod(shape))
         es = torch.empty((), dtype=dt).element_size()
         return self.workspace[off:off + n * es].view(dt).view(*shape)
+
+
+# ----------------------------------------------------------- DiT block
+def edit_dit_block_workspace_bytes(B, H, W, N_T, C, heads, weights: DitBlockWeights) -> int:
+    return int(lib().edit_dit_block_workspace_bytes(B, H, W, N_T, C, heads, ctypes.byref(weights)))
+
+
+def edit_dit_block_forward(x, y, t6, B, H, W, N_T, C, heads, weights: DitBlockWeights, out, stream=None) -> int:
+    return int(lib().edit_dit_block_forward(_ptr(x), _ptr(y), _ptr(t6), B, H, W, N_T, C, heads,
+                                            ctypes.byref(weights), _ptr(out), _stream(stream)))
+
+
+class DitBlock:
+    """One DiT block (EDiT self-attention, cross-attention over the caption
+    tokens, MLP) with weights and workspace on a CUDA device; ``arrays`` is
+    the synthetic-input dict drawn with ``dit_block=...``."""
+
+    def __init__(self, arrays: dict, B: int, H: int, W: int, N_T: int, C: int, heads: int, dtype: str = "bf16",
+                 device="cuda", side: bool = True):
+        import torch
+        self.torch = torch
+        self.B, self.H, self.W, self.N_T, self.C, self.heads = B, H, W, N_T, C, heads
+        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        code = EDIT_BF16 if dtype == "bf16" else EDIT_F32
+        names = WEIGHT_NAMES + DIT_NAMES
+        self.w = {n: torch.from_numpy(np.ascontiguousarray(arrays[n])).to(device=device, dtype=self.tdtype)
+                  for n in names}
+        consts = dict(c_red=arrays["c_red"], gn_groups=arrays["gn_groups"], gn_eps=arrays["gn_eps"],
+                      leaky_slope=arrays["leaky_slope"], attn_eps=arrays["attn_eps"])
+        s = DitBlockWeights()
+        s.attn = make_weights_struct(self.w, code, **consts)
+        for n in DIT_NAMES:
+            setattr(s, n, self.w[n].data_ptr())
+        s.hidden = int(arrays["fc1_w"].shape[0])
+        s.ln_eps = float(arrays["ln_eps"])
+        nbytes = edit_dit_block_workspace_bytes(B, H, W, N_T, C, heads, s)
+        if nbytes == 0:
+            raise ValueError("shape/dtype rejected by the DiT block workspace query")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        s.workspace = self.workspace.data_ptr()
+        s.workspace_bytes = nbytes
+        self.struct = s
+        self.side = make_side(device) if side and code == EDIT_BF16 else None
+        set_side(self.struct, self.side)
+
+    def forward(self, x, y, t6, out=None, stream=None):
+        if out is None:
+            out = self.torch.empty_like(x)
+        rc = edit_dit_block_forward(x, y, t6, self.B, self.H, self.W, self.N_T, self.C, self.heads, self.struct, out,
+                                    stream)
+        if rc != 0:
+            raise EditError(rc)
+        return out
+
+    def status(self, stream=None) -> int:
+        return edit_attn_read_status(self.workspace, stream)

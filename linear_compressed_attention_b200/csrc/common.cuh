@@ -59,6 +59,15 @@ __device__ __forceinline__ void record_wait_site(int* status, int site, int tile
   }
 }
 
+// Epilogue activation of the GEMMs: 0 none, 1 ReLU, 2 GELU in its tanh form
+// 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+enum { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2 };
+__device__ __forceinline__ float act_apply(float v, int mode) {
+  if (mode == ACT_RELU) return fmaxf(v, 0.f);
+  if (mode == ACT_GELU) return 0.5f * v * (1.f + tanhf(0.7978845608028654f * fmaf(0.044715f * v * v, v, v)));
+  return v;
+}
+
 // ----------------------------------------------------------------- PDL
 // Programmatic dependent launch: every kernel of the library calls this before
 // touching memory written by the kernel before it in the stream (a no-op when

@@ -1705,6 +1705,163 @@ int band_checks(const void* x, const edit_attn_weights* w, const BandPlan& bp) {
   return EDIT_OK;
 }
 
+// ------------------------------------------------------------ DiT block
+// The block around the attention: LayerNorm modulation, the EDiT layer with
+// its output Linear, gated residuals, cross-attention over the caption tokens
+// and the tanh-GELU MLP. Workspace: the EDiT layer's (plan `pa`, its variant
+// with the output Linear) at offset 0, then the block's token buffers.
+struct DitPlan {
+  Plan pa;
+  int NT, hidden, nkp;
+  size_t h1, x1, q, kv, vt, att, c, x2, h2, f, m, total;
+};
+
+edit_attn_variant dit_attn_variant(const edit_dit_block_weights* w) {
+  edit_attn_variant v;
+  std::memset(&v, 0, sizeof(v));
+  v.q_proc = EDIT_PROC_CF;
+  v.k_proc = EDIT_PROC_SC;
+  v.v_proc = EDIT_PROC_SC;
+  v.o_w = w->o_w;
+  v.o_b = w->o_b;
+  return v;
+}
+
+int make_dit_plan(int B, int H, int W, int NT, int C, int heads, const edit_dit_block_weights* w, DitPlan& dp) {
+  if (!w) return EDIT_ERR_NULL;
+  const edit_attn_variant var = dit_attn_variant(w);
+  EDIT_TRY_CHECK(make_plan(B, H, W, C, heads, 0, &w->attn, dp.pa, &var));
+  const Plan& pa = dp.pa;
+  if (NT < 1 || w->hidden < 1) return EDIT_ERR_SHAPE;
+  if (!(pa.d == 32 || pa.d == 64 || pa.d == 72)) return EDIT_ERR_UNSUPPORTED;
+  if (pa.bf16 && w->hidden % 128 != 0) return EDIT_ERR_UNSUPPORTED;
+  if (!pa.bf16 && (C % 8 != 0 || w->hidden % 4 != 0)) return EDIT_ERR_UNSUPPORTED;
+  if (C > 2048) return EDIT_ERR_UNSUPPORTED;  // the residual / LayerNorm kernel keeps a row in registers
+  dp.NT = NT;
+  dp.hidden = w->hidden;
+  dp.nkp = (NT + 127) / 128 * 128;
+  const size_t es = pa.es, tok = static_cast<size_t>(B) * pa.HW;
+  size_t off = pa.total;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  dp.h1 = take(tok * C * es);
+  dp.x1 = take(tok * C * es);
+  dp.q = take(tok * C * es);
+  dp.kv = take(static_cast<size_t>(B) * NT * 2 * C * es);
+  dp.vt = pa.bf16 ? take(static_cast<size_t>(B) * heads * (pa.d + 1 <= 48 ? 48 : 80) * dp.nkp * 2) : 0;
+  dp.att = take(tok * C * es);
+  dp.c = take(tok * C * es);
+  dp.x2 = take(tok * C * es);
+  dp.h2 = take(tok * C * es);
+  dp.f = take(tok * w->hidden * es);
+  dp.m = take(tok * C * es);
+  dp.total = off;
+  return EDIT_OK;
+}
+
+template <typename T>
+int dit_residual_ln(const Plan& pl, const void* base, const void* delta, const void* sst, const void* t6, int kg,
+                    int ks, int kh, float eps, void* r_out, void* h_out, cudaStream_t st) {
+  const long rows = static_cast<long>(pl.B) * pl.HW;
+  launch_pdl(dit_residual_ln_kernel<T>, dim3(grid_for(rows * 32, 256)), dim3(256), 0, st,
+             static_cast<const T*>(base), static_cast<const T*>(delta), static_cast<const T*>(sst),
+             static_cast<const T*>(t6), kg, ks, kh, static_cast<long>(pl.HW), rows, pl.C, eps, static_cast<T*>(r_out),
+             static_cast<T*>(h_out));
+  return last_launch();
+}
+
+// out[rows][n] = act(a[rows][K] w^T + b), rows ldo elements apart
+template <typename T>
+int linear_any(const Plan& pl, const void* a, long rows, int K, const void* w, const void* b, int n, void* out,
+               long ldo, int act, int* status, cudaStream_t st) {
+  const void* ws1[1] = {w};
+  const void* bs1[1] = {b};
+  if (pl.bf16) return tc_linear(a, rows, K, ws1, bs1, 1, n, out, ldo, act, status, st);
+  return simt_linear(a, rows, K, ws1, bs1, 1, n, out, static_cast<int>(ldo), act, st);
+}
+
+template <typename T>
+int run_dit(const void* x, const void* y, const void* t6, const DitPlan& dp, const edit_dit_block_weights* w,
+            uint8_t* ws, void* out, cudaStream_t st) {
+  const Plan& pa = dp.pa;
+  const int C = pa.C;
+  const long tok = static_cast<long>(pa.B) * pa.HW, trow = static_cast<long>(pa.B) * dp.NT;
+  int* status = reinterpret_cast<int*>(ws + pa.status);
+  // h1 = LN(x) (1 + scale_a) + shift_a
+  EDIT_TRY(dit_residual_ln<T>(pa, x, nullptr, w->sst, t6, -1, 1, 0, w->ln_eps, nullptr, ws + dp.h1, st));
+  // a = EDiT(h1) o_w^T + o_b (resets the status block)
+  edit_attn_weights aw = w->attn;
+  aw.workspace = ws;
+  aw.workspace_bytes = dp.pa.total;
+  const edit_attn_variant var = dit_attn_variant(w);
+  EDIT_TRY(run_edit<T>(ws + dp.h1, pa, &aw, ws, ws + dp.att, st, side_of(w->side_stream, w->side_events), &var));
+  // x1 = x + gate_a a
+  EDIT_TRY(dit_residual_ln<T>(pa, x, ws + dp.att, w->sst, t6, 2, 0, 0, w->ln_eps, ws + dp.x1, nullptr, st));
+  // cross-attention over the caption tokens
+  EDIT_TRY(linear_any<T>(pa, ws + dp.x1, tok, C, w->cq_w, w->cq_b, C, ws + dp.q, C, ACT_NONE, status, st));
+  {
+    const void* kvw[2] = {w->ck_w, w->cv_w};
+    const void* kvb[2] = {w->ck_b, w->cv_b};
+    if (pa.bf16)
+      EDIT_TRY(tc_linear(y, trow, C, kvw, kvb, 2, C, ws + dp.kv, 2L * C, 0, status, st));
+    else
+      EDIT_TRY(simt_linear(y, trow, C, kvw, kvb, 2, C, ws + dp.kv, 2 * C, 0, st));
+  }
+  const T* kv = reinterpret_cast<const T*>(ws + dp.kv);
+  if (pa.bf16) {
+    EDIT_TRY(vt_ones(kv + C, 2L * C, dp.NT, dp.nkp, pa, ws + dp.vt, st));
+    SdpaTcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.w1 = 1.f;
+    p.out = ws + dp.att;
+    p.ldo = C;
+    p.status = status;
+    const SdpaSet cap = {kv, 2L * C, dp.NT, ws + dp.vt, dp.nkp};
+    EDIT_TRY(sdpa_tc(ws + dp.q, C, static_cast<int>(pa.HW), cap, nullptr, p, pa, st));
+  } else {
+    SdpaParams a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = ws + dp.q;
+    a.ldq = C;
+    a.k1 = kv;
+    a.v1 = kv + C;
+    a.ld1 = 2L * C;
+    a.n1 = dp.NT;
+    a.out = ws + dp.att;
+    a.ldo = C;
+    a.Nq = static_cast<int>(pa.HW);
+    a.heads = pa.heads;
+    a.d = pa.d;
+    a.w1 = 1.f;
+    EDIT_TRY(sdpa_simt(a, pa.B, st));
+  }
+  EDIT_TRY(linear_any<T>(pa, ws + dp.att, tok, C, w->co_w, w->co_b, C, ws + dp.c, C, ACT_NONE, status, st));
+  // x2 = x1 + c; h2 = LN(x2) (1 + scale_f) + shift_f
+  EDIT_TRY(dit_residual_ln<T>(pa, ws + dp.x1, ws + dp.c, w->sst, t6, -1, 4, 3, w->ln_eps, ws + dp.x2, ws + dp.h2, st));
+  // MLP: f = GELU(h2 fc1^T + b1), m = f fc2^T + b2; out = x2 + gate_f m
+  EDIT_TRY(linear_any<T>(pa, ws + dp.h2, tok, C, w->fc1_w, w->fc1_b, dp.hidden, ws + dp.f, dp.hidden, ACT_GELU,
+                         status, st));
+  EDIT_TRY(linear_any<T>(pa, ws + dp.f, tok, dp.hidden, w->fc2_w, w->fc2_b, C, ws + dp.m, C, ACT_NONE, status, st));
+  return dit_residual_ln<T>(pa, ws + dp.x2, ws + dp.m, w->sst, t6, 5, 0, 0, w->ln_eps, out, nullptr, st);
+}
+
+int dit_checks(const void* x, const void* y, const void* t6, const void* out, const edit_dit_block_weights* w,
+               const DitPlan& dp) {
+  if (!x || !y || !t6 || !out || !w->workspace) return EDIT_ERR_NULL;
+  const edit_attn_variant var = dit_attn_variant(w);
+  EDIT_TRY_CHECK(check_weights(&w->attn, dp.pa, &var));
+  const void* blk[] = {w->sst, w->cq_w, w->cq_b, w->ck_w, w->ck_b, w->cv_w, w->cv_b, w->co_w, w->co_b,
+                       w->fc1_w, w->fc1_b, w->fc2_w, w->fc2_b};
+  EDIT_TRY_CHECK(check_ptrs(blk, 13));
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(t6, 16) || !aligned(out, 16)) return EDIT_ERR_ALIGN;
+  if (!aligned(w->workspace, 256)) return EDIT_ERR_ALIGN;
+  if (w->workspace_bytes < dp.total) return EDIT_ERR_WORKSPACE;
+  return check_side(w->side_stream, w->side_events);
+}
+
 int common_checks(const void* x, const void* out, const edit_attn_weights* w, void* ws, size_t ws_bytes,
                   const Plan& pl, const edit_attn_variant* var = nullptr) {
   if (!x || !out || !ws) return EDIT_ERR_NULL;
@@ -1830,6 +1987,23 @@ int edit_attn_band_finish(const void* x_ext, int W, int C, int heads, const edit
   if (!aligned(records, 256) || !aligned(out, 16)) return EDIT_ERR_ALIGN;
   return run_band_finish(x_ext, bp, w, static_cast<uint8_t*>(w->workspace), static_cast<const uint8_t*>(records),
                          nrecords, out, static_cast<cudaStream_t>(stream));
+}
+
+size_t edit_dit_block_workspace_bytes(int B, int H, int W, int N_T, int C, int heads,
+                                      const edit_dit_block_weights* w) {
+  DitPlan dp;
+  return make_dit_plan(B, H, W, N_T, C, heads, w, dp) == EDIT_OK ? dp.total : 0;
+}
+
+int edit_dit_block_forward(const void* x, const void* y, const void* t6, int B, int H, int W, int N_T, int C,
+                           int heads, const edit_dit_block_weights* w, void* out, void* stream) {
+  DitPlan dp;
+  EDIT_TRY(make_dit_plan(B, H, W, N_T, C, heads, w, dp));
+  EDIT_TRY(dit_checks(x, y, t6, out, w, dp));
+  uint8_t* ws = static_cast<uint8_t*>(w->workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dp.pa.bf16 ? run_dit<__nv_bfloat16>(x, y, t6, dp, w, ws, out, st)
+                    : run_dit<float>(x, y, t6, dp, w, ws, out, st);
 }
 
 const char* edit_status_string(int status) {

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(256) simt_gemm_f32(SimtGemmParams p) {
       const int s = n / p.n_split;
       float v = acc[i][j];
       if (p.bias[s]) v += p.bias[s][n - s * p.n_split];
-      if (p.relu) v = fmaxf(v, 0.f);
+      if (p.relu) v = act_apply(v, p.relu);
       p.out[static_cast<long>(m) * p.ldo + n] = v;
     }
   }
@@ -1118,6 +1118,102 @@ __global__ void __launch_bounds__(128) sdpa_blend_kernel(SdpaParams p) {
       v = p.n2 > 0 ? eta * res[c] + (1.f - eta) * res2[c] : (1.f - eta) * res[c];
     if (p.blend_in) v = fmaf(p.exact ? eta : p.w0, to_f32(op[c]), v);
     op[c] = from_f32<T>(v);
+  }
+}
+
+// ============================================================ DiT block
+// 8 consecutive elements (16-byte aligned) to / from fp32 registers.
+__device__ __forceinline__ void load8(const float* p, float (&o)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&o)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void store8(float* p, const float (&o)[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(o[4], o[5], o[6], o[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&o)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(o[0], o[1]);
+  u.y = pack_bf16x2(o[2], o[3]);
+  u.z = pack_bf16x2(o[4], o[5]);
+  u.w = pack_bf16x2(o[6], o[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// Residual stream and LayerNorm modulation of the DiT block around the
+// attention, one warp per token row (C % 8 == 0, C <= 2048):
+//   r = base + g * delta (delta optional; g = sst[kg] + t6[b][kg], or 1 when kg < 0)
+//   h = LN(r) (1 + sst[ks] + t6[b][ks]) + sst[kh] + t6[b][kh]   (LN without affine)
+// r is written to r_out and h to h_out when they are non-NULL. Row stats in
+// fp32 (two passes over the row held in registers).
+template <typename T>
+__global__ void __launch_bounds__(256) dit_residual_ln_kernel(const T* __restrict__ base, const T* __restrict__ delta,
+                                                              const T* __restrict__ sst, const T* __restrict__ t6,
+                                                              int kg, int ks, int kh, long rows_per_img, long rows,
+                                                              int C, float eps, T* __restrict__ r_out,
+                                                              T* __restrict__ h_out) {
+  pdl_wait();
+  constexpr int MAXV = 8;  // 8-element vectors per lane: C <= 32 * 8 * 8
+  const int lane = threadIdx.x & 31;
+  const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= rows) return;
+  const long b = row / rows_per_img;
+  const int nv = C / 8;
+  const T* mb = t6 + b * 6L * C;
+  float v[MAXV][8];
+  float s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      const long off = row * C + 8L * vi;
+      load8(base + off, v[k]);
+      if (delta) {
+        float dl[8], g[8], gt[8];
+        load8(delta + off, dl);
+        if (kg >= 0) {
+          load8(sst + kg * C + 8 * vi, g);
+          load8(mb + kg * C + 8 * vi, gt);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[k][i] = fmaf(kg >= 0 ? g[i] + gt[i] : 1.f, dl[i], v[k][i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s1 += v[k][i];
+      if (r_out) store8(r_out + off, v[k]);
+    }
+  }
+  if (!h_out) return;
+  const float mean = warp_sum(s1) / static_cast<float>(C);
+  float s2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k)
+    if (lane + 32 * k < nv)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s2 = fmaf(v[k][i] - mean, v[k][i] - mean, s2);
+  const float rstd = rsqrtf(warp_sum(s2) / static_cast<float>(C) + eps);
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      float sc[8], sct[8], sh[8], sht[8], o[8];
+      load8(sst + ks * C + 8 * vi, sc);
+      load8(mb + ks * C + 8 * vi, sct);
+      load8(sst + kh * C + 8 * vi, sh);
+      load8(mb + kh * C + 8 * vi, sht);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = fmaf((v[k][i] - mean) * rstd, 1.f + sc[i] + sct[i], sh[i] + sht[i]);
+      store8(h_out + row * C + 8L * vi, o);
+    }
   }
 }
 

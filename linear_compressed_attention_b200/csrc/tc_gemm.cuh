@@ -76,7 +76,7 @@ struct TcGemmParams {
   long ldo;
   const void* bias[3];
   int bias_f32;
-  int relu;
+  int relu;  // epilogue activation: ACT_NONE, ACT_RELU or ACT_GELU
   int* status;
   float* den_out;  // EPI_APPLY: when set, den + eps per row and head, [img][R][heads] fp32
 };
@@ -259,7 +259,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileC
         }
         if (p.relu) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = fmaxf(v[16 * g16 + i], 0.f);
+          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = act_apply(v[16 * g16 + i], p.relu);
         }
         if (valid && n < p.N) store_bf16x16(orow + col, *reinterpret_cast<const float(*)[16]>(&v[16 * g16]), 16);
       }
@@ -585,7 +585,7 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
     }
     if (p.relu) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+      for (int i = 0; i < 64; ++i) v[i] = act_apply(v[i], p.relu);
     }
     // stage this warp's 32 rows x 64 columns (bf16) in 128B-swizzled order
     if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
@@ -864,7 +864,7 @@ __device__ __forceinline__ void ring_store64(const TcGemmParams& p, const TileCo
   }
   if (p.relu) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+    for (int i = 0; i < 64; ++i) v[i] = act_apply(v[i], p.relu);
   }
   if (lane == 0) bulk_wait_read<STGBUF - 1>();  // the store that last read this buffer is done
   __syncwarp();
