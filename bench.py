@@ -273,10 +273,11 @@ def run_reference(args, cfg):
 def side_measurements(dev, peaks, steps=50, warmup=5):
     """The metric's other sizes (4K and 16K tokens, and the 262K-token 8192 px
     layer), the ablation table's query/key/value processing variants (and the
-    output Linear) at 65K tokens, and the MM-EDiT hybrid at 1024 px (4096 image
-    + 333 prompt tokens): median step time with L2 flushed between steps,
-    tokens/s and the fraction of each layer's roofline. The MM line adds its
-    stage times (prompt projections, the two softmax passes)."""
+    output Linear) at 65K tokens, the DiT block around the attention at 4K and
+    65K tokens, and the MM-EDiT hybrid at 1024 px (4096 image + 333 prompt
+    tokens): median step time with L2 flushed between steps, tokens/s and the
+    fraction of each layer's roofline. The MM line adds its stage times
+    (prompt projections, the two softmax passes)."""
     import torch
 
     from linear_compressed_attention_b200 import binding as bd
@@ -357,6 +358,31 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
                 "note": "stage events of one step (no overlap with the neighbouring kernels)"}
         del layer, x, out
     res["variants_px4096"] = var
+    # the DiT block around the attention (300 caption tokens, MLP 4C) at 4K and 64K tokens
+    blocks = {}
+    for name in ("px1024", "px4096"):
+        cfg = dict(WORKLOADS[name])
+        blk = dict(n_cap=300, hidden=4 * cfg["C"])
+        d = make_inputs(**cfg, dit_block=blk)
+        B, H, W, C, heads = cfg["B"], cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+        block = bd.DitBlock(d, B, H, W, blk["n_cap"], C, heads, cfg["dtype"], device=dev)
+        xb = torch.from_numpy(d["x"]).to(dev, block.tdtype)
+        yb = torch.from_numpy(d["y"]).to(dev, block.tdtype)
+        tb = torch.from_numpy(d["t6"]).to(dev, block.tdtype)
+        ob = torch.empty_like(xb)
+        ms, _ = timed(lambda: block.forward(xb, yb, tb, ob))
+        assert block.status() == 0
+        n, nt, hid = B * H * W, B * blk["n_cap"], blk["hidden"]
+        fl = (layer_flops(cfg)["total"] + 2.0 * n * C * C          # EDiT attention + its output Linear
+              + 2.0 * n * C * C + 4.0 * nt * C * C + 4.0 * n * blk["n_cap"] * C + 2.0 * n * C * C  # cross-attention
+              + 4.0 * n * C * hid)                                  # MLP
+        by = min_bytes(cfg) + 2 * (2 * nt * C + 4 * C * C + 2 * C * hid + 6 * C)
+        roof = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+        blocks[name] = {"tokens_per_s": n / (ms / 1e3), "ms_per_step": ms, "gflop": fl / 1e9,
+                        "layer_roofline_frac": roof * 1e3 / ms,
+                        "workload": f"{name} grid, 300 caption tokens, MLP hidden {hid}"}
+        del block, xb, yb, tb, ob
+    res["dit_block"] = blocks
     cfg = dict(WORKLOADS["mm1024"])
     d = make_inputs(**cfg)
     nt = cfg["n_txt"]
