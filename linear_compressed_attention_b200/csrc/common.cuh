@@ -61,10 +61,14 @@ __device__ __forceinline__ void record_wait_site(int* status, int site, int tile
 
 // Epilogue activation of the GEMMs: 0 none, 1 ReLU, 2 GELU in its tanh form
 // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+// (The callers test the mode once per tile, outside their unrolled loops.)
 enum { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2 };
+__device__ __forceinline__ float gelu_tanh(float v) {
+  return 0.5f * v * (1.f + tanhf(0.7978845608028654f * fmaf(0.044715f * v * v, v, v)));
+}
 __device__ __forceinline__ float act_apply(float v, int mode) {
   if (mode == ACT_RELU) return fmaxf(v, 0.f);
-  if (mode == ACT_GELU) return 0.5f * v * (1.f + tanhf(0.7978845608028654f * fmaf(0.044715f * v * v, v, v)));
+  if (mode == ACT_GELU) return gelu_tanh(v);
   return v;
 }
 

@@ -257,9 +257,12 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const TileC
             v[16 * g16 + i] += p.bias_f32 ? reinterpret_cast<const float*>(bias)[j0 + i]
                                           : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
         }
-        if (p.relu) {
+        if (p.relu == ACT_RELU) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = act_apply(v[16 * g16 + i], p.relu);
+          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = fmaxf(v[16 * g16 + i], 0.f);
+        } else if (p.relu == ACT_GELU) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[16 * g16 + i] = gelu_tanh(v[16 * g16 + i]);
         }
         if (valid && n < p.N) store_bf16x16(orow + col, *reinterpret_cast<const float(*)[16]>(&v[16 * g16]), 16);
       }
@@ -583,9 +586,12 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
                                         : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[j0 + i]);
       }
     }
-    if (p.relu) {
+    if (p.relu == ACT_RELU) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = act_apply(v[i], p.relu);
+      for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+    } else if (p.relu == ACT_GELU) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
     }
     // stage this warp's 32 rows x 64 columns (bf16) in 128B-swizzled order
     if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
@@ -862,9 +868,12 @@ __device__ __forceinline__ void ring_store64(const TcGemmParams& p, const TileCo
     v[4 * i + 2] += t.z;
     v[4 * i + 3] += t.w;
   }
-  if (p.relu) {
+  if (p.relu == ACT_RELU) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = act_apply(v[i], p.relu);
+    for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+  } else if (p.relu == ACT_GELU) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
   }
   if (lane == 0) bulk_wait_read<STGBUF - 1>();  // the store that last read this buffer is done
   __syncwarp();
