@@ -762,8 +762,12 @@ int kv_state_tc(const Plan& pl, uint8_t* ws, cudaStream_t st) {
   const __nv_bfloat16* VTx = reinterpret_cast<const __nv_bfloat16*>(ws + pl.VTx);
   TcGemmParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!map_a(&p.a0, KT, pl.Mp, static_cast<long>(pl.B) * pl.C, 1, pl.Mp, static_cast<long>(pl.B) * pl.C * pl.Mp))
-    return EDIT_ERR_CUDA;
+  {  // KT as [img * heads][d][Mp], box 64 x 128 x 1: the M = 128 tile reads one head's d rows, the rest is zero
+    cuuint64_t dims[3] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.d, (cuuint64_t)pl.B * pl.heads};
+    cuuint64_t st2[2] = {(cuuint64_t)pl.Mp * 2, (cuuint64_t)pl.d * pl.Mp * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    if (!encode(&p.a0, 3, KT, dims, st2, box)) return EDIT_ERR_CUDA;
+  }
   p.a1 = p.a0;
   if (!map_b(&p.b0, VTx, pl.Mp, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.Mp, pl.NP)) return EDIT_ERR_CUDA;
   p.b1 = p.b2 = p.bk = p.b0;
@@ -778,7 +782,6 @@ int kv_state_tc(const Plan& pl, uint8_t* ws, cudaStream_t st) {
   p.N = pl.NP;
   p.d = pl.d;
   p.heads = pl.heads;
-  p.kv_rows_per_img = pl.C;
   p.kv_part = reinterpret_cast<float*>(ws + pl.kvpart);
   p.status = reinterpret_cast<int*>(ws + pl.status);
   return gemm_kvstate(p, pl.NP, st);
@@ -1240,7 +1243,12 @@ int run_apply(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, void* out
   if (pl.bf16) {
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
-    if (!map_a(&p.a0, ws + pl.Q, pl.C, pl.HW, pl.B, pl.C, pl.HW * pl.C)) return EDIT_ERR_CUDA;
+    {  // Q as [img][row][head][d], box 64 x 1 x 128 x 1: a head's d columns (the rest reads as zero)
+      cuuint64_t dims[4] = {(cuuint64_t)pl.d, (cuuint64_t)pl.heads, (cuuint64_t)pl.HW, (cuuint64_t)pl.B};
+      cuuint64_t st3[3] = {(cuuint64_t)pl.d * 2, (cuuint64_t)pl.C * 2, (cuuint64_t)pl.HW * pl.C * 2};
+      cuuint32_t box[4] = {64, 1, 128, 1};
+      if (!encode(&p.a0, 4, ws + pl.Q, dims, st3, box)) return EDIT_ERR_CUDA;
+    }
     p.a1 = p.a0;
     if (!map_b(&p.b0, ws + pl.SzT, pl.KP, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.KP, pl.NP))
       return EDIT_ERR_CUDA;

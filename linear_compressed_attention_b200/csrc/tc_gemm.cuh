@@ -59,7 +59,6 @@ struct TcGemmParams {
   // apply / KV-state geometry (EPI_APPLY, EPI_KVSTATE)
   int d, heads;
   float eps;
-  int kv_rows_per_img;  // EPI_KVSTATE: A rows per image (= C)
   int kb_per_chunk, num_chunks;
   // tap-reuse conv: pair tiles [split_first, split_first + split_count) run as
   // two half items over the input-channel blocks, writing fp32 partials to
@@ -334,15 +333,17 @@ __device__ __forceinline__ void load_stage(const TcGemmParams& p, const TileCoor
       tma2_load_4d(&p.a0, bar_addr, dA, c0, tc.w0 + kw - 1, tc.h0 + kh - 1, tc.img);
     else
       tma_load_4d(&p.a0, bar, dA, c0, tc.w0 + kw - 1, tc.h0 + kh - 1, tc.img);
+  } else if (EPI == EPI_APPLY) {
+    // Q as [img][row][head][d]: the head's d columns only (columns past d read as zero)
+    tma_load_4d(&p.a0, bar, dA, kb * 64, tc.n_tile, tc.r0, tc.img);
   } else {
     const CUtensorMap* am = &p.a0;
     int x = kb * 64, y = tc.r0, z = tc.img;
-    if (EPI == EPI_APPLY) {
-      x = tc.n_tile * p.d + kb * 64;
-    } else if (EPI == EPI_KVSTATE) {
+    if (EPI == EPI_KVSTATE) {
+      // KT as [img * heads][d][Mp]: the head's d channel rows only (rows past d read as zero)
       x = (tc.kb0 + kb) * 64;
-      y = tc.img * p.kv_rows_per_img + tc.n_tile * p.d;
-      z = 0;
+      y = 0;
+      z = tc.img * p.heads + tc.n_tile;
     } else if (kb >= p.kb_split) {
       am = &p.a1;
       x = (kb - p.kb_split) * 64;
