@@ -249,7 +249,8 @@ EDIT_API const char *edit_status_string(int status);
  *   K, V [B,M,C] token-major (fp32 calls and MM-EDiT calls only);
  *   KT [B][C][Mp], VTx [B][heads][NP][Mp] channel-major (bf16 only): token
  *     t = i*Wop + j of the compressed grid padded to Wop columns (padding
- *     tokens are 0); row d of each VTx head block is all ones;
+ *     tokens are 0); rows d.. of each VTx head block are not written (the
+ *     KV-state kernel forms the [V | 1] operand's ones row itself);
  *   gn_stats fp32 [B][gn_groups][2] (mean, rstd);
  *   Sz fp32 [B][heads][d][d+1] (S_h with z_h as the last column).
  * Mp, Wop, NP give the padded sizes (Mp = M, Wop = ceil(W/2), NP = 0 for fp32). */

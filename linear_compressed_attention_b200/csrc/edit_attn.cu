@@ -485,6 +485,20 @@ int launch_tc(const TcGemmParams& p, cudaStream_t st) {
   return last_launch();
 }
 
+// Co-resident 2-CTA clusters of a pair kernel on the current device (queried
+// once per kernel instantiation and device, thread-safe).
+template <typename Kern>
+int pair_clusters(Kern kern, cudaLaunchConfig_t cfg, std::atomic<int>* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 // Pair kernel: clusters of 2 CTAs on neighbouring SMs, one persistent pair per
 // co-resident cluster slot.
 template <int BN, int NSPLIT, int STAGES, int EPI>
@@ -508,13 +522,8 @@ int launch_pair(const TcGemmParams& p, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  static int max_clusters = 0;  // per instantiation; same device model throughout a process
-  if (max_clusters == 0) {
-    cfg.gridDim = dim3(2 * 74, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
-    max_clusters = n;
-  }
+  static std::atomic<int> cluster_cache[kMaxDevices];  // per instantiation and device
+  const int max_clusters = pair_clusters(kern, cfg, cluster_cache);
   const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return EDIT_ERR_CUDA;
@@ -543,13 +552,8 @@ int launch_ring(const TcGemmParams& p, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
-    cfg.gridDim = dim3(2 * 74, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
-    max_clusters = n;
-  }
+  static std::atomic<int> cluster_cache[kMaxDevices];  // per instantiation and device
+  const int max_clusters = pair_clusters(kern, cfg, cluster_cache);
   const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return EDIT_ERR_CUDA;
@@ -578,13 +582,8 @@ int launch_conv_pair(TcGemmParams& p, cudaStream_t st, bool* split_out) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
-    cfg.gridDim = dim3(2 * 74, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
-    max_clusters = n;
-  }
+  static std::atomic<int> cluster_cache[kMaxDevices];  // per instantiation and device
+  const int max_clusters = pair_clusters(kern, cfg, cluster_cache);
   // Last partial wave at most half full: split its tiles over the input-channel
   // blocks into two half items each, so every pair has work in that wave.
   const int T = p.num_tiles;
@@ -769,7 +768,13 @@ int kv_state_tc(const Plan& pl, uint8_t* ws, cudaStream_t st) {
     if (!encode(&p.a0, 3, KT, dims, st2, box)) return EDIT_ERR_CUDA;
   }
   p.a1 = p.a0;
-  if (!map_b(&p.b0, VTx, pl.Mp, static_cast<long>(pl.B) * pl.heads * pl.NP, pl.Mp, pl.NP)) return EDIT_ERR_CUDA;
+  {  // VTx as [img * heads][d][Mp] (rows NP apart), box 64 x NP x 1: rows d.. read as zero, and the
+     // kernel sets row d to ones (the [V | 1] operand: z as column d of the product)
+    cuuint64_t dims[3] = {(cuuint64_t)pl.Mp, (cuuint64_t)pl.d, (cuuint64_t)pl.B * pl.heads};
+    cuuint64_t st2[2] = {(cuuint64_t)pl.Mp * 2, (cuuint64_t)pl.NP * pl.Mp * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)pl.NP, 1};
+    if (!encode(&p.b0, 3, VTx, dims, st2, box)) return EDIT_ERR_CUDA;
+  }
   p.b1 = p.b2 = p.bk = p.b0;
   p.num_kb = (pl.Mp + 63) / 64;
   p.kb_split = p.num_kb;
@@ -822,10 +827,6 @@ int dwconv_tc(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, int rows,
              pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
              static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
              static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, row_shift, reinterpret_cast<int*>(ws + pl.status));
-  EDIT_TRY(last_launch());
-  const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
-  launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d, pl.NP,
-             pl.Mp);
   return last_launch();
 }
 
@@ -869,12 +870,8 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
                  dim3(256), 0, st, reinterpret_cast<const __nv_bfloat16*>(ws + pl.KVp), static_cast<long>(pl.HW),
                  pl.C, pl.d, pl.heads, pl.NP, static_cast<long>(pl.Mp), KT, VTx);
       EDIT_TRY(last_launch());
-      const long padn = static_cast<long>(pl.B) * pl.heads * (pl.NP - pl.d) * (pl.Mp / 8);
-      launch_pdl(vtx_pad_rows_kernel, dim3(grid_for(padn, 256)), dim3(256), 0, st, VTx, pl.B * pl.heads, pl.d,
-                 pl.NP, pl.Mp);
-      EDIT_TRY(last_launch());
     } else {
-      EDIT_TRY(dwconv_tc(pl, w, ws, pl.H, 0, st));  // (writes the VTx padding rows too)
+      EDIT_TRY(dwconv_tc(pl, w, ws, pl.H, 0, st));
     }
     stage_mark(2, st);
     EDIT_TRY(kv_state_tc(pl, ws, st));

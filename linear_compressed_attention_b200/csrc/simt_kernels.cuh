@@ -742,26 +742,6 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   }
 }
 
-// Rows d..NP-1 of each head's block of VTx: a row of ones (so the tensor-core
-// KV state also yields z = sum_j K_j) followed by zero rows; 16-byte stores
-// (Mp % 8 == 0).
-__global__ void vtx_pad_rows_kernel(__nv_bfloat16* __restrict__ VTx, int BH, int d, int NP, int Mp) {
-  pdl_wait();
-  const int vpr = Mp / 8;                   // vectors per row
-  const int rows = NP - d;
-  const long total = static_cast<long>(BH) * rows * vpr;
-  const __nv_bfloat162 one2 = __floats2bfloat162_rn(1.f, 1.f);
-  const uint32_t onew = *reinterpret_cast<const uint32_t*>(&one2);
-  for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long ri = e / vpr;
-    const int v = static_cast<int>(e - ri * vpr);
-    const long bh = ri / rows;
-    const int r = d + static_cast<int>(ri - bh * rows);
-    const uint32_t w = r == d ? onew : 0u;
-    *reinterpret_cast<uint4*>(VTx + (bh * NP + r) * Mp + 8L * v) = make_uint4(w, w, w, w);
-  }
-}
 
 // Keys and values without the Spatial Compressor (ablation variants whose
 // keys and values keep all N tokens): the token-major rows kvp [B][N][2C]

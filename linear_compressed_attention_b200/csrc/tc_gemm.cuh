@@ -78,6 +78,7 @@ struct TcGemmParams {
   int relu;  // epilogue activation: ACT_NONE, ACT_RELU or ACT_GELU
   int* status;
   float* den_out;  // EPI_APPLY: when set, den + eps per row and head, [img][R][heads] fp32
+
 };
 
 template <int BN, int NSPLIT, int STAGES, int STG = 0>
@@ -358,9 +359,15 @@ __device__ __forceinline__ void load_stage(const TcGemmParams& p, const TileCoor
   for (int s = 0; s < NSPLIT; ++s) {
     const CUtensorMap* bm;
     int x, y;
-    if (EPI == EPI_APPLY || EPI == EPI_KVSTATE) {
+    if (EPI == EPI_KVSTATE) {
+      // VTx as [img * heads][d][Mp]: the head's d value rows; the rest of the box
+      // reads as zero and the MMA issuer writes the ones row
+      uint8_t* d = dB + s * BROWS * 128;
+      tma_load_3d(&p.b0, bar, d, (tc.kb0 + kb) * 64, 0, tc.img * p.heads + tc.n_tile);
+      continue;
+    } else if (EPI == EPI_APPLY) {
       bm = &p.b0;
-      x = (EPI == EPI_KVSTATE ? tc.kb0 + kb : kb) * 64;
+      x = kb * 64;
       y = (tc.img * p.heads + tc.n_tile) * BN + s * NCHUNK;
     } else {
       const int n = tc.n_tile * BN + s * NCHUNK + (PAIR ? rank * BROWS : 0);
@@ -469,6 +476,13 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             break;
           }
           tc_fence_after();
+          if (EPI == EPI_KVSTATE) {  // [V | 1]: row d of the B tile (64 keys, 128 bytes) is all ones
+            const uint32_t one2 = 0x3F803F80u;  // two bf16 1.0
+            uint4* r1 = reinterpret_cast<uint4*>(sB + stage * Cfg::B_BYTES + p.d * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) r1[j] = make_uint4(one2, one2, one2, one2);
+            fence_proxy_async_smem();
+          }
           const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
 #pragma unroll
