@@ -830,7 +830,7 @@ __global__ void conv_fixup_kernel(const float* __restrict__ part, int split_firs
 
 // Split-K per-tap conv: U = bias + sum of the ksplit k-part partials of each
 // pair tile, summed in part order (deterministic), bf16 out. part is
-// [(tile * ksplit + part) * 2 + rank][128][Cr] fp32; row r of CTA tile m_tile
+// [(tile * ksplit + part) * 2 + rank][Cr / 4][128][4] fp32; row r of CTA tile m_tile
 // is pixel (h0 + r / TW, w0 + r % TW) of a TH x TW tile (TH * TW = 128).
 __global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksplit, int pair_tiles, int tiles_w,
                                          int tiles_h, int TH, int TW, int H, int W, int Cr,
@@ -839,12 +839,15 @@ __global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksp
   pdl_wait();
   const int cv = Cr / 4;
   const long total = static_cast<long>(pair_tiles) * 2 * 128 * cv;
+  // partials are [item][rank][Cr / 4][128 rows][4]: the row varies fastest, so a
+  // warp reads 512 contiguous bytes of each part
   for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(e % cv) * 4;
-    const long rr = e / cv;  // (tile, rank, row)
-    const int row = static_cast<int>(rr & 127), rank = static_cast<int>((rr >> 7) & 1);
-    const int pt = static_cast<int>(rr >> 8);
+    const int row = static_cast<int>(e & 127);
+    const long rq = e >> 7;  // (tile, rank, column quad)
+    const int c4 = static_cast<int>(rq % cv), c = c4 * 4;
+    const int rank = static_cast<int>((rq / cv) & 1);
+    const int pt = static_cast<int>(rq / cv >> 1);
     const int m_tile = 2 * pt + rank;
     if (m_tile >= num_m_tiles) continue;
     const int per_img = tiles_h * tiles_w;
@@ -855,7 +858,7 @@ __global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksp
                            __bfloat162float(bias[c + 3]));
     for (int k = 0; k < ksplit; ++k) {
       const float4 q = *reinterpret_cast<const float4*>(
-          part + (((static_cast<long>(pt) * ksplit + k) * 2 + rank) * 128 + row) * Cr + c);
+          part + ((((static_cast<long>(pt) * ksplit + k) * 2 + rank) * cv + c4) * 128 + row) * 4);
       a.x += q.x;
       a.y += q.y;
       a.z += q.z;

@@ -67,7 +67,7 @@ struct TcGemmParams {
   float* fix_part;
   // per-tap conv (pair kernel, EPI_CONV): ksplit > 1 splits every tile's
   // k-blocks into ksplit parts; item it = tile it / ksplit, part it % ksplit,
-  // whose fp32 partial goes to fix_part [item][rank][128][N]
+  // whose fp32 partial goes to fix_part [item][rank][N / 4][128][4]
   int ksplit;
   float* kv_part;       // EPI_KVSTATE: [img][heads][num_chunks][d][d+1]
   // epilogue
@@ -776,8 +776,10 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
       tc_fence_after();
       const TileCoord tc = decode_pair_tile<EPI>(p, pt, rank);
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      if (EPI == EPI_CONV && p.ksplit > 1) {  // fp32 partial of this k-part, row q * 32 + lane
-        float* prow = p.fix_part + ((static_cast<long>(pt) * 2 + rank) * 128 + q * 32 + lane) * p.N;
+      if (EPI == EPI_CONV && p.ksplit > 1) {
+        // fp32 partial of this k-part, column-quad major ([N / 4][128 rows][4]): a warp's
+        // 16-byte stores of one column quad land on 512 contiguous bytes
+        float* pbase = p.fix_part + (static_cast<long>(pt) * 2 + rank) * 128 * p.N + (q * 32 + lane) * 4;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 64) {
           float v[64];
@@ -785,7 +787,7 @@ __global__ void __launch_bounds__(pair_threads(NSPLIT), 1) tc_gemm_pair_kernel(c
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (c0 + 4 * j < BN)
-              *reinterpret_cast<float4*>(prow + c0 + 4 * j) =
+              *reinterpret_cast<float4*>(pbase + static_cast<long>(c0 / 4 + j) * 512) =
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
       } else {
