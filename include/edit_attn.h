@@ -383,16 +383,19 @@ EDIT_API uint64_t edit_attn_kernel_launches(void);
  *
  * Every device-side wait in the library is bounded and reports
  * EDIT_ERR_TIMEOUT through the workspace status word instead of hanging. This
- * hook lets a test make one such wait run out on purpose, without a fault:
- * while armed (gn_extra_arrivals > 0), the fused GroupNorm kernel of the
- * calling thread's bf16 forward calls waits at its grid barrier for
+ * hook lets a test make one such wait run out on purpose, without a fault.
+ * Larger bf16 layers normalise through a cooperative GroupNorm kernel
+ * (statistics, grid barrier, apply in one grid); small ones, whose conv runs
+ * split over k, take the statistics from column sums the conv's fixup writes.
+ * While the drill is armed (gn_extra_arrivals > 0), the calling thread's bf16
+ * forward calls always run the cooperative kernel, which waits at its barrier for
  * gn_extra_arrivals more blocks than it launched, and gives up after
  * limit_ns nanoseconds (1e3 .. 2e9). Each block then records EDIT_ERR_TIMEOUT
  * and the first one the wait site (word 1 = 30, word 3 = arrivals seen,
  * word 4 = arrivals expected, word 5 = blocks launched) and returns without
  * applying the normalisation; later kernels of the call still run, and their
- * results are invalid. The GPU context stays usable. The fused kernel runs
- * for bf16 layers with at least 8 channels per group and c_red <= 4096.
+ * results are invalid. The GPU context stays usable. The cooperative kernel
+ * runs for bf16 layers with at least 8 channels per group and c_red <= 4096.
  * (0, 0) disarms it. Returns EDIT_ERR_SHAPE for arguments out of range. */
 EDIT_API int edit_attn_set_wait_drill(int gn_extra_arrivals, uint64_t limit_ns);
 

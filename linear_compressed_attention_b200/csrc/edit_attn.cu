@@ -168,6 +168,7 @@ struct Plan {
   int es;  // bytes per element of activations/weights
   int TH, TW, tiles_h, tiles_w;
   int gn_P;       // GroupNorm partials per image
+  int gn_slots = 0;  // bf16: GroupNorm column-sum slots per image (4 per conv tile, 32 rows each)
   int conv_pair_tiles = 0, conv_ksplit = 1;  // per-tap conv: pair tiles, k-parts per tile
   int gn_chunk;   // bf16: tokens per GroupNorm partial
   int kv_chunks;  // KV-state partials per (image, head)
@@ -185,7 +186,7 @@ struct Plan {
   bool oproj = false;    // output Linear after the attention
   // workspace offsets (bytes)
   size_t status, U, Gb, gnpart, gnstats, gnss, W1t, Wqw1, bfold, Q, KVp, K, V, KT, VTx, kvpart, Sz, SzT, QKVt,
-      fixpart, VTi, VTp, den, Y, total;
+      fixpart, VTi, VTp, den, Y, gncol, total;
 };
 
 int next_pow2(int v) {
@@ -347,6 +348,12 @@ int make_plan(int B, int H, int W, int C, int heads, int NT, const edit_attn_wei
   if (pl.bf16 && pl.TW < 128 && pl.conv_ksplit > 1)  // per-tap conv split over k: one fp32 partial per item
     pl.fixpart = take(static_cast<size_t>(pl.conv_pair_tiles) * pl.conv_ksplit * 2 * 128 * pl.Cr * 4);
   pl.Y = pl.oproj ? take(tok * C * es) : 0;  // attention output before the output Linear
+  // GroupNorm column sums of U per 32-row slot of each conv tile, written by
+  // the per-tap conv (bf16, W < 128): [B][gn_slots][Cr][2] fp32. The tap-reuse
+  // conv (W >= 128) keeps a single TMEM accumulator, so work added to its
+  // epilogue is not hidden; its layers take the cooperative GroupNorm.
+  pl.gn_slots = (pl.bf16 && pl.any_cf && pl.TW < 128) ? pl.tiles_h * pl.tiles_w * 4 : 0;
+  pl.gncol = take(static_cast<size_t>(B) * pl.gn_slots * pl.Cr * 2 * 4);
   // the key ConvFusion shares the query's ConvFusion buffers, so it stays serial
   pl.fork = pl.bf16 && pl.k_proc != EDIT_PROC_CF && static_cast<long>(B) * pl.HW <= kForkMaxTokens;
   pl.total = off;
@@ -464,6 +471,16 @@ int last_launch() {
   const cudaError_t e = g_launch_err;
   g_launch_err = cudaSuccess;
   return e == cudaSuccess ? EDIT_OK : EDIT_ERR_CUDA;
+}
+
+// Grid of gn_apply_leaky_bf16x8: B images (y), at most one wave of 8 blocks
+// per SM over the images (x), each thread visiting several tokens.
+dim3 gn_apply_grid(long HW, int B, int per_block) {
+  long gx = (HW + per_block - 1) / per_block;
+  long cap = static_cast<long>(num_sms()) * 8 / B;
+  if (cap < 1) cap = 1;
+  if (gx > cap) gx = cap;
+  return dim3(static_cast<unsigned>(gx < 1 ? 1 : gx), static_cast<unsigned>(B), 1);
 }
 
 int grid_for(long total, int threads) {
@@ -915,7 +932,11 @@ int run_kv(const void* x, const Plan& pl, const edit_attn_weights* w, const edit
 
 // Step 5 on the tensor cores: U = Conv3x3(X) + b for the plan's image grid
 // (stage event 5 after the conv kernel when `marks`).
-int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, cudaStream_t st, bool marks) {
+// gn_col: when set, the conv epilogue (whole tiles) and the fixup (tiles split
+// over k) also write the GroupNorm column sums of U per 32-row slot of every
+// tile, [B][gn_slots][Cr][2].
+int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, cudaStream_t st, bool marks,
+               float* gn_col) {
   int* status = reinterpret_cast<int*>(ws + pl.status);
   const int C = pl.C, Cr = pl.Cr;
   TcGemmParams p;
@@ -942,17 +963,19 @@ int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, 
   if (!map_out_grid(&p.out_map, ws + pl.U, pl.B, pl.H, pl.W, Cr, pl.TW)) return EDIT_ERR_CUDA;
   p.bias[0] = cf.cf3_b;
   p.status = status;
+  p.gn_col = gn_col;
   if (pl.TW == 128) {  // tap reuse: one input patch per channel block feeds all 9 taps
     if (!map_patch(&p.a1, x, pl.B, pl.H, pl.W, C)) return EDIT_ERR_CUDA;
     p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
     bool split = false;
     EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
     if (marks) stage_mark(5, st);
-    if (split) {
+    if (split) {  // the last wave's split tiles: two halves over the channel blocks
       const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
-      launch_pdl(conv_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, 
-          p.fix_part, p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.H, pl.W, Cr,
-          static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, 2,
+                 p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
+                 static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U),
+                 gn_col);
       EDIT_TRY(last_launch());
     }
   } else {
@@ -960,11 +983,12 @@ int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, 
     p.fix_part = reinterpret_cast<float*>(ws + pl.fixpart);
     EDIT_TRY(gemm_conv(p, Cr, st));
     if (marks) stage_mark(5, st);
-    if (pl.conv_ksplit > 1) {
+    if (pl.conv_ksplit > 1) {  // every tile split over k
       const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
-      launch_pdl(conv_splitk_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit,
+      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit, 0,
                  pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
-                 static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U));
+                 static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U),
+                 gn_col);
       EDIT_TRY(last_launch());
     }
   }
@@ -1123,18 +1147,35 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
   // 5. U = Conv3x3(X) (+ GroupNorm partials)
   float* gnpart = reinterpret_cast<float*>(ws + pl.gnpart);
   bool gn_fused = false;
+  // GroupNorm partials: (P, cols) of the layout gn_finalize_kernel reads
+  int gn_parts = pl.gn_P, gn_cols = 1;
+  float* gn_src = gnpart;
   if (pl.bf16) {
-    EDIT_TRY(conv3x3_tc(x, pl, cf, ws, st, marks));
-    if ((Cr / pl.G) >= 8 && Cr / 8 <= 512) {
-      // 6. G = LeakyReLU(GN(U)) in one cooperative grid: statistics, grid barrier, apply
+    // The per-tap conv (W < 128) writes the GroupNorm column sums of U per
+    // 32-row slot of each of its tiles, so no pass over U forms the statistics
+    // and no grid-wide barrier is needed; wider layers run the cooperative
+    // GroupNorm (statistics, bounded grid barrier, apply in one grid). With the
+    // wait drill armed the cooperative kernel always runs: its barrier is the
+    // wait the drill drives out.
+    const bool colsum = pl.gn_slots > 0 && g_drill_extra <= 0;
+    EDIT_TRY(conv3x3_tc(x, pl, cf, ws, st, marks, colsum ? reinterpret_cast<float*>(ws + pl.gncol) : nullptr));
+    if (!colsum && (Cr / pl.G) >= 8 && Cr / 8 <= 512) {
+      // 6. G = LeakyReLU(GN(U)) in one cooperative grid
       const int r = launch_gn_fused(pl, cf, gn_eps, slope, barrier_off, ws, st);
       if (r != EDIT_OK && r != EDIT_ERR_UNSUPPORTED) return r;
       gn_fused = r == EDIT_OK;
     }
     if (!gn_fused) {
-      launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st, 
-          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P, gnpart);
-      EDIT_TRY(last_launch());
+      if (!colsum) {
+        launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pl.gn_P, pl.B)), dim3(256), 0, st,
+                   reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), static_cast<int>(pl.HW), Cr, pl.G, pl.gn_P,
+                   gnpart);
+        EDIT_TRY(last_launch());
+      } else {
+        gn_parts = pl.gn_slots;
+        gn_cols = Cr / pl.G;
+        gn_src = reinterpret_cast<float*>(ws + pl.gncol);
+      }
     }
   } else {
     SimtGemmParams p;
@@ -1162,7 +1203,9 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
   }
   // 6. G = LeakyReLU(GN(U))
   if (!gn_fused) {
-    launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(256), 0, st, gnpart, pl.gn_P, pl.G, Cr, pl.HW * (Cr / pl.G), gn_eps,
+    launch_pdl(gn_finalize_kernel<T>, dim3(dim3(pl.G, pl.B)), dim3(gn_cols > 1 ? 1024 : 256), 0, st, gn_src, gn_parts,
+               gn_cols, pl.G, Cr,
+               pl.HW * (Cr / pl.G), gn_eps,
                                                 static_cast<const T*>(cf.gamma), static_cast<const T*>(cf.beta),
                                                 reinterpret_cast<float*>(ws + pl.gnstats),
                                                 reinterpret_cast<float*>(ws + pl.gnss));
@@ -1171,9 +1214,9 @@ int run_convfusion(const void* x, const Plan& pl, const CfWeights& cf, float gn_
       const int nvec = Cr / 8;
       const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
       const int threads = per_block * nvec;
-      launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(threads), 0, st, 
-          reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW, Cr,
-          slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb), tok);
+      launch_pdl(gn_apply_leaky_bf16x8, gn_apply_grid(pl.HW, pl.B, per_block), dim3(threads), 0, st,
+                 reinterpret_cast<const __nv_bfloat16*>(ws + pl.U), reinterpret_cast<const float*>(ws + pl.gnss), pl.HW,
+                 Cr, slope, reinterpret_cast<__nv_bfloat16*>(ws + pl.Gb));
     } else {
       const long total = tok * Cr;
       launch_pdl(gn_apply_leaky_kernel<float>, dim3(grid_for(total, 256)), dim3(256), 0, st, 
@@ -1653,7 +1696,7 @@ int run_band_partials(const void* x, const BandPlan& bp, const edit_attn_weights
              reinterpret_cast<float*>(rec + bp.sz_off));
   EDIT_TRY(last_launch());
   // U of the band with its halo rows (the halo rows' own outputs are not used)
-  EDIT_TRY(conv3x3_tc(x, pe, query_cf(w), ws, st, false));
+  EDIT_TRY(conv3x3_tc(x, pe, query_cf(w), ws, st, false, nullptr));
   const __nv_bfloat16* Ub = reinterpret_cast<const __nv_bfloat16*>(ws + pe.U) + static_cast<long>(bp.top) * W * Cr;
   float* gnpart = reinterpret_cast<float*>(ws + pe.gnpart);
   launch_pdl(gn_partial_kernel<__nv_bfloat16>, dim3(dim3(pq.gn_P, 1)), dim3(256), 0, st, Ub,
@@ -1682,10 +1725,10 @@ int run_band_finish(const void* x, const BandPlan& bp, const edit_attn_weights* 
   {
     const int nvec = Cr / 8;
     const int per_block = 256 / nvec > 0 ? 256 / nvec : 1;
-    launch_pdl(gn_apply_leaky_bf16x8, dim3(grid_for(tok, per_block)), dim3(per_block * nvec), 0, st,
+    launch_pdl(gn_apply_leaky_bf16x8, gn_apply_grid(tok, 1, per_block), dim3(per_block * nvec), 0, st,
                reinterpret_cast<const __nv_bfloat16*>(ws + pe.U) + static_cast<long>(bp.top) * W * Cr,
                reinterpret_cast<const float*>(ws + pe.gnss), tok, Cr, w->leaky_slope,
-               reinterpret_cast<__nv_bfloat16*>(ws + pe.Gb), tok);
+               reinterpret_cast<__nv_bfloat16*>(ws + pe.Gb));
     EDIT_TRY(last_launch());
   }
   const CfWeights cf = query_cf(w);

@@ -374,23 +374,26 @@ __global__ void __launch_bounds__(512) gn_fused_bf16_kernel(const __nv_bfloat16*
 // (group, image): thread t sums partials t, t+blockDim, ... in order, then a
 // fixed shared-memory tree (blockDim a power of two).
 template <typename T>
-__device__ void gn_finalize_body(const float* __restrict__ part, int P, int groups, int Cr, long count, float eps,
-                                 const T* __restrict__ gamma, const T* __restrict__ beta, float* __restrict__ stats,
-                                 float* __restrict__ ss, int g, int b, double* r1, double* r2) {
+__device__ void gn_finalize_body(const float* __restrict__ part, int P, int cols, int groups, int Cr, long count,
+                                 float eps, const T* __restrict__ gamma, const T* __restrict__ beta,
+                                 float* __restrict__ stats, float* __restrict__ ss, int g, int b, double* r1,
+                                 double* r2) {
   const int cpg = Cr / groups;
-  const int nt = blockDim.x >= 256 ? 256 : 128;
+  const int nt = blockDim.x;  // a power of two, at most the length of r1 / r2
   double s1 = 0.0, s2 = 0.0;
-  if (threadIdx.x < nt)
-    for (int i = threadIdx.x; i < P; i += nt) {
-      const float2 q = *reinterpret_cast<const float2*>(part + ((static_cast<long>(b) * P + i) * groups + g) * 2);
-      s1 += q.x;
-      s2 += q.y;
-    }
-  __syncthreads();
-  if (threadIdx.x < nt) {
-    r1[threadIdx.x] = s1;
-    r2[threadIdx.x] = s2;
+  // element e = (partial i, column j) of group g, e = i * cols + j: thread t
+  // sums e = t, t + nt, ... in that order
+  const int n = P * cols;
+#pragma unroll 8
+  for (int e = threadIdx.x; e < n; e += nt) {
+    const int i = e / cols, j = e - i * cols;
+    const float2 q = *reinterpret_cast<const float2*>(part + (((static_cast<long>(b) * P + i) * groups + g) * cols + j) * 2);
+    s1 += q.x;
+    s2 += q.y;
   }
+  __syncthreads();
+  r1[threadIdx.x] = s1;
+  r2[threadIdx.x] = s2;
   __syncthreads();
   for (int w = nt / 2; w > 0; w >>= 1) {
     if (threadIdx.x < w) {
@@ -415,14 +418,18 @@ __device__ void gn_finalize_body(const float* __restrict__ part, int P, int grou
   __syncthreads();
 }
 
+// Block (g, b): group g of image b from part [b][P][groups][cols][2] (sum,
+// sum of squares), summed in a fixed order in fp64: cols = 1 for the token-chunk
+// partials of gn_partial_kernel, cols = Cr / groups for the column sums the
+// conv writes per 32-row slot of each tile.
 template <typename T>
-__global__ void __launch_bounds__(256) gn_finalize_kernel(const float* __restrict__ part, int P, int groups, int Cr,
-                                                          long count, float eps, const T* __restrict__ gamma,
+__global__ void __launch_bounds__(1024) gn_finalize_kernel(const float* __restrict__ part, int P, int cols, int groups,
+                                                          int Cr, long count, float eps, const T* __restrict__ gamma,
                                                           const T* __restrict__ beta, float* __restrict__ stats,
                                                           float* __restrict__ ss) {
   pdl_wait();
-  __shared__ double r1[256], r2[256];
-  gn_finalize_body<T>(part, P, groups, Cr, count, eps, gamma, beta, stats, ss, blockIdx.x, blockIdx.y, r1, r2);
+  __shared__ double r1[1024], r2[1024];
+  gn_finalize_body<T>(part, P, cols, groups, Cr, count, eps, gamma, beta, stats, ss, blockIdx.x, blockIdx.y, r1, r2);
 }
 
 // G = LeakyReLU(scale * U + shift), elementwise over [B][HW][Cr].
@@ -441,36 +448,32 @@ __global__ void gn_apply_leaky_kernel(const T* __restrict__ U, const float* __re
   }
 }
 
-// bf16 variant, 8 channels per thread with 16-byte loads/stores (Cr % 8 == 0).
-// Thread t always handles channel vector t % (Cr/8) (blockDim a multiple of
-// Cr/8), so its scale/shift stay in registers across the tokens it visits.
+// bf16 variant, 8 channels per thread with 16-byte loads/stores (Cr % 8 == 0),
+// image blockIdx.y. Thread t always handles channel vector t % (Cr/8) (blockDim
+// a multiple of Cr/8), so its scale/shift stay in registers; it visits tokens
+// blockDim/(Cr/8) * gridDim.x apart, four loads in flight.
 __global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const float* __restrict__ ss, long HW,
-                                      int Cr, float slope, __nv_bfloat16* __restrict__ G, long tokens) {
+                                      int Cr, float slope, __nv_bfloat16* __restrict__ G) {
   pdl_wait();
   const int nvec = Cr / 8;
   const int per_block = blockDim.x / nvec;
   const int v = threadIdx.x % nvec, kt = threadIdx.x / nvec;
   if (kt >= per_block) return;
   const int c = v * 8;
-  long b_cur = -1;
+  const long b = blockIdx.y;
   float sc[8], sh[8];
-  for (long tok = static_cast<long>(blockIdx.x) * per_block + kt; tok < tokens;
-       tok += static_cast<long>(gridDim.x) * per_block) {
-    const long b = tok / HW;
-    if (b != b_cur) {
-      const float4* s4 = reinterpret_cast<const float4*>(ss + (b * Cr + c) * 2);
+  {
+    const float4* s4 = reinterpret_cast<const float4*>(ss + (b * Cr + c) * 2);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 q = s4[j];
-        sc[2 * j] = q.x;
-        sh[2 * j] = q.y;
-        sc[2 * j + 1] = q.z;
-        sh[2 * j + 1] = q.w;
-      }
-      b_cur = b;
+    for (int j = 0; j < 4; ++j) {
+      const float4 q = s4[j];
+      sc[2 * j] = q.x;
+      sh[2 * j] = q.y;
+      sc[2 * j + 1] = q.z;
+      sh[2 * j + 1] = q.w;
     }
-    const long e = tok * Cr + c;
-    const uint4 raw = *reinterpret_cast<const uint4*>(U + e);
+  }
+  auto apply = [&](const uint4& raw) {
     const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(&raw);
     float o[8];
 #pragma unroll
@@ -483,8 +486,20 @@ __global__ void gn_apply_leaky_bf16x8(const __nv_bfloat16* __restrict__ U, const
     out.y = pack_bf16x2(o[2], o[3]);
     out.z = pack_bf16x2(o[4], o[5]);
     out.w = pack_bf16x2(o[6], o[7]);
-    *reinterpret_cast<uint4*>(G + e) = out;
+    return out;
+  };
+  const __nv_bfloat16* ub = U + b * HW * Cr + c;
+  __nv_bfloat16* gb = G + b * HW * Cr + c;
+  const long step = static_cast<long>(gridDim.x) * per_block;
+  long tok = static_cast<long>(blockIdx.x) * per_block + kt;
+  for (; tok + 3 * step < HW; tok += 4 * step) {
+    uint4 r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r[j] = *reinterpret_cast<const uint4*>(ub + (tok + j * step) * Cr);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(gb + (tok + j * step) * Cr) = apply(r[j]);
   }
+  for (; tok < HW; tok += step) *reinterpret_cast<uint4*>(gb + tok * Cr) = apply(*reinterpret_cast<const uint4*>(ub + tok * Cr));
 }
 
 // ============================================================ weight folding
@@ -795,65 +810,37 @@ __global__ void __launch_bounds__(256) kv_transpose_kernel(const __nv_bfloat16* 
   }
 }
 
-// Sum of the two fp32 halves of each split conv tile plus the bias -> U (bf16),
-// 4 channels per thread (Cr % 4 == 0). Tile t of the pair grid: CTA `rank`
-// holds 128-pixel tile 2t + rank (one image-row segment of 128 pixels).
-// part [split][half][rank][128][Cr].
-__global__ void conv_fixup_kernel(const float* __restrict__ part, int split_first, int split_count, int tiles_w,
-                                  int tiles_h, int H, int W, int Cr, const __nv_bfloat16* __restrict__ bias,
-                                  int num_m_tiles, __nv_bfloat16* __restrict__ U) {
+// U of the conv tiles that ran split over k: bias + the ksplit fp32 partials
+// of each tile, summed in part order (deterministic), bf16 out. Pair tiles
+// [pt_first, pt_first + pt_count) are split; part is [(local pair tile * ksplit
+// + k) * 2 + rank][Cr / 4][128][4], and row r of CTA tile m_tile = 2 * pair tile
+// + rank is pixel (h0 + r / TW, w0 + r % TW) of a TH x TW tile (TH * TW = 128).
+// Thread e takes row e % 128 of one column quad, so a warp reads 512 contiguous
+// bytes of each part and holds rows 32j .. 32j + 31 of one quad: when gn_col is
+// set, the warp also writes that quad's GroupNorm column sums of the 32 rows
+// (bf16 values; pixels outside the image add nothing), in the layout the conv
+// epilogue writes for the tiles it finishes itself.
+__global__ void conv_parts_fixup_kernel(const float* __restrict__ part, int ksplit, int pt_first, int pt_count,
+                                        int tiles_w, int tiles_h, int TH, int TW, int H, int W, int Cr,
+                                        const __nv_bfloat16* __restrict__ bias, int num_m_tiles,
+                                        __nv_bfloat16* __restrict__ U, float* __restrict__ gn_col) {
   pdl_wait();
   const int cv = Cr / 4;
-  const int total = split_count * 2 * 128 * cv;
-  const int per = 2 * 128 * Cr;  // one split tile, one half
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int c = (e % cv) * 4;
-    const int rr = e / cv;  // (split, rank, row)
-    const int row = rr & 127;
-    const int rank = (rr >> 7) & 1;
-    const int sp = rr >> 8;
-    const int m_tile = 2 * (split_first + sp) + rank;
-    if (m_tile >= num_m_tiles) continue;
-    const int per_img = tiles_h * tiles_w;
-    const int img = m_tile / per_img, u = m_tile - img * per_img;
-    const int hh = u / tiles_w, ww = (u % tiles_w) * 128 + row;
-    if (hh >= H || ww >= W) continue;
-    const int off = (rank * 128 + row) * Cr + c;
-    const float4 a = *reinterpret_cast<const float4*>(part + (2 * sp) * per + off);
-    const float4 b = *reinterpret_cast<const float4*>(part + (2 * sp + 1) * per + off);
-    __nv_bfloat16* dst = U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c;
-    const uint2 o = make_uint2(pack_bf16x2(a.x + b.x + __bfloat162float(bias[c]), a.y + b.y + __bfloat162float(bias[c + 1])),
-                               pack_bf16x2(a.z + b.z + __bfloat162float(bias[c + 2]), a.w + b.w + __bfloat162float(bias[c + 3])));
-    *reinterpret_cast<uint2*>(dst) = o;
-  }
-}
-
-// Split-K per-tap conv: U = bias + sum of the ksplit k-part partials of each
-// pair tile, summed in part order (deterministic), bf16 out. part is
-// [(tile * ksplit + part) * 2 + rank][Cr / 4][128][4] fp32; row r of CTA tile m_tile
-// is pixel (h0 + r / TW, w0 + r % TW) of a TH x TW tile (TH * TW = 128).
-__global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksplit, int pair_tiles, int tiles_w,
-                                         int tiles_h, int TH, int TW, int H, int W, int Cr,
-                                         const __nv_bfloat16* __restrict__ bias, int num_m_tiles,
-                                         __nv_bfloat16* __restrict__ U) {
-  pdl_wait();
-  const int cv = Cr / 4;
-  const long total = static_cast<long>(pair_tiles) * 2 * 128 * cv;
-  // partials are [item][rank][Cr / 4][128 rows][4]: the row varies fastest, so a
-  // warp reads 512 contiguous bytes of each part
+  const long total = static_cast<long>(pt_count) * 2 * 128 * cv;
+  const int per_img = tiles_h * tiles_w;
+  // (total and the grid stride are multiples of 32: a warp never straddles a quad)
   for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long>(gridDim.x) * blockDim.x) {
     const int row = static_cast<int>(e & 127);
-    const long rq = e >> 7;  // (tile, rank, column quad)
+    const long rq = e >> 7;  // (local pair tile, rank, column quad)
     const int c4 = static_cast<int>(rq % cv), c = c4 * 4;
     const int rank = static_cast<int>((rq / cv) & 1);
     const int pt = static_cast<int>(rq / cv >> 1);
-    const int m_tile = 2 * pt + rank;
-    if (m_tile >= num_m_tiles) continue;
-    const int per_img = tiles_h * tiles_w;
+    const int m_tile = 2 * (pt_first + pt) + rank;
+    if (m_tile >= num_m_tiles) continue;  // the pair grid's empty tile (whole warp)
     const int img = m_tile / per_img, u = m_tile - img * per_img;
     const int hh = (u / tiles_w) * TH + row / TW, ww = (u % tiles_w) * TW + row % TW;
-    if (hh >= H || ww >= W) continue;
+    const bool inside = hh < H && ww < W;
     float4 a = make_float4(__bfloat162float(bias[c]), __bfloat162float(bias[c + 1]), __bfloat162float(bias[c + 2]),
                            __bfloat162float(bias[c + 3]));
     for (int k = 0; k < ksplit; ++k) {
@@ -864,8 +851,25 @@ __global__ void conv_splitk_fixup_kernel(const float* __restrict__ part, int ksp
       a.z += q.z;
       a.w += q.w;
     }
-    __nv_bfloat16* dst = U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    const uint2 o = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    if (inside) *reinterpret_cast<uint2*>(U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c) = o;
+    if (gn_col != nullptr) {
+      float v[4] = {__uint_as_float(o.x << 16), __uint_as_float(o.x & 0xffff0000u), __uint_as_float(o.y << 16),
+                    __uint_as_float(o.y & 0xffff0000u)};
+      float r[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        r[2 * j] = inside ? v[j] : 0.f;
+        r[2 * j + 1] = inside ? v[j] * v[j] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) r[j] = warp_sum(r[j]);
+      if ((threadIdx.x & 31) == 0) {
+        float* dst = gn_col + ((static_cast<long>(img) * per_img * 4 + u * 4 + row / 32) * Cr + c) * 2;
+        *reinterpret_cast<float4*>(dst) = make_float4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(r[4], r[5], r[6], r[7]);
+      }
+    }
   }
 }
 

@@ -236,9 +236,10 @@ __global__ void __launch_bounds__(conv_threads(NSPLIT), 1) tc_conv_pair_kernel(c
       const uint32_t t_row = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
       if (ci.half < 0) {
         epilogue_tile_staged<BN, EPI_CONV>(p, tc, t_row, q, lane, stg, sbuf);
-      } else {  // fp32 partial of this half, row q*32 + lane
-        float* prow = p.fix_part + ((((static_cast<long>(ci.pt - p.split_first) * 2 + ci.half) * 2 + rank) * 128) +
-                                    q * 32 + lane) * p.N;
+      } else {  // fp32 partial of this half, column-quad major ([N / 4][128 rows][4]):
+                // a warp's 16-byte stores of one column quad land on 512 contiguous bytes
+        float* pbase = p.fix_part + ((static_cast<long>(ci.pt - p.split_first) * 2 + ci.half) * 2 + rank) * 128 * p.N +
+                       (q * 32 + lane) * 4;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 64) {
           float v[64];
@@ -246,7 +247,8 @@ __global__ void __launch_bounds__(conv_threads(NSPLIT), 1) tc_conv_pair_kernel(c
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (c0 + 4 * j < BN)
-              *reinterpret_cast<float4*>(prow + c0 + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              *reinterpret_cast<float4*>(pbase + static_cast<long>(c0 / 4 + j) * 512) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
       }
       tc_fence_before();

@@ -62,7 +62,8 @@ struct TcGemmParams {
   int kb_per_chunk, num_chunks;
   // tap-reuse conv: pair tiles [split_first, split_first + split_count) run as
   // two half items over the input-channel blocks, writing fp32 partials to
-  // fix_part [split tile][half][rank][128][N] (summed with the bias afterwards)
+  // fix_part [(split tile * 2 + half) * 2 + rank][N / 4][128][4] (summed with
+  // the bias afterwards)
   int split_first, split_count;
   float* fix_part;
   // per-tap conv (pair kernel, EPI_CONV): ksplit > 1 splits every tile's
@@ -78,6 +79,11 @@ struct TcGemmParams {
   int relu;  // epilogue activation: ACT_NONE, ACT_RELU or ACT_GELU
   int* status;
   float* den_out;  // EPI_APPLY: when set, den + eps per row and head, [img][R][heads] fp32
+  // EPI_CONV: when set, the GroupNorm column sums of the stored U (bf16 values):
+  // gn_col[img][tile * 4 + row / 32][N][2] = (sum, sum of squares) over rows
+  // 32 (row / 32) .. + 31 of the image's 128-pixel tile `tile` (pixels outside
+  // the image add nothing). Tiles split over k get theirs from the fixup kernel.
+  float* gn_col;
 
 };
 
@@ -583,6 +589,12 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
                                                      int q, int lane, uint8_t* stg, int& sbuf) {
   const bool real = tc.m_tile < p.num_m_tiles;
   const int n0 = tc.n_tile * BN;
+  // EPI_CONV with gn_col: bit i = row q*32 + i of the tile is a pixel of the image
+  uint32_t inside = 0;
+  if (EPI == EPI_CONV && p.gn_col != nullptr) {
+    const int r = q * 32 + lane;
+    inside = __ballot_sync(0xffffffffu, real && tc.h0 + r / p.TW < p.H && tc.w0 + r % p.TW < p.W);
+  }
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 64) {
     float v[64];
@@ -624,6 +636,30 @@ __device__ __forceinline__ void epilogue_tile_staged(const TcGemmParams& p, cons
     }
     fence_proxy_async_smem();
     __syncwarp();
+    if (EPI == EPI_CONV && p.gn_col != nullptr && real) {
+      // column sums of the staged bf16 values over this warp's 32 rows: lane l
+      // takes columns c0 + 2l, c0 + 2l + 1 (one 32-bit word per row; the 128-byte
+      // swizzle puts the eight lanes of a 16-byte chunk on distinct banks)
+      float s0 = 0.f, q0 = 0.f, s1 = 0.f, q1 = 0.f;
+      const uint8_t* colp = buf + ((lane & 3) << 2);
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        if ((inside >> i) & 1u) {
+          const uint32_t wd = *reinterpret_cast<const uint32_t*>(colp + i * 128 + (((lane >> 2) ^ (i & 7)) << 4));
+          const float a = __uint_as_float(wd << 16), b = __uint_as_float(wd & 0xffff0000u);
+          s0 += a;
+          q0 = fmaf(a, a, q0);
+          s1 += b;
+          q1 = fmaf(b, b, q1);
+        }
+      }
+      const int col = n0 + c0 + 2 * lane;
+      if (col < p.N) {
+        const int per_img = p.tiles_h * p.tiles_w;
+        const long slot = (static_cast<long>(tc.img) * per_img + (tc.m_tile - tc.img * per_img)) * 4 + q;
+        *reinterpret_cast<float4*>(p.gn_col + (slot * p.N + col) * 2) = make_float4(s0, q0, s1, q1);
+      }
+    }
     if (lane == 0 && real) {
       if (EPI == EPI_CONV) {
         const int r0w = q * 32;

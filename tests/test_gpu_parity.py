@@ -87,7 +87,8 @@ SMALL_BF16 = [
     dict(B=3, H=12, W=20, C=384, c_red=256, gn_groups=8, heads=6),     # d = 64, 3 images
     dict(B=1, H=8, W=8, C=1536, c_red=384, gn_groups=32, heads=24),    # MM widths
     dict(B=1, H=160, W=128, C=128, c_red=64, gn_groups=8, heads=2),    # conv tiles > one wave: last wave split
-    dict(B=2, H=8, W=12, C=128, c_red=64, gn_groups=16, heads=2),      # 4 channels per GN group: unfused GN path
+    dict(B=2, H=8, W=12, C=128, c_red=64, gn_groups=16, heads=2),      # 4 channels per GN group
+    dict(B=4, H=80, W=60, C=128, c_red=64, gn_groups=8, heads=2),      # per-tap conv over > one wave (no k split), ragged tiles
     dict(B=2, H=48, W=50, C=1152, c_red=288, gn_groups=32, heads=16),  # d = 72, apply CTAs cross the image boundary
 ]
 
