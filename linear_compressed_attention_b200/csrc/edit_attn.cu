@@ -638,8 +638,9 @@ int conv_chunk(int cr) { return (cr == 288) ? 144 : (cr == 384) ? 192 : cr; }
 // Linear GEMMs on CTA pairs: 256 x 256 pair tiles (one N = 256 MMA per
 // k-step), or 256 x 384 tiles (three N = 128 chunks over a TMEM slot ring),
 // which need 17% fewer operand bytes per MMA cycle. 384 is taken where the
-// weight sources split on 192-row boundaries and its tile waves are not
-// longer: per column of a wave the 384 kernel takes ~0.85 of the time.
+// weight sources split on 192-row boundaries and it needs no more waves of
+// pair tiles than 256 (measured: with equal waves, e.g. the K|V GEMM of 2 x
+// 1,024 tokens, the 384 ring still finishes first, 24.8 -> 22.7 us).
 constexpr int kPairBN = 256;
 int ceil_div(long a, long b);
 int linear_bn(long rows, int N, int n_split, const void* const* biases, int nbias) {
@@ -650,7 +651,7 @@ int linear_bn(long rows, int N, int n_split, const void* const* biases, int nbia
   const long pairs = num_sms() / 2;
   const long w256 = (m_pairs * ceil_div(N, 256) + pairs - 1) / pairs;
   const long w384 = (m_pairs * ceil_div(N, 384) + pairs - 1) / pairs;
-  return w384 * 384 * 85 < w256 * 256 * 100 ? 384 : kPairBN;
+  return w384 <= w256 ? 384 : kPairBN;
 }
 // Weight-map box height (rows per CTA of a pair tile) for tile width bn.
 int linear_box(int bn) { return bn / 2; }
