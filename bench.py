@@ -564,7 +564,8 @@ def run_ours(args, cfg):
         fl = layer_flops(cfg)
         # dominant kernel: the 3x3 conv of the ConvFusion query, else the K|V GEMM
         dominant, dom_kernel, dom_flops = (
-            (DOMINANT, "tc_conv_pair_kernel conv3x3 implicit GEMM", fl["conv3x3"]) if qkv[0] == "cf" else
+            (DOMINANT, ("tc_conv_pair_kernel" if cfg["W"] >= 128 else "tc_gemm_pair_kernel (per-tap)")
+             + " conv3x3 implicit GEMM", fl["conv3x3"]) if qkv[0] == "cf" else
             ("kv_linear", "tc_linear_ring_kernel K|V Linear", fl["kv_linear"]))
         dom_ms = statistics.mean(stage_ms[dominant])
         achieved = dom_flops / (dom_ms / 1e3) / 1e12
