@@ -570,7 +570,7 @@ def run_ours(args, cfg):
         dom_ms = statistics.mean(stage_ms[dominant])
         achieved = dom_flops / (dom_ms / 1e3) / 1e12
         traffic = (TRAFFIC["bytes_per_launch"] if TRAFFIC["src_sha"] == kernel_src_sha() and not is_variant
-                   and args.workload == "px4096" else None)
+                   and args.workload == "px4096" and not args.lib else None)
         ms_per_step = total_ms / args.steps
         vflops = variant_flops(cfg, qkv, proj)
         vbytes = min_bytes(cfg) + (2 * C * C * 2 if proj else 0)
@@ -581,7 +581,8 @@ def run_ours(args, cfg):
             "vs_baseline": None, "dtype": "bf16" if cfg["dtype"] == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": args.workload_desc, "global_batch": world * B, "seq_len": N,
                        "parallelism": f"independent images, {world} rank(s)",
-                       "l2": "flushed between steps (256 MB write, outside the timed events); input 151 MB > L2"},
+                       "l2": "flushed between steps (256 MB write, outside the timed events); input "
+                             f"{B * N * cfg['C'] * 2 / 1e6:.0f} MB", **({"lib": args.lib} if args.lib else {})},
             "roofline": {"bound": "tensor", "kernel": dom_kernel, "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
@@ -634,12 +635,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the side measurements (other sizes, variants, MM-EDiT)")
+    ap.add_argument("--lib", default=None,
+                    help="time this build of the library instead of the in-tree one (e.g. an older commit's, "
+                         "for a same-box A/B); the line then records it under config.lib")
     ap.add_argument("--variant", default="cf-sc-sc",
                     help="query-key-value processing of the timed layer, each cf | sc | none (ablation table), "
                          "optionally +out_linear; default the EDiT layer cf-sc-sc")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.lib:
+        if not os.path.exists(args.lib):
+            raise SystemExit(f"--lib {args.lib}: no such file")
+        from linear_compressed_attention_b200 import binding as bd
+        bd.LIB_PATH = os.path.abspath(args.lib)
     cfg = dict(WORKLOADS[args.workload])
     if cfg.get("n_txt"):
         raise SystemExit("bench.py times the EDiT layer workloads; MM-EDiT is covered by the tests")
