@@ -40,7 +40,7 @@ DOMINANT = "conv3x3"   # largest FLOP share of the layer (40%)
 # the dominant kernel, from the ncu capture summarised in
 # profiles/conv3x3_px4096.md; reported only while the kernel's sources are the
 # ones that capture measured (hash of tc_conv.cuh + tc_gemm.cuh + common.cuh).
-TRAFFIC = {"src_sha": "d3f6defd9a529003", "bytes_per_launch": 160921088 + 25559296}
+TRAFFIC = {"src_sha": "a0406f4948f6e4ae", "bytes_per_launch": 159911168 + 25748992}
 
 
 def kernel_src_sha():
