@@ -841,7 +841,13 @@ int dwconv_tc(const Plan& pl, const edit_attn_weights* w, uint8_t* ws, int rows,
         !encode(&mp.vtok, 4, ws + pl.V, d_t, s_t, b_t, SWZ_NONE))
       return EDIT_ERR_CUDA;
   }
-  launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), 0, st, mp, rows,
+  // The token-major staging block (MM-EDiT) is dynamic shared memory: without
+  // it 7 blocks fit per SM instead of 6 (64K tokens: 84 -> 79 us). A layer
+  // whose K/V branch runs beside the query branch keeps 6, leaving that
+  // branch its share of the SMs (2 x 1K tokens: 0.088 ms with 6, 0.090 with 7).
+  const size_t tok_bytes = (tokmajor || pl.fork) ? 32 * 64 * 2 : 0;
+  launch_pdl(dwconv_s2_tma_kernel, dim3(dim3(pl.Wop / 32, pl.B * (2 * pl.C / 64), pl.Ho)), dim3(256), tok_bytes, st,
+             mp, rows,
              pl.W, pl.C, pl.d, pl.heads, pl.Wop, static_cast<const __nv_bfloat16*>(w->kdw_w),
              static_cast<const __nv_bfloat16*>(w->kdw_b), static_cast<const __nv_bfloat16*>(w->vdw_w),
              static_cast<const __nv_bfloat16*>(w->vdw_b), tokmajor, row_shift, reinterpret_cast<int*>(ws + pl.status));
@@ -972,8 +978,8 @@ int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, 
     EDIT_TRY(gemm_conv_reuse(p, Cr, st, &split));
     if (marks) stage_mark(5, st);
     if (split) {  // the last wave's split tiles: two halves over the channel blocks
-      const long total = static_cast<long>(p.split_count) * 2 * 128 * (Cr / 4);
-      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, 2,
+      const long nblk = static_cast<long>(p.split_count) * 2 * 4 * (Cr / 32);  // (tile, 32 rows, 8 quads)
+      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(nblk * 256, 256)), dim3(256), 0, st, p.fix_part, 2,
                  p.split_first, p.split_count, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
                  static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U),
                  gn_col);
@@ -985,8 +991,8 @@ int conv3x3_tc(const void* x, const Plan& pl, const CfWeights& cf, uint8_t* ws, 
     EDIT_TRY(gemm_conv(p, Cr, st));
     if (marks) stage_mark(5, st);
     if (pl.conv_ksplit > 1) {  // every tile split over k
-      const long total = static_cast<long>(pl.conv_pair_tiles) * 2 * 128 * (Cr / 4);
-      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(total, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit, 0,
+      const long nblk = static_cast<long>(pl.conv_pair_tiles) * 2 * 4 * (Cr / 32);  // (tile, 32 rows, 8 quads)
+      launch_pdl(conv_parts_fixup_kernel, dim3(grid_for(nblk * 256, 256)), dim3(256), 0, st, p.fix_part, pl.conv_ksplit, 0,
                  pl.conv_pair_tiles, pl.tiles_w, pl.tiles_h, pl.TH, pl.TW, pl.H, pl.W, Cr,
                  static_cast<const __nv_bfloat16*>(cf.cf3_b), p.num_m_tiles, reinterpret_cast<__nv_bfloat16*>(ws + pl.U),
                  gn_col);

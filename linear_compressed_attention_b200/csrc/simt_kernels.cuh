@@ -671,7 +671,10 @@ __global__ void __launch_bounds__(256) dwconv_s2_tma_kernel(const __grid_constan
   constexpr int JT = 32, CB = 64, PW = 2 * JT + 1;
   __shared__ __align__(1024) __nv_bfloat16 out_s[CB * JT];  // [channel][token], 64-byte swizzled rows
   __shared__ __align__(128) __nv_bfloat16 in_s[3][PW][CB];
-  __shared__ __align__(128) __nv_bfloat16 tok_s[JT][CB];    // [token][channel]
+  // [token][channel] copy for the token-major stores (MM-EDiT only): dynamic
+  // shared memory, so the EDiT layer's blocks do without it (7 per SM, not 6)
+  extern __shared__ __align__(128) __nv_bfloat16 dw_tok[];
+  __nv_bfloat16(*tok_s)[CB] = reinterpret_cast<__nv_bfloat16(*)[CB]>(dw_tok);
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   const int Wo = (W + 1) / 2;
@@ -815,61 +818,78 @@ __global__ void __launch_bounds__(256) kv_transpose_kernel(const __nv_bfloat16* 
 // [pt_first, pt_first + pt_count) are split; part is [(local pair tile * ksplit
 // + k) * 2 + rank][Cr / 4][128][4], and row r of CTA tile m_tile = 2 * pair tile
 // + rank is pixel (h0 + r / TW, w0 + r % TW) of a TH x TW tile (TH * TW = 128).
-// Thread e takes row e % 128 of one column quad, so a warp reads 512 contiguous
-// bytes of each part and holds rows 32j .. 32j + 31 of one quad: when gn_col is
-// set, the warp also writes that quad's GroupNorm column sums of the 32 rows
-// (bf16 values; pixels outside the image add nothing), in the layout the conv
-// epilogue writes for the tiles it finishes itself.
-__global__ void conv_parts_fixup_kernel(const float* __restrict__ part, int ksplit, int pt_first, int pt_count,
-                                        int tiles_w, int tiles_h, int TH, int TW, int H, int W, int Cr,
-                                        const __nv_bfloat16* __restrict__ bias, int num_m_tiles,
-                                        __nv_bfloat16* __restrict__ U, float* __restrict__ gn_col) {
+// A block (256 threads, Cr / 4 a multiple of 8) takes 32 rows x 8 column quads
+// of one tile: warp w sums quad w of the 32 rows (lane = row, so each part is
+// read as 512 contiguous bytes), the results meet in shared memory, and the
+// block writes U as 64 contiguous bytes per row. When gn_col is set, each warp
+// also writes its quad's GroupNorm column sums of the 32 rows (bf16 values;
+// pixels outside the image add nothing), in the layout the conv epilogue
+// writes for the tiles it finishes itself.
+__global__ void __launch_bounds__(256) conv_parts_fixup_kernel(const float* __restrict__ part, int ksplit,
+                                                               int pt_first, int pt_count, int tiles_w, int tiles_h,
+                                                               int TH, int TW, int H, int W, int Cr,
+                                                               const __nv_bfloat16* __restrict__ bias,
+                                                               int num_m_tiles, __nv_bfloat16* __restrict__ U,
+                                                               float* __restrict__ gn_col) {
   pdl_wait();
-  const int cv = Cr / 4;
-  const long total = static_cast<long>(pt_count) * 2 * 128 * cv;
+  __shared__ uint2 tile[32][9];  // [row][quad] of the block's results (padded: fewer bank conflicts)
+  const int cv = Cr / 4, ngroups = cv / 8;
+  const long nblocks = static_cast<long>(pt_count) * 2 * 4 * ngroups;  // (tile, row group, quad group)
   const int per_img = tiles_h * tiles_w;
-  // (total and the grid stride are multiples of 32: a warp never straddles a quad)
-  for (long e = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long>(gridDim.x) * blockDim.x) {
-    const int row = static_cast<int>(e & 127);
-    const long rq = e >> 7;  // (local pair tile, rank, column quad)
-    const int c4 = static_cast<int>(rq % cv), c = c4 * 4;
-    const int rank = static_cast<int>((rq / cv) & 1);
-    const int pt = static_cast<int>(rq / cv >> 1);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (long blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {  // uniform across the block
+    const int qg = static_cast<int>(blk % ngroups);
+    const int rg = static_cast<int>((blk / ngroups) & 3);
+    const int rank = static_cast<int>((blk / ngroups / 4) & 1);
+    const int pt = static_cast<int>(blk / ngroups / 8);
     const int m_tile = 2 * (pt_first + pt) + rank;
-    if (m_tile >= num_m_tiles) continue;  // the pair grid's empty tile (whole warp)
+    if (m_tile >= num_m_tiles) continue;  // the pair grid's empty tile (whole block)
     const int img = m_tile / per_img, u = m_tile - img * per_img;
-    const int hh = (u / tiles_w) * TH + row / TW, ww = (u % tiles_w) * TW + row % TW;
-    const bool inside = hh < H && ww < W;
-    float4 a = make_float4(__bfloat162float(bias[c]), __bfloat162float(bias[c + 1]), __bfloat162float(bias[c + 2]),
-                           __bfloat162float(bias[c + 3]));
-    for (int k = 0; k < ksplit; ++k) {
-      const float4 q = *reinterpret_cast<const float4*>(
-          part + ((((static_cast<long>(pt) * ksplit + k) * 2 + rank) * cv + c4) * 128 + row) * 4);
-      a.x += q.x;
-      a.y += q.y;
-      a.z += q.z;
-      a.w += q.w;
-    }
-    const uint2 o = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-    if (inside) *reinterpret_cast<uint2*>(U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + c) = o;
-    if (gn_col != nullptr) {
-      float v[4] = {__uint_as_float(o.x << 16), __uint_as_float(o.x & 0xffff0000u), __uint_as_float(o.y << 16),
-                    __uint_as_float(o.y & 0xffff0000u)};
-      float r[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        r[2 * j] = inside ? v[j] : 0.f;
-        r[2 * j + 1] = inside ? v[j] * v[j] : 0.f;
+    const int h0 = (u / tiles_w) * TH, w0 = (u % tiles_w) * TW;
+    // ---- warp w: quad qg * 8 + w of rows 32 rg + lane
+    {
+      const int row = rg * 32 + lane, c4 = qg * 8 + w, c = c4 * 4;
+      const bool inside = h0 + row / TW < H && w0 + row % TW < W;
+      float4 a = make_float4(__bfloat162float(bias[c]), __bfloat162float(bias[c + 1]), __bfloat162float(bias[c + 2]),
+                             __bfloat162float(bias[c + 3]));
+      for (int k = 0; k < ksplit; ++k) {
+        const float4 q = *reinterpret_cast<const float4*>(
+            part + ((((static_cast<long>(pt) * ksplit + k) * 2 + rank) * cv + c4) * 128 + row) * 4);
+        a.x += q.x;
+        a.y += q.y;
+        a.z += q.z;
+        a.w += q.w;
       }
+      const uint2 o = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+      tile[lane][w] = o;
+      if (gn_col != nullptr) {
+        float v[4] = {__uint_as_float(o.x << 16), __uint_as_float(o.x & 0xffff0000u), __uint_as_float(o.y << 16),
+                      __uint_as_float(o.y & 0xffff0000u)};
+        float r[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) r[j] = warp_sum(r[j]);
-      if ((threadIdx.x & 31) == 0) {
-        float* dst = gn_col + ((static_cast<long>(img) * per_img * 4 + u * 4 + row / 32) * Cr + c) * 2;
-        *reinterpret_cast<float4*>(dst) = make_float4(r[0], r[1], r[2], r[3]);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(r[4], r[5], r[6], r[7]);
+        for (int j = 0; j < 4; ++j) {
+          r[2 * j] = inside ? v[j] : 0.f;
+          r[2 * j + 1] = inside ? v[j] * v[j] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[j] = warp_sum(r[j]);
+        if (lane == 0) {
+          float* dst = gn_col + ((static_cast<long>(img) * per_img * 4 + u * 4 + rg) * Cr + c) * 2;
+          *reinterpret_cast<float4*>(dst) = make_float4(r[0], r[1], r[2], r[3]);
+          *reinterpret_cast<float4*>(dst + 4) = make_float4(r[4], r[5], r[6], r[7]);
+        }
       }
     }
+    __syncthreads();
+    // ---- thread t: quad t % 8 of row t / 8: eight threads write one row's 64 bytes
+    {
+      const int row = rg * 32 + (threadIdx.x >> 3), q = threadIdx.x & 7;
+      const int hh = h0 + row / TW, ww = w0 + row % TW;
+      if (hh < H && ww < W)
+        *reinterpret_cast<uint2*>(U + ((static_cast<long>(img) * H + hh) * W + ww) * Cr + (qg * 8 + q) * 4) =
+            tile[threadIdx.x >> 3][q];
+    }
+    __syncthreads();
   }
 }
 
