@@ -322,7 +322,10 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
         roof = max(layer_flops(cfg)["total"] / (peaks["bf16_tflops"] * 1e12), min_bytes(cfg) / (peaks["hbm_gbs"] * 1e9))
         res[str(n)] = {"workload": name, "tokens_per_s": n / (ms / 1e3), "ms_per_step": ms,
                        "layer_roofline_frac": roof * 1e3 / ms}
-        del layer, x, out
+        del layer, out
+        if name == "px8192":
+            res["row_bands_px8192"] = band_measurements(d, cfg, x, ms, flush, stream, dev)
+        del x
     # the ablation table's query/key/value processing rows and the output Linear,
     # on the 65,536-token workload
     cfg = dict(WORKLOADS["px4096"], variant_weights=True)
@@ -408,6 +411,63 @@ def side_measurements(dev, peaks, steps=50, warmup=5):
                                     "image_row_softmax": stage_ms[9] if len(stage_ms) > 9 else None,
                                     "prompt_row_softmax": stage_ms[10] if len(stage_ms) > 10 else None}}
     return res
+
+
+def band_measurements(d, cfg, x, full_ms, flush, stream, dev, reps=5):
+    """The row-band split of one 8192 px image (seqpar: halo rows, band partials,
+    records in band order, band finish) for 2 and 8 bands, run one band after
+    another on this one GPU with L2 flushed before each band's kernels, as each
+    rank's own GPU would start. Per band: median device time of its partials and
+    of its finish. A rank of an N-GPU run would take about max(partials) +
+    max(finish) plus the halo exchange and the record all-gather, which one GPU
+    cannot measure; `compute_only_efficiency` = full-image layer time / (N x that
+    compute time)."""
+    import torch
+
+    from linear_compressed_attention_b200 import seqpar
+
+    H, W, C, heads = cfg["H"], cfg["W"], cfg["C"], cfg["heads"]
+    x3 = x[0].reshape(H, W, C)
+    out = {}
+    for world in (2, 8):
+        bands = [seqpar.band_bounds(H, world, r) for r in range(world)]
+        layers = [seqpar.BandLayer(d, H, W, C, heads, device=dev) for _ in bands]
+        exts = []
+        for r0, nr in bands:
+            top, bot = seqpar.halo(H, r0, nr)
+            exts.append(x3[r0 - top:r0 + nr + bot].contiguous())
+        records = torch.empty((world, layers[0].record_bytes), dtype=torch.uint8, device=dev)
+        outs = [torch.empty((nr, W, C), dtype=torch.bfloat16, device=dev) for _, nr in bands]
+        tp = [[] for _ in bands]
+        tf = [[] for _ in bands]
+        for rep in range(reps + 1):  # the first pass warms up
+            for r, ((r0, nr), layer, ext) in enumerate(zip(bands, layers, exts)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer.partials(ext, r0, nr, record=records[r])
+                e1.record(stream)
+                if rep:
+                    tp[r].append((e0, e1))
+            for r, ((r0, nr), layer, ext) in enumerate(zip(bands, layers, exts)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer.finish(ext, records, r0, nr, out=outs[r])
+                e1.record(stream)
+                if rep:
+                    tf[r].append((e0, e1))
+        torch.cuda.synchronize(dev)
+        assert all(layer.status() == 0 for layer in layers)
+        pm = [statistics.median(a.elapsed_time(b) for a, b in t) for t in tp]
+        fm = [statistics.median(a.elapsed_time(b) for a, b in t) for t in tf]
+        band_ms = max(pm) + max(fm)
+        out[str(world)] = {"partials_ms": pm, "finish_ms": fm, "rank_compute_ms": band_ms,
+                           "compute_only_efficiency": full_ms / (world * band_ms)}
+        del layers, exts, records, outs
+    out["note"] = ("one GPU, bands one after another, L2 flushed before each band; halo exchange and record "
+                   "all-gather not included (one GPU per call)")
+    return out
 
 
 def sustained_run(layer, x, out, flush, stream, dev, gpu_id, ms_hint, seconds=2.5):
