@@ -452,8 +452,7 @@ thread_local cudaError_t g_launch_err = cudaSuccess;
 
 template <typename... KArgs, typename... Args>
 void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
@@ -525,8 +524,7 @@ int launch_pair(const TcGemmParams& p, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
     return EDIT_ERR_CUDA;
   if (p.num_tiles < 1) return EDIT_OK;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -555,8 +553,7 @@ int launch_ring(const TcGemmParams& p, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
     return EDIT_ERR_CUDA;
   if (p.num_tiles < 1) return EDIT_OK;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -585,8 +582,7 @@ int launch_conv_pair(TcGemmParams& p, cudaStream_t st, bool* split_out) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
     return EDIT_ERR_CUDA;
   if (p.num_tiles < 1) return EDIT_OK;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -1060,8 +1056,7 @@ int launch_gn_fused(const Plan& pl, const CfWeights& cf, float gn_eps, float slo
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gn_fused_bf16_kernel, 512, smem) != cudaSuccess ||
       per_sm * num_sms() < nblk)
     return EDIT_ERR_UNSUPPORTED;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
