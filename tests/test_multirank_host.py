@@ -53,3 +53,12 @@ def test_single_rank_and_throughput():
     assert bench.rank_config(dict(seed=3, H=8), 0) == dict(seed=3, H=8)
     # 2 ranks x 1 image x 65,536 tokens x 10 steps in 9.4 ms (slowest rank)
     assert abs(bench.job_tokens_per_s(2, 1, 65536, 10, 9.4) - 2 * 65536 * 10 / 0.0094) < 1e-3
+
+
+def test_lib_option_rejects_a_missing_build(monkeypatch):
+    import pytest
+
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--lib", os.path.join(ROOT, "no-such-dir", "libedit_attn.so")])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert "no such file" in str(e.value)
