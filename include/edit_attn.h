@@ -384,9 +384,10 @@ EDIT_API uint64_t edit_attn_kernel_launches(void);
  * Every device-side wait in the library is bounded and reports
  * EDIT_ERR_TIMEOUT through the workspace status word instead of hanging. This
  * hook lets a test make one such wait run out on purpose, without a fault.
- * Larger bf16 layers normalise through a cooperative GroupNorm kernel
- * (statistics, grid barrier, apply in one grid); small ones, whose conv runs
- * split over k, take the statistics from column sums the conv's fixup writes.
+ * bf16 layers at least 128 pixels wide normalise through a cooperative
+ * GroupNorm kernel (statistics, grid barrier, apply in one grid); narrower ones
+ * take the statistics from column sums their conv writes (in its epilogue, or
+ * in the fixup of tiles split over k).
  * While the drill is armed (gn_extra_arrivals > 0), the calling thread's bf16
  * forward calls always run the cooperative kernel, which waits at its barrier for
  * gn_extra_arrivals more blocks than it launched, and gives up after
